@@ -1,0 +1,18 @@
+"""Plain fp64 CPU oracle for paged GQA/MQA decode attention (test infrastructure).
+
+Only the tests, the package's smoke check and the benchmark's CPU-baseline leg
+may import this package.  The product path never calls it.
+"""
+from .paged_attention import (  # noqa: F401
+    bf16_bits_to_f64,
+    f64_to_bf16_bits,
+    kv_head_of,
+    gather_sequence_kv,
+    attend_one_query,
+    paged_decode_attention,
+    paged_decode_attention_rows,
+    kv_append,
+    partial_softmax_piece,
+    merge_partial_pieces,
+    kv_cache_bytes,
+)

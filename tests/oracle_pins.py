@@ -1,0 +1,380 @@
+"""Checks that pin the fp64 oracle to facts outside itself.
+
+Each check raises AssertionError on failure.  They look the oracle's functions
+up through the module object at call time, so tests/test_oracle_mutants.py can
+swap in a deliberately wrong function and confirm some check rejects it.
+
+Sources of the facts (by page and section):
+  * "TensorRT对Multi-Query Attention的专项优化支持": MHA has per-head K_i, V_i; MQA
+    shares one K, V across all query heads (so MQA == MHA whose K/V heads are
+    all copies of the shared one); the KV cache shrinks from h*d_k*s to d_k*s;
+    the cache is paged.
+  * tiny-llm "优化" page: GQA (num_kv_heads != num_heads); KV bytes
+    2 x layers x kv_heads x head_dim x seq_len x 2 B; paged KV by block table
+    with scatter/gather, diffed token by token against a contiguous cache;
+    FlashDecoding for long contexts.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import torch
+
+import oracle.paged_attention as PA
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "closed_forms.json")
+
+
+def golden():
+    with open(GOLDEN) as f:
+        return json.load(f)
+
+
+def _rand_bits(rng, shape, scale=1.0):
+    return PA.f64_to_bf16_bits(rng.standard_normal(shape) * scale)
+
+
+def _random_paged(rng, seq_lens, H, Hk, D, ps, extra_pages=2, scale=1.0):
+    """Random contiguous per-sequence K/V, then scattered into a shuffled pool.
+
+    Returns (q, k_pages, v_pages, block_table, contiguous K list, contiguous V list).
+    The scatter here is written independently of the oracle's gather.
+    """
+    B = len(seq_lens)
+    npg = [(L + ps - 1) // ps for L in seq_lens]
+    P = sum(npg) + extra_pages
+    MB = max(1, max(npg))
+    perm = rng.permutation(P)
+    bt = np.full((B, MB), -1, dtype=np.int64)
+    off = 0
+    for b, n in enumerate(npg):
+        bt[b, :n] = perm[off:off + n]
+        off += n
+    q = _rand_bits(rng, (B, H, D))
+    kp = np.full((P, Hk, ps, D), 0x7FC0, dtype=np.uint16)  # NaN everywhere unused
+    vp = np.full((P, Hk, ps, D), 0x7FC0, dtype=np.uint16)
+    Kc, Vc = [], []
+    for b, L in enumerate(seq_lens):
+        K = _rand_bits(rng, (Hk, L, D), scale)
+        V = _rand_bits(rng, (Hk, L, D))
+        Kc.append(K)
+        Vc.append(V)
+        for j in range(npg[b]):
+            n = min(ps, L - j * ps)
+            kp[bt[b, j], :, :n, :] = K[:, j * ps:j * ps + n, :]
+            vp[bt[b, j], :, :n, :] = V[:, j * ps:j * ps + n, :]
+    return q, kp, vp, bt, Kc, Vc
+
+
+def _sdpa_reference(q_bits, Kc, Vc, H, Hk, scale):
+    """torch scaled_dot_product_attention (CPU, float64) on contiguous K/V.
+
+    K/V heads are expanded to query heads with repeat_interleave (query head h
+    reads kv head h // G).  Empty contexts give zeros.
+    """
+    B, _, D = q_bits.shape
+    G = H // Hk
+    out = np.zeros((B, H, D))
+    for b in range(B):
+        L = Kc[b].shape[1]
+        if L == 0:
+            continue
+        qt = torch.from_numpy(PA.bf16_bits_to_f64(q_bits[b])).reshape(1, H, 1, D)
+        Kt = torch.from_numpy(PA.bf16_bits_to_f64(Kc[b])).repeat_interleave(G, dim=0)[None]
+        Vt = torch.from_numpy(PA.bf16_bits_to_f64(Vc[b])).repeat_interleave(G, dim=0)[None]
+        o = torch.nn.functional.scaled_dot_product_attention(qt, Kt, Vt, scale=scale)
+        out[b] = o[0, :, 0, :].numpy()
+    return out
+
+
+# --------------------------------------------------------------------------- checks
+
+def check_bf16_decode():
+    """bf16 -> fp64 decoding on known bit patterns and against torch's cast."""
+    bits = np.array([0x3F80, 0xC000, 0x0000, 0x8000, 0x3F81, 0x7F80, 0x0001, 0x4049],
+                    dtype=np.uint16)
+    want = [1.0, -2.0, 0.0, -0.0, 1.0 + 2.0 ** -7, math.inf, 2.0 ** -133, 3.140625]
+    got = PA.bf16_bits_to_f64(bits)
+    assert np.array_equal(got, np.array(want)), got
+    x = np.random.default_rng(0).standard_normal(1000) * 100
+    tb = torch.from_numpy(x).to(torch.bfloat16)
+    assert np.array_equal(PA.f64_to_bf16_bits(x), tb.view(torch.int16).numpy().view(np.uint16))
+    assert np.array_equal(PA.bf16_bits_to_f64(PA.f64_to_bf16_bits(x)), tb.to(torch.float64).numpy())
+
+
+def check_closed_form_three_tokens():
+    g = golden()["three_token_softmax"]
+    q = PA.f64_to_bf16_bits(np.array(g["q"]))
+    K = PA.bf16_bits_to_f64(PA.f64_to_bf16_bits(np.array(g["K"])))
+    V = PA.bf16_bits_to_f64(PA.f64_to_bf16_bits(np.array(g["V"])))
+    out = PA.attend_one_query(PA.bf16_bits_to_f64(q), K, V, g["scale"])
+    assert np.allclose(out, g["expected_out"], rtol=0, atol=1e-13), out
+
+
+def check_closed_form_paged():
+    """The golden three tokens, stored through a reversed block table, single and MQA heads."""
+    g = golden()["three_token_softmax"]
+    p = golden()["paged_three_token"]
+    ps, P = p["page_size"], p["num_pages"]
+    K = PA.f64_to_bf16_bits(np.array(g["K"]))
+    V = PA.f64_to_bf16_bits(np.array(g["V"]))
+    kp = np.full((P, 1, ps, 2), 0x7FC0, dtype=np.uint16)
+    vp = np.full((P, 1, ps, 2), 0x7FC0, dtype=np.uint16)
+    bt = np.array([p["block_table"]])
+    for t in range(3):
+        kp[bt[0, t // ps], 0, t % ps] = K[t]
+        vp[bt[0, t // ps], 0, t % ps] = V[t]
+    # Three query heads sharing the single kv head (MQA): e0 -> golden answer,
+    # 0 -> mean of V rows, -e0 -> weights 1/7, 2/7, 4/7.
+    q = PA.f64_to_bf16_bits(np.array([[[1.0, 0.0], [0.0, 0.0], [-1.0, 0.0]]]))
+    out = PA.paged_decode_attention(q, kp, vp, bt, np.array([3]), g["scale"])
+    Vf = PA.bf16_bits_to_f64(V)
+    assert np.allclose(out[0, 0], p["expected_out"], atol=1e-13), out
+    assert np.allclose(out[0, 1], Vf.mean(axis=0), atol=1e-13), out
+    assert np.allclose(out[0, 2], (Vf[0] + 2 * Vf[1] + 4 * Vf[2]) / 7, atol=1e-13), out
+
+
+def check_single_token_returns_v():
+    rng = np.random.default_rng(1)
+    q, kp, vp, bt, Kc, Vc = _random_paged(rng, [1, 1, 1], 8, 2, 64, 16)
+    out = PA.paged_decode_attention(q, kp, vp, bt, np.array([1, 1, 1]), 0.125)
+    for b in range(3):
+        for h in range(8):
+            assert np.array_equal(out[b, h], PA.bf16_bits_to_f64(Vc[b][h // 4, 0])), (b, h)
+
+
+def check_identical_v_rows():
+    rng = np.random.default_rng(2)
+    L = 37
+    q, kp, vp, bt, Kc, Vc = _random_paged(rng, [L], 4, 1, 32, 16)
+    row = _rand_bits(rng, (32,))
+    for j in range((L + 15) // 16):
+        n = min(16, L - 16 * j)
+        vp[bt[0, j], 0, :n, :] = row
+    out = PA.paged_decode_attention(q, kp, vp, bt, np.array([L]), 0.3)
+    for h in range(4):
+        assert np.allclose(out[0, h], PA.bf16_bits_to_f64(row), rtol=0, atol=1e-13)
+
+
+def check_zero_query_gives_mean():
+    rng = np.random.default_rng(3)
+    L = 50
+    q, kp, vp, bt, Kc, Vc = _random_paged(rng, [L], 2, 2, 16, 16)
+    q[:] = 0
+    out = PA.paged_decode_attention(q, kp, vp, bt, np.array([L]), 1.0)
+    for h in range(2):
+        assert np.allclose(out[0, h], PA.bf16_bits_to_f64(Vc[0][h]).mean(axis=0), atol=1e-14)
+
+
+def _pure_python_attention(q_bits, kp, vp, bt, seq_lens, scale):
+    """Triple loop, no numpy arithmetic: math.exp and float sums only."""
+    B, H, D = q_bits.shape
+    Hk, ps = kp.shape[1], kp.shape[2]
+    G = H // Hk
+    f = lambda bits: float(PA.bf16_bits_to_f64(np.uint16(bits)))  # noqa: E731
+    out = [[[0.0] * D for _ in range(H)] for _ in range(B)]
+    for b in range(B):
+        L = int(seq_lens[b])
+        for h in range(H):
+            kvh = h // G
+            qv = [f(q_bits[b, h, d]) for d in range(D)]
+            scores = []
+            for t in range(L):
+                pg, sl = int(bt[b][t // ps]), t % ps
+                scores.append(scale * sum(qv[d] * f(kp[pg, kvh, sl, d]) for d in range(D)))
+            if L == 0:
+                continue
+            mx = max(scores)
+            w = [math.exp(s - mx) for s in scores]
+            tot = sum(w)
+            for d in range(D):
+                acc = 0.0
+                for t in range(L):
+                    pg, sl = int(bt[b][t // ps]), t % ps
+                    acc += w[t] * f(vp[pg, kvh, sl, d])
+                out[b][h][d] = acc / tot
+    return np.array(out)
+
+
+def check_brute_force_tiny():
+    """Workload-1 shapes (MQA, D=64) and a small GQA case against pure Python."""
+    rng = np.random.default_rng(4)
+    for seq_lens, H, Hk, D, ps in [([17, 40], 4, 1, 16, 16), ([5, 0, 9], 6, 3, 8, 4)]:
+        q, kp, vp, bt, Kc, Vc = _random_paged(rng, seq_lens, H, Hk, D, ps)
+        sl = np.array(seq_lens)
+        got = PA.paged_decode_attention(q, kp, vp, bt, sl, 1.0 / math.sqrt(D))
+        want = _pure_python_attention(q, kp, vp, bt, sl, 1.0 / math.sqrt(D))
+        assert np.allclose(got, want, rtol=0, atol=1e-12), np.abs(got - want).max()
+
+
+def check_against_sdpa():
+    """Paged oracle == torch SDPA (float64) on the contiguous K/V it was scattered from."""
+    rng = np.random.default_rng(5)
+    cases = [([17, 40], 4, 1, 64, 16, 0.125),
+             ([3, 100, 33, 64], 8, 2, 32, 16, 0.2),
+             ([70, 1, 129], 12, 4, 16, 32, 0.5),
+             ([200], 96, 1, 8, 64, 0.35),
+             ([31, 0, 16], 8, 8, 8, 16, 1.0)]
+    for seq_lens, H, Hk, D, ps, scale in cases:
+        q, kp, vp, bt, Kc, Vc = _random_paged(rng, seq_lens, H, Hk, D, ps)
+        got = PA.paged_decode_attention(q, kp, vp, bt, np.array(seq_lens), scale)
+        want = _sdpa_reference(q, Kc, Vc, H, Hk, scale)
+        assert np.allclose(got, want, rtol=0, atol=1e-12), (seq_lens, np.abs(got - want).max())
+
+
+def check_mqa_equals_mha_replicated():
+    """MQA (one shared K/V head) equals MHA whose per-head K/V are copies of it."""
+    rng = np.random.default_rng(6)
+    H = 6
+    q, kp, vp, bt, Kc, Vc = _random_paged(rng, [23, 48], H, 1, 16, 8)
+    sl = np.array([23, 48])
+    mqa = PA.paged_decode_attention(q, kp, vp, bt, sl, 0.25)
+    mha = PA.paged_decode_attention(q, np.repeat(kp, H, axis=1), np.repeat(vp, H, axis=1),
+                                    bt, sl, 0.25)
+    assert np.array_equal(mqa, mha)
+    # GQA with G=1 on the replicated cache also equals MHA per head.
+    assert mqa.shape == (2, H, 16)
+
+
+def check_page_permutation_invariance():
+    """Relabelling pages (moving their data and the block table together) changes nothing."""
+    rng = np.random.default_rng(7)
+    sl = np.array([45, 16, 3])
+    q, kp, vp, bt, Kc, Vc = _random_paged(rng, list(sl), 4, 2, 16, 16, extra_pages=3)
+    base = PA.paged_decode_attention(q, kp, vp, bt, sl, 0.3)
+    P = kp.shape[0]
+    sigma = rng.permutation(P)  # new page id of old page p is sigma[p]
+    kp2 = np.empty_like(kp)
+    vp2 = np.empty_like(vp)
+    kp2[sigma] = kp
+    vp2[sigma] = vp
+    bt2 = np.where(bt >= 0, sigma[np.maximum(bt, 0)], -1)
+    perm_out = PA.paged_decode_attention(q, kp2, vp2, bt2, sl, 0.3)
+    assert np.array_equal(base, perm_out)
+
+
+def check_large_scores_stay_finite():
+    """Scores near 1e3 (overflow for a naive exp) give the one-hot closed form."""
+    K = np.zeros((4, 2))
+    K[2, 0] = 1.0
+    V = np.arange(8, dtype=np.float64).reshape(4, 2)
+    out = PA.attend_one_query(np.array([1.0, 0.0]), K, V, 2000.0)
+    assert np.all(np.isfinite(out))
+    assert np.allclose(out, V[2], atol=1e-12)
+
+
+def check_zero_length_context():
+    rng = np.random.default_rng(8)
+    q, kp, vp, bt, Kc, Vc = _random_paged(rng, [0, 5], 4, 2, 8, 16)
+    out = PA.paged_decode_attention(q, kp, vp, bt, np.array([0, 5]), 0.5)
+    assert np.array_equal(out[0], np.zeros((4, 8)))
+    assert np.all(np.isfinite(out[1]))
+
+
+def check_unused_slots_never_read():
+    """NaN in unused pages and tail slots does not reach the output (the scatter
+    in _random_paged leaves them NaN)."""
+    rng = np.random.default_rng(9)
+    sl = np.array([19, 1, 32])
+    q, kp, vp, bt, Kc, Vc = _random_paged(rng, list(sl), 4, 2, 8, 16, extra_pages=4)
+    out = PA.paged_decode_attention(q, kp, vp, bt, sl, 0.5)
+    assert np.all(np.isfinite(out))
+
+
+def check_rows_subset_matches_full():
+    rng = np.random.default_rng(10)
+    sl = np.array([30, 7, 64])
+    q, kp, vp, bt, Kc, Vc = _random_paged(rng, list(sl), 8, 2, 16, 16)
+    full = PA.paged_decode_attention(q, kp, vp, bt, sl, 0.4)
+    rows = [(2, 7), (0, 0), (1, 3), (2, 0)]
+    sub = PA.paged_decode_attention_rows(q, kp, vp, bt, sl, 0.4, rows)
+    for i, (b, h) in enumerate(rows):
+        assert np.array_equal(sub[i], full[b, h])
+
+
+def check_kv_append():
+    """After the scatter, the gather at positions[b] returns k_new[b] bit for bit;
+    every other byte of both pools is unchanged."""
+    rng = np.random.default_rng(11)
+    sl = [5, 16, 33, 1]
+    Hk, D, ps = 2, 8, 16
+    q, kp, vp, bt, Kc, Vc = _random_paged(rng, sl, 4, Hk, D, ps, extra_pages=2)
+    pos = np.array([4, 15, 32, 0])
+    kn = _rand_bits(rng, (4, Hk, D))
+    vn = _rand_bits(rng, (4, Hk, D))
+    k2, v2 = PA.kv_append(kp, vp, kn, vn, bt, pos)
+    changed_k = np.zeros(kp.shape[:3], dtype=bool)
+    for b in range(4):
+        for kvh in range(Hk):
+            gk = PA.gather_sequence_kv(k2, bt[b], kvh, pos[b] + 1, ps)
+            gv = PA.gather_sequence_kv(v2, bt[b], kvh, pos[b] + 1, ps)
+            assert np.array_equal(gk[pos[b]], PA.bf16_bits_to_f64(kn[b, kvh]))
+            assert np.array_equal(gv[pos[b]], PA.bf16_bits_to_f64(vn[b, kvh]))
+        changed_k[bt[b, pos[b] // ps], :, pos[b] % ps] = True
+    assert np.array_equal(k2[~changed_k], kp[~changed_k])
+    assert np.array_equal(v2[~changed_k], vp[~changed_k])
+    # inputs untouched
+    assert not np.shares_memory(k2, kp)
+
+
+def check_kv_cache_bytes():
+    g = golden()
+    for c in g["kv_cache_bytes"]["cases"]:
+        assert PA.kv_cache_bytes(c["num_layers"], c["num_kv_heads"], c["head_dim"],
+                                 c["seq_len"], c["batch"]) == c["bytes"], c
+    # Bytes the gather touches equal the formula (one layer, bf16).
+    rng = np.random.default_rng(12)
+    sl = [37, 5]
+    Hk, D, ps = 2, 8, 16
+    q, kp, vp, bt, Kc, Vc = _random_paged(rng, sl, 4, Hk, D, ps)
+    touched = 0
+    for b, L in enumerate(sl):
+        slots = {(int(bt[b][t // ps]), t % ps) for t in range(L)}
+        touched += 2 * len(slots) * Hk * D * 2
+    assert touched == sum(PA.kv_cache_bytes(1, Hk, D, L) for L in sl)
+    r = g["mqa_cache_ratio"]
+    assert PA.kv_cache_bytes(1, r["num_heads"], 128, 1000) // PA.kv_cache_bytes(1, 1, 128, 1000) == r["ratio"]
+
+
+def check_lse_merge():
+    """Splitting the context anywhere and merging (o_i, lse_i) gives the full result."""
+    rng = np.random.default_rng(13)
+    L, D = 97, 16
+    qv = rng.standard_normal(D)
+    K = rng.standard_normal((L, D)) * 3
+    V = rng.standard_normal((L, D))
+    full = PA.attend_one_query(qv, K, V, 0.7)
+    for cuts in ([97], [1, 96], [50, 47], [10, 10, 10, 67], [1] * 97):
+        pieces, s = [], 0
+        for n in cuts:
+            pieces.append(PA.partial_softmax_piece(qv, K[s:s + n], V[s:s + n], 0.7))
+            s += n
+        assert np.allclose(PA.merge_partial_pieces(pieces), full, atol=1e-13), cuts
+    # The lse of the whole context is log(sum exp(s)) directly.
+    _, lse = PA.partial_softmax_piece(qv, K, V, 0.7)
+    s = 0.7 * (K @ qv)
+    assert abs(lse - math.log(np.sum(np.exp(s)))) < 1e-11
+
+
+ALL_CHECKS = [
+    check_bf16_decode,
+    check_closed_form_three_tokens,
+    check_closed_form_paged,
+    check_single_token_returns_v,
+    check_identical_v_rows,
+    check_zero_query_gives_mean,
+    check_brute_force_tiny,
+    check_against_sdpa,
+    check_mqa_equals_mha_replicated,
+    check_page_permutation_invariance,
+    check_large_scores_stay_finite,
+    check_zero_length_context,
+    check_unused_slots_never_read,
+    check_rows_subset_matches_full,
+    check_kv_append,
+    check_kv_cache_bytes,
+    check_lse_merge,
+]

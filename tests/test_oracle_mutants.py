@@ -1,0 +1,111 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check a pin rejects each.
+
+Each mutant replaces one oracle function through the module object; the pins
+in tests/oracle_pins.py then run against the mutated oracle.  A mutant that no
+pin catches would mean the pins cannot see that class of mistake.
+"""
+import numpy as np
+import pytest
+
+import oracle.paged_attention as PA
+import oracle_pins as P
+
+
+def _kv_head_modulo(h, num_heads, num_kv_heads):
+    return h % num_kv_heads                      # wrong head -> kv-head map
+
+
+def _gather_swapped(pages_bits, bt_row, kv_head, seq_len, page_size):
+    t = np.arange(seq_len)
+    page = np.asarray(bt_row)[np.minimum(t % page_size, len(bt_row) - 1)]
+    slot = np.minimum(t // page_size, page_size - 1)  # page/slot indices swapped
+    return PA.bf16_bits_to_f64(pages_bits[page, kv_head, slot, :])
+
+
+def _gather_off_by_one(pages_bits, bt_row, kv_head, seq_len, page_size):
+    n = max(seq_len - 1, 0)                     # drops the newest token
+    t = np.arange(n)
+    page = np.asarray(bt_row)[t // page_size]
+    return PA.bf16_bits_to_f64(pages_bits[page, kv_head, t % page_size, :])
+
+
+def _attend_no_scale(q_row, K, V, scale):
+    if K.shape[0] == 0:
+        return np.zeros(V.shape[-1])
+    s = K @ q_row                               # scale dropped
+    w = np.exp(s - s.max())
+    return (w @ V) / w.sum()
+
+
+def _attend_no_max(q_row, K, V, scale):
+    if K.shape[0] == 0:
+        return np.zeros(V.shape[-1])
+    with np.errstate(over="ignore", invalid="ignore"):
+        w = np.exp(scale * (K @ q_row))         # max not subtracted
+        return (w @ V) / w.sum()
+
+
+def _attend_transposed(q_row, K, V, scale):
+    if K.shape[0] == 0:
+        return np.zeros(V.shape[-1])
+    s = scale * (K @ q_row)
+    w = np.exp(s - s.max())
+    w = w / w.sum()
+    if V.shape[0] == V.shape[1]:
+        return V @ w                            # transposed operand
+    return (w @ V)[::-1].copy()                 # reversed output dims
+
+
+def _attend_sign(q_row, K, V, scale):
+    if K.shape[0] == 0:
+        return np.zeros(V.shape[-1])
+    s = -scale * (K @ q_row)                    # wrong sign on the scores
+    w = np.exp(s - s.max())
+    return (w @ V) / w.sum()
+
+
+def _merge_no_weights(pieces):
+    return sum(p[0] for p in pieces) / len(pieces)  # ignores the lse weights
+
+
+def _append_wrong_slot(kp, vp, kn, vn, bt, positions):
+    k = np.array(kp, copy=True)
+    v = np.array(vp, copy=True)
+    ps = k.shape[2]
+    for b in range(kn.shape[0]):
+        pos = int(positions[b]) + 1               # off by one slot
+        pg = int(bt[b][min(pos // ps, bt.shape[1] - 1)])
+        k[pg, :, pos % ps, :] = kn[b]
+        v[pg, :, pos % ps, :] = vn[b]
+    return k, v
+
+
+def _cache_bytes_single(num_layers, num_kv_heads, head_dim, seq_len, batch=1, bytes_per_elem=2):
+    return num_layers * num_kv_heads * head_dim * seq_len * batch * bytes_per_elem  # K only
+
+
+MUTANTS = [
+    ("kv_head_of", _kv_head_modulo),
+    ("gather_sequence_kv", _gather_swapped),
+    ("gather_sequence_kv", _gather_off_by_one),
+    ("attend_one_query", _attend_no_scale),
+    ("attend_one_query", _attend_no_max),
+    ("attend_one_query", _attend_transposed),
+    ("attend_one_query", _attend_sign),
+    ("merge_partial_pieces", _merge_no_weights),
+    ("kv_append", _append_wrong_slot),
+    ("kv_cache_bytes", _cache_bytes_single),
+]
+
+
+@pytest.mark.parametrize("name,fn", MUTANTS, ids=[f.__name__ for _, f in MUTANTS])
+def test_mutant_is_caught(monkeypatch, name, fn):
+    monkeypatch.setattr(PA, name, fn)
+    caught = []
+    for check in P.ALL_CHECKS:
+        try:
+            with np.errstate(all="ignore"):
+                check()
+        except (AssertionError, IndexError, ValueError, FloatingPointError):
+            caught.append(check.__name__)
+    assert caught, f"no pin rejects mutant {fn.__name__} of {name}"
