@@ -1,0 +1,197 @@
+"""Paged GQA/MQA decode attention for B200 (sm_100a): Python binding of libgqa_decode.so.
+
+The binding only marshals arguments: every step of the computation runs in the
+library's CUDA kernels (see include/gqa_decode.h).  PyTorch supplies device
+memory and the current stream.  There is no CPU fallback: if the shared library
+is missing or the tensors are not on a CUDA device, the calls raise.
+
+    kv_append(k_new, v_new, k_pages, v_pages, block_table, positions)
+    paged_decode_attn(q, k_pages, v_pages, block_table, seq_lens, out=None, scale=None)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "GQAError",
+    "library_path",
+    "load_library",
+    "kv_append",
+    "paged_decode_attn",
+    "check_device_error",
+    "kv_cache_bytes",
+    "set_num_workers",
+    "set_wait_limit_ns",
+    "launch_count",
+    "EXPORTED_SYMBOLS",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_NAME = "libgqa_decode.so"
+
+GQA_OK = 0
+STATUS_NAMES = {0: "GQA_OK", -1: "GQA_ERR_INVALID_ARG", -2: "GQA_ERR_UNSUPPORTED",
+                -3: "GQA_ERR_CUDA", -4: "GQA_ERR_DEVICE_BOUNDS", -5: "GQA_ERR_TIMEOUT"}
+
+# Every extern "C" entry point declared in include/gqa_decode.h.
+EXPORTED_SYMBOLS = (
+    "gqa_kv_append",
+    "gqa_paged_decode_attn",
+    "gqa_check_device_error",
+    "gqa_last_error_string",
+    "gqa_kv_cache_bytes",
+    "gqa_set_num_workers",
+    "gqa_set_wait_limit_ns",
+    "gqa_launch_count",
+    "gqa_abi_version",
+)
+
+
+class GQAError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, _LIB_NAME)
+
+
+_lib = None
+
+
+def load_library() -> ctypes.CDLL:
+    """Load the in-tree shared library (built by gqa_decode_attention_04_b200.build)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = library_path()
+    if not os.path.exists(path):
+        raise ImportError(
+            f"{path} not found: build it with `python -m gqa_decode_attention_04_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, i32, f32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_int64
+    lib.gqa_kv_append.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]
+    lib.gqa_kv_append.restype = i32
+    lib.gqa_paged_decode_attn.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32,
+                                          i32, i32, vp]
+    lib.gqa_paged_decode_attn.restype = i32
+    lib.gqa_check_device_error.argtypes = [vp]
+    lib.gqa_check_device_error.restype = i32
+    lib.gqa_last_error_string.argtypes = []
+    lib.gqa_last_error_string.restype = ctypes.c_char_p
+    lib.gqa_kv_cache_bytes.argtypes = [i32, i32, i32, i64]
+    lib.gqa_kv_cache_bytes.restype = ctypes.c_size_t
+    lib.gqa_set_num_workers.argtypes = [i32]
+    lib.gqa_set_num_workers.restype = i32
+    lib.gqa_set_wait_limit_ns.argtypes = [i64, i32]
+    lib.gqa_set_wait_limit_ns.restype = i32
+    lib.gqa_launch_count.argtypes = []
+    lib.gqa_launch_count.restype = ctypes.c_uint64
+    lib.gqa_abi_version.argtypes = []
+    lib.gqa_abi_version.restype = i32
+    _lib = lib
+    return lib
+
+
+def _check(status: int) -> None:
+    if status != GQA_OK:
+        msg = load_library().gqa_last_error_string().decode(errors="replace")
+        raise GQAError(status, msg)
+
+
+def _stream_ptr(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _need(t: torch.Tensor, name: str, dtype, device) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor (no CPU path exists)")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def kv_append(k_new, v_new, k_pages, v_pages, block_table, positions, stream=None) -> None:
+    """Write k_new/v_new [B, Hk, D] into the pages at positions[b] (bit-exact scatter)."""
+    dev = k_pages.device
+    for t, n, dt in ((k_new, "k_new", torch.bfloat16), (v_new, "v_new", torch.bfloat16),
+                     (k_pages, "k_pages", torch.bfloat16), (v_pages, "v_pages", torch.bfloat16),
+                     (block_table, "block_table", torch.int32), (positions, "positions", torch.int32)):
+        _need(t, n, dt, dev)
+    P, Hk, ps, D = k_pages.shape
+    if tuple(v_pages.shape) != (P, Hk, ps, D):
+        raise ValueError("v_pages shape differs from k_pages")
+    B = k_new.shape[0]
+    if tuple(k_new.shape) != (B, Hk, D) or tuple(v_new.shape) != (B, Hk, D):
+        raise ValueError("k_new / v_new must be [num_seqs, num_kv_heads, head_dim]")
+    if block_table.dim() != 2 or block_table.shape[0] != B or tuple(positions.shape) != (B,):
+        raise ValueError("block_table must be [num_seqs, max_blocks], positions [num_seqs]")
+    lib = load_library()
+    with torch.cuda.device(dev):
+        _check(lib.gqa_kv_append(k_new.data_ptr(), v_new.data_ptr(), k_pages.data_ptr(),
+                                 v_pages.data_ptr(), block_table.data_ptr(), positions.data_ptr(),
+                                 B, Hk, D, ps, block_table.shape[1], P, _stream_ptr(stream)))
+
+
+def paged_decode_attn(q, k_pages, v_pages, block_table, seq_lens, out: Optional[torch.Tensor] = None,
+                      scale: Optional[float] = None, stream=None) -> torch.Tensor:
+    """out[b, h] = softmax(scale * q[b, h] . K_b^T) V_b over the paged cache (bf16 out)."""
+    dev = q.device
+    for t, n, dt in ((q, "q", torch.bfloat16), (k_pages, "k_pages", torch.bfloat16),
+                     (v_pages, "v_pages", torch.bfloat16), (block_table, "block_table", torch.int32),
+                     (seq_lens, "seq_lens", torch.int32)):
+        _need(t, n, dt, dev)
+    B, H, D = q.shape
+    P, Hk, ps, D2 = k_pages.shape
+    if D2 != D or tuple(v_pages.shape) != (P, Hk, ps, D):
+        raise ValueError("page pools must be [num_pages, num_kv_heads, page_size, head_dim]")
+    if block_table.dim() != 2 or block_table.shape[0] != B or tuple(seq_lens.shape) != (B,):
+        raise ValueError("block_table must be [num_seqs, max_blocks], seq_lens [num_seqs]")
+    if out is None:
+        out = torch.empty((B, H, D), dtype=torch.bfloat16, device=dev)
+    else:
+        _need(out, "out", torch.bfloat16, dev)
+        if tuple(out.shape) != (B, H, D):
+            raise ValueError("out must be [num_seqs, num_heads, head_dim]")
+    if scale is None:
+        scale = 1.0 / (D ** 0.5)
+    lib = load_library()
+    with torch.cuda.device(dev):
+        _check(lib.gqa_paged_decode_attn(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(),
+                                         block_table.data_ptr(), seq_lens.data_ptr(), out.data_ptr(),
+                                         B, H, Hk, D, ps, float(scale), block_table.shape[1], P,
+                                         _stream_ptr(stream)))
+    return out
+
+
+def check_device_error(stream=None) -> None:
+    """Synchronise the stream; raise GQAError if a kernel flagged a device-side error."""
+    _check(load_library().gqa_check_device_error(_stream_ptr(stream)))
+
+
+def kv_cache_bytes(num_layers: int, num_kv_heads: int, head_dim: int, seq_len: int) -> int:
+    return int(load_library().gqa_kv_cache_bytes(num_layers, num_kv_heads, head_dim, seq_len))
+
+
+def set_num_workers(n: int) -> None:
+    _check(load_library().gqa_set_num_workers(int(n)))
+
+
+def set_wait_limit_ns(limit_ns: int, arm_without_copy: bool = False) -> None:
+    _check(load_library().gqa_set_wait_limit_ns(int(limit_ns), 1 if arm_without_copy else 0))
+
+
+def launch_count() -> int:
+    return int(load_library().gqa_launch_count())

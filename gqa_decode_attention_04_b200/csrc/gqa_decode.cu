@@ -1,0 +1,346 @@
+// C ABI of the paged GQA/MQA decode-attention library (declared in include/gqa_decode.h).
+//
+// Host responsibilities: argument validation (nothing is launched on a bad argument),
+// the per-device workspace (error word, split counters, split partials), TMA tensor
+// maps over the page pools, and kernel launches.  No call synchronises the stream
+// except gqa_check_device_error.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <unordered_map>
+
+#include "gqa_decode.h"
+#include "internal.cuh"
+
+namespace {
+
+thread_local char g_err_msg[512] = "no error";
+std::atomic<int> g_num_workers{0};
+std::atomic<int64_t> g_wait_limit_ns{1000000000LL};
+std::atomic<int> g_arm_without_copy{0};
+std::atomic<uint64_t> g_launches{0};
+
+gqa_status fail(gqa_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err_msg, sizeof(g_err_msg), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+gqa_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(GQA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// ------------------------------------------------------------------ per-device state
+struct DeviceState {
+  int sms = 0;
+  uint32_t* err = nullptr;
+  int32_t* counters = nullptr;
+  size_t counters_cap = 0;  // entries
+  float* part_o = nullptr;
+  float* part_ml = nullptr;
+  size_t slots_cap = 0;     // partial slots (each kHeadTile rows x 128 floats)
+};
+
+std::mutex g_mu;
+std::unordered_map<int, DeviceState> g_states;
+
+gqa_status get_state(DeviceState** out, int* dev_out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState& s = g_states[dev];
+  if (s.err == nullptr) {
+    e = cudaDeviceGetAttribute(&s.sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    e = cudaMalloc(&s.err, sizeof(uint32_t));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(error word)");
+    e = cudaMemset(s.err, 0, sizeof(uint32_t));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(error word)");
+  }
+  *out = &s;
+  *dev_out = dev;
+  return GQA_OK;
+}
+
+// Grow-only decode workspace.  Counters must be zero between launches: they are
+// zeroed when allocated and every launch leaves them zero.
+gqa_status ensure_workspace(DeviceState& s, size_t counters, size_t slots, cudaStream_t stream) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  cudaError_t e;
+  if (counters > s.counters_cap) {
+    if (s.counters) cudaFree(s.counters);
+    s.counters = nullptr;
+    s.counters_cap = 0;
+    size_t n = counters < 4096 ? 4096 : counters;
+    e = cudaMalloc(&s.counters, n * sizeof(int32_t));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(split counters)");
+    e = cudaMemsetAsync(s.counters, 0, n * sizeof(int32_t), stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(split counters)");
+    s.counters_cap = n;
+  }
+  if (slots > s.slots_cap) {
+    if (s.part_o) cudaFree(s.part_o);
+    if (s.part_ml) cudaFree(s.part_ml);
+    s.part_o = s.part_ml = nullptr;
+    s.slots_cap = 0;
+    e = cudaMalloc(&s.part_o, slots * gqa::kHeadTile * 128 * sizeof(float));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(split partials)");
+    e = cudaMalloc(&s.part_ml, slots * gqa::kHeadTile * 2 * sizeof(float));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(split partials)");
+    s.slots_cap = slots;
+  }
+  return GQA_OK;
+}
+
+// ------------------------------------------------------------------ tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// The pool [num_pages, Hk, ps, D] viewed as a 2-D bf16 tensor of P*Hk*ps rows and D
+// columns; one box is 16 rows (one chunk) x 64 columns (128 bytes), 128-byte swizzle.
+struct MapKey {
+  const void* ptr;
+  int64_t rows;
+  int d;
+  int dev;
+  bool operator==(const MapKey& o) const {
+    return ptr == o.ptr && rows == o.rows && d == o.d && dev == o.dev;
+  }
+};
+
+gqa_status make_pool_map(CUtensorMap* m, const void* pool, int64_t rows, int d, int dev) {
+  static thread_local MapKey keys[8];
+  static thread_local CUtensorMap maps[8];
+  static thread_local int next = 0;
+  MapKey k{pool, rows, d, dev};
+  for (int i = 0; i < 8; ++i)
+    if (keys[i] == k) {
+      *m = maps[i];
+      return GQA_OK;
+    }
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return fail(GQA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(gqa::kChunk)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(pool), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(GQA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  keys[next] = k;
+  maps[next] = *m;
+  next = (next + 1) % 8;
+  return GQA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* gqa_last_error_string(void) { return g_err_msg; }
+
+int gqa_abi_version(void) { return 1; }
+
+uint64_t gqa_launch_count(void) { return g_launches.load(); }
+
+size_t gqa_kv_cache_bytes(int num_layers, int num_kv_heads, int head_dim, int64_t seq_len) {
+  if (num_layers < 0 || num_kv_heads < 0 || head_dim < 0 || seq_len < 0) return 0;
+  return static_cast<size_t>(2) * num_layers * num_kv_heads * head_dim *
+         static_cast<size_t>(seq_len) * 2;
+}
+
+gqa_status gqa_set_num_workers(int n) {
+  if (n < 0 || n > (1 << 20)) return fail(GQA_ERR_INVALID_ARG, "num_workers must be in [0, 2^20]");
+  g_num_workers.store(n);
+  return GQA_OK;
+}
+
+gqa_status gqa_set_wait_limit_ns(int64_t limit_ns, int arm_without_copy) {
+  if (limit_ns <= 0) return fail(GQA_ERR_INVALID_ARG, "wait limit must be positive");
+  g_wait_limit_ns.store(limit_ns);
+  g_arm_without_copy.store(arm_without_copy ? 1 : 0);
+  return GQA_OK;
+}
+
+gqa_status gqa_kv_append(const void* k_new, const void* v_new, void* k_pages, void* v_pages,
+                         const int32_t* block_table, const int32_t* positions, int num_seqs,
+                         int num_kv_heads, int head_dim, int page_size, int max_blocks_per_seq,
+                         int num_pages, void* stream) {
+  if (num_seqs < 0) return fail(GQA_ERR_INVALID_ARG, "num_seqs < 0");
+  if (num_kv_heads < 1 || head_dim < 1 || page_size < 1 || max_blocks_per_seq < 1 || num_pages < 1)
+    return fail(GQA_ERR_INVALID_ARG, "sizes must be positive");
+  if (head_dim % 8 != 0) return fail(GQA_ERR_UNSUPPORTED, "head_dim must be a multiple of 8");
+  if (static_cast<int64_t>(max_blocks_per_seq) * page_size > INT32_MAX)
+    return fail(GQA_ERR_UNSUPPORTED, "max_blocks_per_seq * page_size exceeds 2^31");
+  if (num_seqs == 0) return GQA_OK;
+  if (!k_new || !v_new || !k_pages || !v_pages || !block_table || !positions)
+    return fail(GQA_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_pages, 16) || !aligned(v_pages, 16))
+    return fail(GQA_ERR_INVALID_ARG, "bf16 tensors must be 16-byte aligned");
+  DeviceState* st;
+  int dev;
+  gqa_status s = get_state(&st, &dev);
+  if (s != GQA_OK) return s;
+  gqa::AppendParams p;
+  p.k_new = static_cast<const uint4*>(k_new);
+  p.v_new = static_cast<const uint4*>(v_new);
+  p.k_pages = static_cast<uint4*>(k_pages);
+  p.v_pages = static_cast<uint4*>(v_pages);
+  p.block_table = block_table;
+  p.positions = positions;
+  p.err = st->err;
+  p.num_seqs = num_seqs;
+  p.num_kv_heads = num_kv_heads;
+  p.vec_per_row = head_dim / 8;
+  p.page_size = page_size;
+  p.max_blocks = max_blocks_per_seq;
+  p.num_pages = num_pages;
+  cudaError_t e = gqa::launch_kv_append(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "kv_append launch");
+  g_launches.fetch_add(1);
+  return GQA_OK;
+}
+
+gqa_status gqa_paged_decode_attn(const void* q, const void* k_pages, const void* v_pages,
+                                 const int32_t* block_table, const int32_t* seq_lens, void* out,
+                                 int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                 int page_size, float scale, int max_blocks_per_seq,
+                                 int num_pages, void* stream) {
+  if (num_seqs < 0) return fail(GQA_ERR_INVALID_ARG, "num_seqs < 0");
+  if (num_seqs > 65536) return fail(GQA_ERR_UNSUPPORTED, "num_seqs > 65536");
+  if (num_heads < 1 || num_kv_heads < 1 || head_dim < 1 || page_size < 1 ||
+      max_blocks_per_seq < 1 || num_pages < 1)
+    return fail(GQA_ERR_INVALID_ARG, "sizes must be positive");
+  if (num_heads % num_kv_heads != 0)
+    return fail(GQA_ERR_INVALID_ARG, "num_heads (%d) is not a multiple of num_kv_heads (%d)",
+                num_heads, num_kv_heads);
+  if (head_dim != 64 && head_dim != 128)
+    return fail(GQA_ERR_UNSUPPORTED, "head_dim %d not built (64, 128)", head_dim);
+  if (page_size % gqa::kChunk != 0 || page_size > 256)
+    return fail(GQA_ERR_UNSUPPORTED, "page_size %d not built (multiple of 16, <= 256)", page_size);
+  if (!std::isfinite(scale)) return fail(GQA_ERR_INVALID_ARG, "scale is not finite");
+  const int64_t rows = static_cast<int64_t>(num_pages) * num_kv_heads * page_size;
+  if (rows >= (int64_t{1} << 31))
+    return fail(GQA_ERR_UNSUPPORTED, "num_pages * num_kv_heads * page_size exceeds 2^31");
+  if (static_cast<int64_t>(max_blocks_per_seq) * page_size >= (int64_t{1} << 31))
+    return fail(GQA_ERR_UNSUPPORTED, "max_blocks_per_seq * page_size exceeds 2^31");
+  if (num_seqs == 0) return GQA_OK;
+  if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !out)
+    return fail(GQA_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned(k_pages, 16) || !aligned(v_pages, 16))
+    return fail(GQA_ERR_INVALID_ARG, "k_pages / v_pages must be 16-byte aligned");
+  if (!aligned(q, 4) || !aligned(out, 8))
+    return fail(GQA_ERR_INVALID_ARG, "q must be 4-byte and out 8-byte aligned");
+
+  DeviceState* st;
+  int dev;
+  gqa_status s = get_state(&st, &dev);
+  if (s != GQA_OK) return s;
+  cudaStream_t strm = static_cast<cudaStream_t>(stream);
+
+  const int group = num_heads / num_kv_heads;
+  const int n_ht = (group + gqa::kHeadTile - 1) / gqa::kHeadTile;
+  const gqa::DecodeLaunch cfg = gqa::decode_launch_config(head_dim, group);
+  // Upper bound on the chunk count (seq_lens are device data).
+  const int64_t chunks_per_seq =
+      static_cast<int64_t>(max_blocks_per_seq) * (page_size / gqa::kChunk);
+  const int64_t max_chunks = static_cast<int64_t>(num_seqs) * num_kv_heads * n_ht * chunks_per_seq;
+  int64_t workers = static_cast<int64_t>(st->sms) * cfg.ctas_per_sm * cfg.warps_per_cta;
+  const int forced = g_num_workers.load();
+  if (forced > 0) workers = forced;
+  if (workers > max_chunks) workers = max_chunks;
+  if (workers < 1) workers = 1;
+  const int grid = static_cast<int>((workers + cfg.warps_per_cta - 1) / cfg.warps_per_cta);
+
+  const size_t segments = static_cast<size_t>(num_seqs) * num_kv_heads * n_ht;
+  s = ensure_workspace(*st, segments, static_cast<size_t>(2 * workers), strm);
+  if (s != GQA_OK) return s;
+
+  CUtensorMap tk, tv;
+  s = make_pool_map(&tk, k_pages, rows, head_dim, dev);
+  if (s != GQA_OK) return s;
+  s = make_pool_map(&tv, v_pages, rows, head_dim, dev);
+  if (s != GQA_OK) return s;
+
+  gqa::DecodeParams p;
+  p.q = static_cast<const uint16_t*>(q);
+  p.out = static_cast<uint16_t*>(out);
+  p.block_table = block_table;
+  p.seq_lens = seq_lens;
+  p.part_o = st->part_o;
+  p.part_ml = st->part_ml;
+  p.counters = st->counters;
+  p.err = st->err;
+  p.num_seqs = num_seqs;
+  p.num_heads = num_heads;
+  p.num_kv_heads = num_kv_heads;
+  p.group = group;
+  p.n_ht = n_ht;
+  p.page_size = page_size;
+  p.max_blocks = max_blocks_per_seq;
+  p.num_pages = num_pages;
+  p.head_dim = head_dim;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.num_workers = static_cast<int>(workers);
+  p.wait_limit_ns = static_cast<uint64_t>(g_wait_limit_ns.load());
+  p.arm_without_copy = g_arm_without_copy.load();
+  cudaError_t e = gqa::launch_decode(p, tk, tv, grid, strm);
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  g_launches.fetch_add(1);
+  return GQA_OK;
+}
+
+gqa_status gqa_check_device_error(void* stream) {
+  cudaStream_t strm = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(strm);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  DeviceState* st;
+  int dev;
+  gqa_status s = get_state(&st, &dev);
+  if (s != GQA_OK) return s;
+  uint32_t word = 0;
+  e = cudaMemcpy(&word, st->err, sizeof(word), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(error word)");
+  if (word == 0) return GQA_OK;
+  e = cudaMemset(st->err, 0, sizeof(uint32_t));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(error word)");
+  if (word & gqa::kErrTimeout) {
+    {
+      std::lock_guard<std::mutex> lk(g_mu);
+      if (st->counters) cudaMemset(st->counters, 0, st->counters_cap * sizeof(int32_t));
+    }
+    cudaDeviceSynchronize();
+    return fail(GQA_ERR_TIMEOUT, "a kernel wait ran out of time; its work was skipped");
+  }
+  return fail(GQA_ERR_DEVICE_BOUNDS,
+              "a page id, position or sequence length was out of range; that work was skipped");
+}
+
+}  // extern "C"

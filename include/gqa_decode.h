@@ -1,0 +1,168 @@
+/*
+ * gqa_decode.h -- C ABI of the B200 (sm_100a) paged GQA/MQA decode-attention library.
+ *
+ * The library computes, for one new query token per sequence,
+ *
+ *     out[b, h, :] = sum_t softmax_t( scale * <q[b, h, :], K_b[t, kvh(h), :]> ) * V_b[t, kvh(h), :]
+ *
+ * over the sequence's cached keys/values K_b, V_b, t in [0, seq_lens[b]), where
+ * the cache is paged and addressed through a per-sequence block table.  It also
+ * provides the scatter that writes each step's new K/V row into its page.
+ *
+ * Sources (web pages the method is described on):
+ *   - "TensorRT对Multi-Query Attention的专项优化支持": each decoded token re-reads all
+ *     cached K/V of its sequence (the bandwidth-bound step); MHA keeps K_i, V_i per
+ *     head, MQA shares one K, V among all query heads (cache h*d_k*s -> d_k*s);
+ *     multi-head Q against shared K/V is computed without copying or broadcasting
+ *     K/V; QK^T and AV with tiled shared-memory K/V prefetch; fixed-length pages
+ *     ("Page-Based管理机制").  Its plugin entry launch_mqa_kernel(q, k, v, out,
+ *     batch, heads, seq_q, seq_kv, head_dim, stream) is the model for the call shape.
+ *   - tiny-llm "优化" page: GQA (num_kv_heads may differ from num_heads, section 3);
+ *     preallocated KV cache and its size formula (section 2); paged KV "strategy 1"
+ *     = block table + scatter/gather; FlashDecoding for long-context decode
+ *     (planned-optimisation table).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *   All tensor arguments are DEVICE pointers to row-major, contiguous memory on the
+ *   current CUDA device, owned by the caller; the library never frees or retains them
+ *   beyond the call.  bf16 means IEEE bfloat16 stored as 16-bit words.
+ *
+ *     q, out             [num_seqs, num_heads, head_dim]                 bf16
+ *     k_pages, v_pages   [num_pages, num_kv_heads, page_size, head_dim]   bf16
+ *     block_table        [num_seqs, max_blocks_per_seq]                   int32
+ *     seq_lens           [num_seqs]                                       int32
+ *     positions          [num_seqs]                                       int32
+ *     k_new, v_new       [num_seqs, num_kv_heads, head_dim]               bf16
+ *
+ *   Token t of sequence b is slot (t % page_size) of page block_table[b][t / page_size];
+ *   query head h reads kv head h / (num_heads / num_kv_heads).  Block-table entries
+ *   past ceil(seq_lens[b] / page_size) are never read.
+ *
+ *   `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  Calls
+ *   only enqueue work: they never synchronise the stream and never read device data
+ *   on the host.
+ *
+ *   Errors: a negative gqa_status.  Argument errors are detected on the host before
+ *   anything is launched, and gqa_last_error_string() explains them.  Errors that
+ *   depend on device data (a page id outside [0, num_pages), a position or seq_len
+ *   beyond max_blocks_per_seq * page_size, a negative length, a bounded wait that
+ *   ran out) cannot be seen at launch time: the kernels skip the offending work,
+ *   never fault or trap, and set a per-device error word that
+ *   gqa_check_device_error() reports.
+ *
+ *   Scratch memory: gqa_paged_decode_attn needs a per-device workspace (split
+ *   partial results and per-segment arrival counters).  The library allocates it with
+ *   cudaMalloc on the first call per device and grows it when a call needs more;
+ *   it is freed at process exit.  Calls on different streams of the same device that
+ *   overlap in time share that workspace and must not run concurrently.
+ */
+#ifndef GQA_DECODE_H_
+#define GQA_DECODE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GQA_OK = 0,
+  GQA_ERR_INVALID_ARG = -1,   /* null pointer, bad size, misaligned pointer        */
+  GQA_ERR_UNSUPPORTED = -2,   /* valid but not built: head_dim, page_size, limits  */
+  GQA_ERR_CUDA = -3,          /* a CUDA runtime/driver call failed                 */
+  GQA_ERR_DEVICE_BOUNDS = -4, /* device-side index out of range (work skipped)     */
+  GQA_ERR_TIMEOUT = -5        /* a kernel's bounded wait ran out (work skipped)    */
+} gqa_status;
+
+/*
+ * gqa_kv_append -- scatter one new K and V row per (sequence, kv head) into the
+ * paged cache (the "scatter" half of the block-table scheme on the tiny-llm
+ * "优化" page; the decode step's "append pos").
+ *
+ *   k_pages[block_table[b][p / page_size], kvh, p % page_size, :] = k_new[b, kvh, :]
+ *   v_pages[...same slot...]                                      = v_new[b, kvh, :]
+ *   with p = positions[b], for every b < num_seqs and kvh < num_kv_heads.
+ *
+ * Bits are copied unchanged (bit-exact); no other byte of the pools is written.
+ * Requirements: head_dim % 8 == 0, page_size >= 1, all bf16 pointers 16-byte
+ * aligned, num_seqs >= 0 (0 launches nothing).  A position outside
+ * [0, max_blocks_per_seq * page_size) or a page id outside [0, num_pages) skips that
+ * sequence's row and sets GQA_ERR_DEVICE_BOUNDS in the device error word.
+ */
+gqa_status gqa_kv_append(const void* k_new, const void* v_new, void* k_pages, void* v_pages,
+                         const int32_t* block_table, const int32_t* positions, int num_seqs,
+                         int num_kv_heads, int head_dim, int page_size, int max_blocks_per_seq,
+                         int num_pages, void* stream);
+
+/*
+ * gqa_paged_decode_attn -- decode attention of one query token per sequence over the
+ * paged cache, with num_heads query heads sharing num_kv_heads K/V heads (MQA when
+ * num_kv_heads == 1, MHA when equal, GQA between): the definition at the top of this
+ * file, written to out as bf16 (round to nearest even) from fp32 accumulation.
+ *
+ * Each kv head's K/V are read from HBM once for all of its query heads.  Long
+ * contexts are split across the GPU (FlashDecoding, named on the tiny-llm page);
+ * partial results are merged with their log-sum-exp inside the same launch.
+ *
+ *   scale           multiplier of q.k (usually 1/sqrt(head_dim)), finite.
+ *   seq_lens[b]     context length of sequence b including any token appended this
+ *                   step; 0 gives an all-zero output row.
+ * Requirements: head_dim in {64, 128}; page_size a multiple of 16 in [16, 256];
+ * num_heads % num_kv_heads == 0; q, out 4-byte aligned; k_pages, v_pages 16-byte
+ * aligned; num_seqs <= 65536.  Slots at or beyond seq_lens[b] and unused pages may
+ * hold any bits (NaN included) without affecting out.
+ */
+gqa_status gqa_paged_decode_attn(const void* q, const void* k_pages, const void* v_pages,
+                                 const int32_t* block_table, const int32_t* seq_lens, void* out,
+                                 int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                 int page_size, float scale, int max_blocks_per_seq,
+                                 int num_pages, void* stream);
+
+/*
+ * gqa_check_device_error -- synchronise `stream`, then read and clear the current
+ * device's error word.  Returns GQA_OK, GQA_ERR_DEVICE_BOUNDS, GQA_ERR_TIMEOUT (takes
+ * precedence when both are set; it also resets the decode workspace counters a
+ * timed-out launch may have left behind) or GQA_ERR_CUDA.
+ */
+gqa_status gqa_check_device_error(void* stream);
+
+/* Human-readable message of the last error returned on this host thread. */
+const char* gqa_last_error_string(void);
+
+/*
+ * gqa_kv_cache_bytes -- bytes of a bf16 K+V cache for one sequence:
+ * 2 x num_layers x num_kv_heads x head_dim x seq_len x 2 bytes (tiny-llm "优化" page,
+ * section 2).  Returns 0 for negative arguments.
+ */
+size_t gqa_kv_cache_bytes(int num_layers, int num_kv_heads, int head_dim, int64_t seq_len);
+
+/*
+ * gqa_set_num_workers -- number of split workers (one warp each) used by the next
+ * gqa_paged_decode_attn calls on this process; 0 (default) picks it from the SM count.
+ * A fixed count changes how the context is split, never the result beyond fp32
+ * rounding order; tests use it to force many or few splits.  Returns
+ * GQA_ERR_INVALID_ARG for n < 0.
+ */
+gqa_status gqa_set_num_workers(int n);
+
+/*
+ * gqa_set_wait_limit_ns -- upper bound on any single wait inside the kernels
+ * (default 1e9 ns).  When `arm_without_copy` is non-zero the next decode launches arm
+ * their copy barriers without issuing the copies, so every wait runs out: this
+ * exercises the GQA_ERR_TIMEOUT path without faulting anything.  Tests only.
+ */
+gqa_status gqa_set_wait_limit_ns(int64_t limit_ns, int arm_without_copy);
+
+/* Kernels launched by this library since the process started (all devices). */
+uint64_t gqa_launch_count(void);
+
+/* ABI version of this header: 1. */
+int gqa_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQA_DECODE_H_ */

@@ -1,0 +1,190 @@
+"""GPU parity: paged_decode_attn through the C ABI against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import gqa_decode_attention_04_b200 as gq
+import oracle
+from parity import assert_close, gpu_f64, host_arrays, oracle_out, oracle_rows
+from workloads import bf16_bits, make_custom_inputs, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _default_workers():
+    gq.set_num_workers(0)
+    yield
+    gq.set_num_workers(0)
+
+
+def _run(inp, dev):
+    d = inp.to(dev)
+    out = gq.paged_decode_attn(d.q, d.k_pages, d.v_pages, d.block_table, d.seq_lens, scale=d.scale)
+    gq.check_device_error()
+    return d, out
+
+
+# (seq_lens, H, Hk, D, ps): several chunks and pages per sequence, ragged tails,
+# every group size the kernels specialise on, both head dims, all page-size classes.
+SMALL_CASES = [
+    ([17, 40], 4, 1, 64, 16),                      # workload-1 shapes
+    ([1, 15, 16, 17, 31, 33, 100], 8, 2, 128, 16),  # G=4
+    ([300, 1, 77], 32, 8, 128, 16),                # G=4, longer
+    ([129, 64, 65], 16, 2, 128, 32),               # G=8, ps=32
+    ([250, 7], 12, 1, 128, 64),                    # G=12 (16-row tile)
+    ([90, 200], 16, 1, 64, 128),                   # G=16, D=64, ps=128
+    ([40, 160], 32, 1, 128, 64),                   # G=32: two head tiles
+    ([70], 96, 1, 128, 64),                        # G=96 (MQA, workload-3 shape)
+    ([5, 0, 33], 8, 8, 128, 16),                   # MHA (G=1) and an empty sequence
+    ([1000, 3, 500, 2048], 8, 1, 64, 16),          # D=64 long
+]
+
+
+@pytest.mark.parametrize("case", SMALL_CASES, ids=lambda c: f"L{len(c[0])}_H{c[1]}_Hk{c[2]}_D{c[3]}_ps{c[4]}")
+def test_small_parity(cuda_device, case):
+    seq_lens, H, Hk, D, ps = case
+    inp = make_custom_inputs(seq_lens, H, Hk, D, ps, seed=(sum(seq_lens) * 31 + H * 7 + D + ps) % 10007, extra_pages=3)
+    d, out = _run(inp, cuda_device)
+    assert_close(gpu_f64(out), oracle_out(host_arrays(inp)), what=str(case))
+    # an empty sequence gives exact zeros
+    for b, L in enumerate(seq_lens):
+        if L == 0:
+            assert torch.count_nonzero(out[b]) == 0
+
+
+@pytest.mark.parametrize("workers", [1, 2, 3, 7, 64, 1000, 5000])
+def test_forced_split_counts(cuda_device, workers):
+    """Any number of split workers (1 .. more than chunks) gives the oracle's answer."""
+    inp = make_custom_inputs([700, 33, 1, 2000, 129], 16, 4, 128, 16, seed=11)
+    gq.set_num_workers(workers)
+    d, out = _run(inp, cuda_device)
+    assert_close(gpu_f64(out), oracle_out(host_arrays(inp)), what=f"workers={workers}")
+
+
+def test_splits_agree_with_each_other(cuda_device):
+    inp = make_custom_inputs([3000, 17], 8, 1, 128, 16, seed=12)
+    outs = []
+    for w in (1, 5, 999):
+        gq.set_num_workers(w)
+        outs.append(_run(inp, cuda_device)[1].float())
+    for o in outs[1:]:
+        assert (o - outs[0]).abs().max().item() <= 1e-2
+
+
+def test_single_token_context_returns_v_exactly(cuda_device):
+    inp = make_custom_inputs([1, 1, 1, 1], 16, 4, 128, 16, seed=13)
+    d, out = _run(inp, cuda_device)
+    G = 4
+    for b in range(4):
+        page = int(inp.block_table[b, 0])
+        for h in range(16):
+            assert torch.equal(out[b, h].cpu(), inp.v_pages[page, h // G, 0].cpu()), (b, h)
+
+
+def test_identical_v_rows_return_that_row(cuda_device):
+    inp = make_custom_inputs([333], 8, 2, 128, 16, seed=14)
+    row = torch.randn(128).to(torch.bfloat16)
+    vp = inp.v_pages.clone()
+    live = ~vp.float().isnan()
+    vp[live.all(dim=-1)] = row
+    inp.v_pages = vp
+    d, out = _run(inp, cuda_device)
+    err = (out.float().cpu() - row.float()).abs().max().item()
+    assert err <= 2e-2
+
+
+def test_identity_and_shuffled_block_tables_agree(cuda_device):
+    """The same token data through an identity and a shuffled block table."""
+    seq_lens = [150, 47, 16]
+    inp = make_custom_inputs(seq_lens, 8, 2, 128, 16, seed=15, poison=False)
+    # rebuild the pool so pages are laid out in identity order
+    bt = inp.block_table
+    npg = [(L + 15) // 16 for L in seq_lens]
+    order = torch.cat([bt[b, :n] for b, n in enumerate(npg)]).long()
+    ident = inp.to("cpu")
+    ident.k_pages = inp.k_pages[order].contiguous()
+    ident.v_pages = inp.v_pages[order].contiguous()
+    ident.num_pages = len(order)
+    nbt = torch.full_like(bt, -1)
+    off = 0
+    for b, n in enumerate(npg):
+        nbt[b, :n] = torch.arange(off, off + n, dtype=torch.int32)
+        off += n
+    ident.block_table = nbt
+    _, o1 = _run(inp, cuda_device)
+    _, o2 = _run(ident, cuda_device)
+    assert torch.equal(o1, o2)
+
+
+def test_nan_in_unread_slots_does_not_leak(cuda_device):
+    inp = make_custom_inputs([17, 31, 2], 8, 2, 128, 16, seed=16, extra_pages=5)
+    assert inp.k_pages.float().isnan().any()
+    _, out = _run(inp, cuda_device)
+    assert torch.isfinite(out.float()).all()
+
+
+def test_large_scale_peaked_softmax(cuda_device):
+    inp = make_custom_inputs([2000, 517], 16, 2, 128, 16, seed=17, spike_fraction=0.01, scale=0.5)
+    _, out = _run(inp, cuda_device)
+    assert_close(gpu_f64(out), oracle_out(host_arrays(inp)), what="peaked")
+
+
+def test_out_buffer_is_written_in_place(cuda_device):
+    inp = make_custom_inputs([40, 9], 4, 1, 64, 16, seed=18)
+    d = inp.to(cuda_device)
+    out = torch.full((2, 4, 64), float("nan"), dtype=torch.bfloat16, device=cuda_device)
+    r = gq.paged_decode_attn(d.q, d.k_pages, d.v_pages, d.block_table, d.seq_lens, out=out, scale=d.scale)
+    assert r.data_ptr() == out.data_ptr()
+    assert_close(gpu_f64(out), oracle_out(host_arrays(inp)))
+
+
+# ------------------------------------------------------------------ full-size workloads
+
+def _sample_rows(inp, n_seq=6, seed=0):
+    rng = np.random.default_rng(seed)
+    B, H = inp.num_seqs, inp.num_heads
+    L = inp.seq_lens.cpu().numpy()
+    seqs = {int(np.argmax(L)), int(np.argmin(L))}
+    seqs |= set(int(b) for b in rng.choice(B, size=min(n_seq, B), replace=False))
+    return [(b, h) for b in sorted(seqs) for h in range(H)]
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("index", [1, 2, 3])
+def test_workload_full_parity(cuda_device, index):
+    """Workloads 1-3 at full size, every output row, default launch configuration."""
+    inp = make_inputs(index)
+    d, out = _run(inp, cuda_device)
+    mx, mean = assert_close(gpu_f64(out), oracle_out(host_arrays(inp)), what=inp.name)
+    print(f"{inp.name}: max abs {mx:.2e} mean abs {mean:.2e}")
+
+
+@pytest.mark.slow
+def test_workload4_long_context_sampled(cuda_device):
+    """131072-token contexts with a peaked softmax: every head of sampled sequences."""
+    inp = make_inputs(4)
+    d, out = _run(inp, cuda_device)
+    rows = [(b, h) for b in range(4) for h in range(0, 64, 3)]
+    got = gpu_f64(out)[[r[0] for r in rows], [r[1] for r in rows]]
+    assert_close(got, oracle_rows(host_arrays(inp), rows), what="long_context")
+
+
+@pytest.mark.slow
+def test_workload5_append_then_attend(cuda_device):
+    """Continuous batch: kv_append of each sequence's new token, then decode attention."""
+    inp = make_inputs(5)
+    d = inp.to(cuda_device)
+    gq.kv_append(d.k_new, d.v_new, d.k_pages, d.v_pages, d.block_table, d.positions)
+    out = gq.paged_decode_attn(d.q, d.k_pages, d.v_pages, d.block_table, d.seq_lens, scale=d.scale)
+    gq.check_device_error()
+    h = host_arrays(inp)
+    k2, v2 = oracle.kv_append(h["k"], h["v"], bf16_bits(inp.k_new), bf16_bits(inp.v_new),
+                              h["bt"], inp.positions.numpy())
+    # the scatter is bit-exact over the whole pool (NaN patterns included)
+    assert np.array_equal(bf16_bits(d.k_pages), k2)
+    assert np.array_equal(bf16_bits(d.v_pages), v2)
+    h["k"], h["v"] = k2, v2
+    rows = _sample_rows(inp, n_seq=10)
+    got = gpu_f64(out)[[r[0] for r in rows], [r[1] for r in rows]]
+    assert_close(got, oracle_rows(h, rows), what="continuous_batch")
