@@ -46,11 +46,13 @@ KERNEL_SOURCES = ["gqa_decode_attention_04_b200/csrc/decode_split.cu",
 
 # ------------------------------------------------------------------ helpers
 
-def algorithmic_bytes(inp, with_append: bool) -> dict:
+def algorithmic_bytes(inp, with_append: bool, num_seqs=None) -> dict:
     """Bytes the step must move: every cached K/V byte once, q in, out back, plus
-    the block-table entries and lengths read, and the appended rows."""
-    B, H, Hk, D, ps = inp.num_seqs, inp.num_heads, inp.num_kv_heads, inp.head_dim, inp.page_size
-    L = inp.seq_lens.to(torch.int64).cpu()
+    the block-table entries and lengths read, and the appended rows.  With
+    num_seqs, only the first num_seqs sequences count."""
+    B = inp.num_seqs if num_seqs is None else num_seqs
+    H, Hk, D, ps = inp.num_heads, inp.num_kv_heads, inp.head_dim, inp.page_size
+    L = inp.seq_lens[:B].to(torch.int64).cpu()
     kv = int(L.sum()) * Hk * D * 2 * 2
     pages = int(((L + ps - 1) // ps).sum())
     qo = 2 * B * H * D * 2
@@ -185,97 +187,114 @@ def barrier():
 # ------------------------------------------------------------------ CPU oracle timing
 
 def time_oracle(inp, min_seconds: float, max_seconds: float):
-    """Time the fp64 oracle, as it stands, on whole passes over the workload (or on a
-    prefix of its sequences when one pass is too long).  Returns (bytes/s, seqs/s,
-    description).  BLAS is held to one thread, so exactly one host core is used."""
-    import numpy as np
+    """Time the fp64 oracle, as it stands, on the same step (its kv_append, then its
+    attention) over the workload, repeated for at least min_seconds, or over a prefix
+    of the sequences when one pass would exceed max_seconds.  Returns (bytes/s,
+    seqs/s, description).  BLAS is held to one thread: exactly one host core."""
     from threadpoolctl import threadpool_limits
     import oracle
 
     q, k, v = bf16_bits(inp.q), bf16_bits(inp.k_pages), bf16_bits(inp.v_pages)
-    bt, sl = inp.block_table.cpu().numpy(), inp.seq_lens.cpu().numpy()
+    kn, vn = bf16_bits(inp.k_new), bf16_bits(inp.v_new)
+    bt, sl, pos = inp.block_table.numpy(), inp.seq_lens.numpy(), inp.positions.numpy()
     B = inp.num_seqs
-    Hk, D = inp.num_kv_heads, inp.head_dim
-    done_seqs, done_bytes, elapsed, passes = 0, 0, 0.0, 0
+
+    def one_step(n):
+        k2, v2 = oracle.kv_append(k, v, kn[:n], vn[:n], bt[:n], pos[:n])
+        oracle.paged_decode_attention(q[:n], k2, v2, bt[:n], sl[:n], inp.scale)
+
     with threadpool_limits(1):
-        n = B
-        # size the sample: shrink to a prefix if one pass would exceed max_seconds
         t0 = time.perf_counter()
-        oracle.paged_decode_attention(q[:1], k, v, bt[:1], sl[:1], inp.scale)
-        per_tok = (time.perf_counter() - t0) / max(1, int(sl[0]))
-        est = per_tok * float(sl.sum())
-        if est > max_seconds:
-            n = max(1, int(B * max_seconds / est))
-        while elapsed < min_seconds or passes == 0:
+        one_step(1)
+        est_all = (time.perf_counter() - t0) * float(sl.sum()) / max(1, int(sl[0]))
+        n = B if est_all <= max_seconds else max(1, int(B * max_seconds / est_all))
+        step_bytes = algorithmic_bytes(inp, with_append=True, num_seqs=n)["step"]
+        elapsed, passes = 0.0, 0
+        while elapsed < min_seconds and elapsed < max_seconds:
             t0 = time.perf_counter()
-            oracle.paged_decode_attention(q[:n], k, v, bt[:n], sl[:n], inp.scale)
+            one_step(n)
             elapsed += time.perf_counter() - t0
             passes += 1
-            done_seqs += n
-            done_bytes += int(sl[:n].astype(np.int64).sum()) * Hk * D * 4 + 2 * n * inp.num_heads * D * 2
-            if elapsed > max_seconds:
-                break
-    desc = (f"{passes} pass(es) of the fp64 oracle over {n} of {B} sequences "
-            f"({int(sl[:n].sum())} context tokens each pass), single thread")
-    return done_bytes / elapsed, done_seqs / elapsed, desc
+    desc = (f"{passes} pass(es) of the fp64 oracle step (kv_append + attention) over {n} of "
+            f"{B} sequences ({int(sl[:n].sum())} context tokens per pass), single thread")
+    return step_bytes * passes / elapsed, n * passes / elapsed, desc
 
 
 # ------------------------------------------------------------------ arms
 
 def run_reference(args, rank, world):
-    """Reference arm: the fp64 CPU oracle on the host cores, rank 0 only."""
+    """Reference arm: the fp64 CPU oracle on the host, rank 0 only.  Each step is a
+    bounded sample of the workload: the oracle's kv_append, then its attention over a
+    prefix of the sequences (all of them when that fits the time budget)."""
     if rank != 0:
         return None
-    inp = make_inputs(args.workload, poison=False)
-    bytes_per_step = algorithmic_bytes(inp, with_append=False)["decode"]
-    # each step is a bounded sample: the oracle over a prefix of the sequences
-    sl = inp.seq_lens.cpu()
     import numpy as np
     from threadpoolctl import threadpool_limits
     import oracle
+
+    seed = 1000 + args.workload
+    inp = _with_append(make_inputs(args.workload, seed=seed, poison=False), seed)
     q, k, v = bf16_bits(inp.q), bf16_bits(inp.k_pages), bf16_bits(inp.v_pages)
-    bt, sln = inp.block_table.cpu().numpy(), sl.numpy()
-    n = inp.num_seqs
+    kn, vn = bf16_bits(inp.k_new), bf16_bits(inp.v_new)
+    bt, sl, pos = inp.block_table.numpy(), inp.seq_lens.numpy(), inp.positions.numpy()
+    B = inp.num_seqs
+
+    def one_step(n):
+        k2, v2 = oracle.kv_append(k, v, kn[:n], vn[:n], bt[:n], pos[:n])
+        oracle.paged_decode_attention(q[:n], k2, v2, bt[:n], sl[:n], inp.scale)
+
     times, byts, seqs = [], [], []
     with threadpool_limits(1):
         t0 = time.perf_counter()
-        oracle.paged_decode_attention(q[:1], k, v, bt[:1], sln[:1], inp.scale)
-        per_tok = (time.perf_counter() - t0) / max(1, int(sln[0]))
+        one_step(1)
+        t_one = time.perf_counter() - t0
         budget = max(0.5, min(4.0, 150.0 / max(1, args.steps + args.warmup)))
-        n = max(1, min(n, int(inp.num_seqs * budget / max(1e-9, per_tok * float(sln.sum())))))
+        est_all = t_one * float(sl.sum()) / max(1, int(sl[0]))
+        n = B if est_all <= budget else max(1, int(B * budget / est_all))
+        step_bytes = algorithmic_bytes(inp, with_append=True, num_seqs=n)["step"]
         for i in range(args.warmup + args.steps):
             t0 = time.perf_counter()
-            oracle.paged_decode_attention(q[:n], k, v, bt[:n], sln[:n], inp.scale)
+            one_step(n)
             dt = time.perf_counter() - t0
             if i >= args.warmup:
                 times.append(dt)
-                byts.append(int(sln[:n].astype(np.int64).sum()) * inp.num_kv_heads * inp.head_dim * 4
-                            + 2 * n * inp.num_heads * inp.head_dim * 2)
+                byts.append(step_bytes)
                 seqs.append(n)
     total_t = sum(times)
     value = sum(byts) / total_t / 1e12
-    sample = (f"each step: fp64 oracle over the first {n} of {inp.num_seqs} sequences "
-              f"({int(sln[:n].sum())} context tokens), single thread")
-    line = {
+    sample = (f"each step: fp64 oracle kv_append + attention over the first {n} of {B} sequences "
+              f"({int(sl[:n].sum())} context tokens), single thread")
+    return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TB/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total_t / len(times), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "tokens_per_s": sum(seqs) / total_t,
-        "config": {"workload": WORKLOADS[args.workload].name, **_config_keys(inp)},
+        "config": {**_config_keys(inp, world), "l2": "host memory (CPU oracle)"},
         "cpu_baseline": {"value": value, "unit": "TB/s", "cores": 1, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-        "bytes_per_step_full_workload": bytes_per_step,
     }
-    return line
 
 
-def _config_keys(inp):
+def _config_keys(inp, world):
     L = inp.seq_lens.to(torch.int64).cpu()
-    return {"num_seqs": inp.num_seqs, "num_heads": inp.num_heads, "num_kv_heads": inp.num_kv_heads,
-            "head_dim": inp.head_dim, "page_size": inp.page_size, "num_pages": inp.num_pages,
-            "context_tokens": int(L.sum()), "seq_len_min": int(L.min()), "seq_len_max": int(L.max()),
-            "seed": 1000 + inp.meta.get("workload", 0)}
+    return {"workload": inp.name, "num_seqs": inp.num_seqs, "num_heads": inp.num_heads,
+            "num_kv_heads": inp.num_kv_heads, "head_dim": inp.head_dim, "page_size": inp.page_size,
+            "num_pages": inp.num_pages, "context_tokens": int(L.sum()), "seq_len_min": int(L.min()),
+            "seq_len_max": int(L.max()), "seed": 1000 + inp.meta.get("workload", 0),
+            "step": "kv_append + paged_decode_attn",
+            "parallelism": f"dp{world} (independent batch per GPU)" if world > 1 else "single GPU"}
+
+
+def _with_append(inp, seed):
+    """Give a workload without its own append step one new K/V token per sequence
+    (positions = seq_len - 1, already counted in seq_lens)."""
+    if inp.positions is None:
+        g = torch.Generator().manual_seed(seed + 2)
+        inp.positions = (inp.seq_lens - 1).clamp(min=0).to(torch.int32)
+        inp.k_new = torch.randn(inp.num_seqs, inp.num_kv_heads, inp.head_dim, generator=g).to(torch.bfloat16)
+        inp.v_new = torch.randn(inp.num_seqs, inp.num_kv_heads, inp.head_dim, generator=g).to(torch.bfloat16)
+    return inp
 
 
 def run_ours(args, rank, world, local):
@@ -284,15 +303,7 @@ def run_ours(args, rank, world, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     seed = 1000 + args.workload + 7919 * rank
-    inp_cpu = make_inputs(args.workload, seed=seed, poison=False)
-    # the decode step appends this step's token before attending (positions = len - 1)
-    if inp_cpu.positions is None:
-        g = torch.Generator().manual_seed(seed + 2)
-        inp_cpu.positions = (inp_cpu.seq_lens - 1).clamp(min=0).to(torch.int32)
-        inp_cpu.k_new = torch.randn(inp_cpu.num_seqs, inp_cpu.num_kv_heads, inp_cpu.head_dim,
-                                    generator=g).to(torch.bfloat16)
-        inp_cpu.v_new = torch.randn(inp_cpu.num_seqs, inp_cpu.num_kv_heads, inp_cpu.head_dim,
-                                    generator=g).to(torch.bfloat16)
+    inp_cpu = _with_append(make_inputs(args.workload, seed=seed, poison=False), seed)
     nbytes = algorithmic_bytes(inp_cpu, with_append=True)
 
     # Rotate between independent copies of the pools so consecutive steps never
@@ -328,7 +339,9 @@ def run_ours(args, rank, world, local):
            for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     launches0 = gq.launch_count()
-    with ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ else 0) as clocks:
+    visible = [x for x in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if x.strip()]
+    smi_index = visible[local] if local < len(visible) else str(local)
+    with ClockSampler(smi_index) as clocks:
         barrier()
         torch.cuda.synchronize()
         start.record(stream)
@@ -395,11 +408,9 @@ def run_ours(args, rank, world, local):
         "pct_of_peak": 100.0 * value_tbps * 1e3 / (peak * world),
         "tokens_per_s": tokens_per_s,
         "kv_tbps": nbytes["kv"] * args.steps * world / (total_ms * 1e-3) / 1e12,
-        "config": {"workload": WORKLOADS[args.workload].name, **_config_keys(inp_cpu),
-                   "step": "kv_append + paged_decode_attn",
+        "config": {**_config_keys(inp_cpu, world),
                    "l2": f"inputs larger than L2: {n_sets} rotated pool copies of "
-                         f"{kv_bytes / 1e6:.0f} MB each vs {l2 / 1e6:.0f} MB L2",
-                   "parallelism": f"dp{world} (independent batch per GPU)" if world > 1 else "single GPU"},
+                         f"{kv_bytes / 1e6:.0f} MB each vs {l2 / 1e6:.0f} MB L2"},
         "e2e": {"value": e2e_tbps, "unit": "TB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms / args.steps},
         "gpu_launches": int(launches),
