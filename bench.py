@@ -39,7 +39,7 @@ from workloads import WORKLOADS, make_inputs, bf16_bits  # noqa: E402
 METRIC = "paged GQA decode attn: achieved HBM TB/s (% of B200 peak), tokens/s"
 FALLBACK_HBM_GBS = 6650.0
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
-KERNEL_SOURCES = ["gqa_decode_attention_04_b200/csrc/decode_split.cu",
+KERNEL_SOURCES = ["gqa_decode_attention_04_b200/csrc/decode_ws.cu",
                   "gqa_decode_attention_04_b200/csrc/ptx.cuh",
                   "gqa_decode_attention_04_b200/csrc/internal.cuh"]
 
@@ -414,7 +414,7 @@ def run_ours(args, rank, world, local):
         "e2e": {"value": e2e_tbps, "unit": "TB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms / args.steps},
         "gpu_launches": int(launches),
-        "roofline": {"bound": "hbm", "kernel": "decode_split_kernel",
+        "roofline": {"bound": "hbm", "kernel": "decode_ws_kernel",
                      "achieved": achieved_gbs, "peak": peak, "unit": "GB/s",
                      "frac": achieved_gbs / peak, "peak_kind": f"{peak_kind} (hbm_gbs)",
                      "traffic": profiled_traffic(WORKLOADS[args.workload].name, units),

@@ -58,7 +58,8 @@ class GQAError(RuntimeError):
 
 
 def library_path() -> str:
-    return os.path.join(_HERE, _LIB_NAME)
+    """The in-tree library; GQA_DECODE_LIB may name another build of the same ABI."""
+    return os.environ.get("GQA_DECODE_LIB") or os.path.join(_HERE, _LIB_NAME)
 
 
 _lib = None

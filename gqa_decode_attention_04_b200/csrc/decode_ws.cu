@@ -1,0 +1,838 @@
+// Paged GQA/MQA decode attention: one new query token per sequence.
+//
+// What is computed (page "TensorRT对Multi-Query Attention的专项优化支持": decode re-reads
+// all cached K/V; MQA/GQA query heads share K/V heads and the plugin avoids copying or
+// broadcasting K/V to them; QK^T then AV on tensor cores with tiled shared-memory K/V
+// prefetch; paged cache.  tiny-llm "优化" page: GQA, block table + gather,
+// FlashDecoding for long contexts):
+//
+//   out[b, h] = sum_t softmax_t(scale * q[b, h] . K_b[t, kvh]) V_b[t, kvh],  kvh = h / G.
+//
+// Design (B200, sm_100a), one CTA per SM:
+//   * Work list.  The context of every (sequence b, segment s = kv head x head tile) is
+//     cut into 64-token blocks; all blocks of all segments form one linear list in
+//     (b, s, block) order, split into equal contiguous ranges, one per CTA (split-KV /
+//     FlashDecoding, balanced at block granularity whatever the length mix).  Each CTA
+//     derives its range from seq_lens in a short prologue: no planning kernel and no
+//     host synchronisation.
+//   * Producer warp.  Walks the CTA's blocks, reads page ids from the block table
+//     through a prefetched register window and issues one 3-D TMA copy per 16-token
+//     sub-chunk and tensor (box: 64 columns x 16 rows x head_dim/64 column groups,
+//     128-byte swizzle) into a ring of 64-token stages (full/empty mbarriers).  It also
+//     writes a small descriptor per stage.
+//   * Consumer warps (mma.sync m16n8k16, bf16 in, fp32 accumulate), tokens on the M side:
+//     S^T = K Q^T, softmax down the token axis, P^T moved to B-fragment layout with
+//     movmatrix, O^T += V^T P^T with V^T read by ldmatrix.trans.  Every K/V row in shared
+//     memory serves all query heads of its kv head, so HBM is read once per kv head.
+//       - small groups (G <= 16): each of the 4 consumers takes one 16-token sub-chunk
+//         of every stage for all G heads; at a piece end their partial softmax states
+//         are combined in shared memory.
+//       - large groups (MQA-like, G > 16): each consumer takes 8 or 16 of the query heads
+//         over all 64 tokens of every stage.
+//   * Online softmax in the log2 domain with a lazily moved reference: O and the sum are
+//     rescaled only when a head's running maximum rises by more than 8 (factor 256);
+//     numerator and denominator share the reference, so the result is unchanged.
+//   * Cross-CTA merge.  A segment spanning several CTAs leaves one piece per CTA
+//     (unnormalised O, reference max, sum); the last CTA to finish its piece (arrival
+//     counter) merges all pieces with their log-sum-exp weights using all consumer
+//     threads, writes out, and resets the counter to zero.
+//   * Safety.  Page ids and lengths are range-checked on the device (bad work is skipped
+//     and an error bit set); every mbarrier wait is bounded in time.
+#include "internal.cuh"
+#include "ptx.cuh"
+
+namespace gqa {
+
+namespace {
+
+template <int D>
+struct Geo {
+  static constexpr int kBoxes = D / 64;                      // 64-column (128-byte) boxes
+  static constexpr int kBoxBytes = kChunk * 128;             // 16 rows x 128 bytes
+  static constexpr int kSubBytes = kBoxes * kBoxBytes;       // one 16-token K (or V) tile
+  static constexpr int kTileBytes = kSubChunks * kSubBytes;  // 64-token K (or V) tile
+  static constexpr int kStageBytes = 2 * kTileBytes;
+};
+
+constexpr float kRescaleThreshold = 8.0f;
+constexpr int kMaxWarps = 9;
+
+// Per-stage descriptor, written by the producer before the stage's full barrier
+// completes (release/acquire through the mbarrier).
+struct StageInfo {
+  int64_t seg_base;  // linear index of block 0 of this block's segment
+  int b, seg, blk, nblk;
+  int nvalid;        // valid tokens of this block (1..64)
+  int submask;       // bit s: sub-chunk s was loaded
+  int flags;
+  int pad;
+};
+enum : int { kFirstOfPiece = 1, kLastOfPiece = 2, kSole = 4, kFirstPieceOfCta = 8 };
+
+__device__ __forceinline__ int eff_len(int L, int cap) { return L < 0 ? 0 : (L > cap ? cap : L); }
+
+struct Cursor {
+  int b;     // sequence
+  int seg;   // kv_head * n_ht + head_tile
+  int blk;   // block within the segment
+  int nblk;  // blocks per segment of sequence b
+  int len;   // effective context length of sequence b
+};
+
+__device__ __forceinline__ void cursor_load_seq(Cursor& cu, const DecodeParams& p, int cap) {
+  cu.len = (cu.b >= 0 && cu.b < p.num_seqs) ? eff_len(__ldg(p.seq_lens + cu.b), cap) : 0;
+  cu.nblk = (cu.len + kBlock - 1) / kBlock;
+}
+
+__device__ __forceinline__ int64_t worker_start(int64_t w, int64_t T, int64_t W) { return w * T / W; }
+// The worker (CTA) whose range holds linear block x.
+__device__ __forceinline__ int64_t worker_of(int64_t x, int64_t T, int64_t W) {
+  return ((x + 1) * W - 1) / T;
+}
+__device__ __forceinline__ int piece_slot(int64_t w, int64_t seg_base, int64_t T, int64_t W) {
+  return static_cast<int>(w * 2 + (seg_base <= worker_start(w, T, W) ? 0 : 1));
+}
+
+// One 16-token sub-chunk for NT n-tiles of 8 heads: S^T = K Q^T, online softmax down the
+// token axis, O^T += V^T P^T.  kb/vb: shared addresses of the sub-chunk's swizzled K/V.
+template <int D, int NT>
+__device__ __forceinline__ void attend_subchunk(uint32_t kb, uint32_t vb, int nvalid,
+                                                const uint32_t (&kofs)[4], const uint32_t (&vofs)[4],
+                                                const uint32_t (&qf)[D / 16][NT][2],
+                                                float (&o)[D / 16][NT][4], float (&mref)[NT][2],
+                                                float (&lsum)[NT][2], float sl2, int g, int q) {
+  using G_ = Geo<D>;
+  constexpr int KS = D / 16;
+  constexpr int MT = D / 16;
+  float s[2][NT][4];
+#pragma unroll
+  for (int c = 0; c < 2; ++c)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) s[c][nt][0] = s[c][nt][1] = s[c][nt][2] = s[c][nt][3] = 0.f;
+#pragma unroll
+  for (int ks = 0; ks < KS; ++ks) {
+    uint32_t a[4];
+    ptx::ldmatrix_x4(kb + (ks >> 2) * G_::kBoxBytes + kofs[ks & 3], a[0], a[1], a[2], a[3]);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) ptx::mma_bf16_16816(s[ks & 1][nt], a, qf[ks][nt][0], qf[ks][nt][1]);
+  }
+  // c0,c1: token g, heads 2q, 2q+1;  c2,c3: token g + 8.
+  float sc[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) sc[nt][e] = (s[0][nt][e] + s[1][nt][e]) * sl2;
+  if (nvalid < kChunk) {
+    const bool v0 = g < nvalid, v1 = g + 8 < nvalid;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      if (!v0) sc[nt][0] = sc[nt][1] = -INFINITY;
+      if (!v1) sc[nt][2] = sc[nt][3] = -INFINITY;
+    }
+  }
+  float mx[NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      float m = fmaxf(sc[nt][e], sc[nt][e + 2]);
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+      mx[nt][e] = m;
+    }
+  bool need = false;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) need |= mx[nt][e] > mref[nt][e] + kRescaleThreshold;
+  if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float mn = fmaxf(mref[nt][e], mx[nt][e]);
+        const float alpha = (mn == mref[nt][e]) ? 1.f : ptx::ex2(mref[nt][e] - mn);
+        mref[nt][e] = mn;
+        lsum[nt][e] *= alpha;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          o[mt][nt][e] *= alpha;
+          o[mt][nt][e + 2] *= alpha;
+        }
+      }
+  }
+  uint32_t pb[NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const float mu0 = (mref[nt][0] == -INFINITY) ? 0.f : mref[nt][0];
+    const float mu1 = (mref[nt][1] == -INFINITY) ? 0.f : mref[nt][1];
+    const float p0 = ptx::ex2(sc[nt][0] - mu0), p1 = ptx::ex2(sc[nt][1] - mu1);
+    const float p2 = ptx::ex2(sc[nt][2] - mu0), p3 = ptx::ex2(sc[nt][3] - mu1);
+    lsum[nt][0] += p0 + p2;
+    lsum[nt][1] += p1 + p3;
+    pb[nt][0] = ptx::movmatrix_trans(ptx::pack_bf16x2(p0, p1));  // tokens 2q, 2q+1 of head g
+    pb[nt][1] = ptx::movmatrix_trans(ptx::pack_bf16x2(p2, p3));  // tokens 8 + 2q ..
+  }
+  // Slots past the sequence end may hold any bits (NaN included): their V words are
+  // zeroed in registers so 0 * NaN never reaches O.
+  uint32_t vm0 = 0xffffffffu, vm1 = 0xffffffffu;
+  if (nvalid < kChunk) {
+    const int t0 = 2 * q, t1 = 8 + 2 * q;
+    vm0 = (t0 < nvalid ? 0x0000ffffu : 0u) | (t0 + 1 < nvalid ? 0xffff0000u : 0u);
+    vm1 = (t1 < nvalid ? 0x0000ffffu : 0u) | (t1 + 1 < nvalid ? 0xffff0000u : 0u);
+  }
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) {
+    uint32_t a[4];
+    ptx::ldmatrix_x4_trans(vb + (mt >> 2) * G_::kBoxBytes + vofs[mt & 3], a[0], a[1], a[2], a[3]);
+    a[0] &= vm0;
+    a[1] &= vm0;
+    a[2] &= vm1;
+    a[3] &= vm1;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) ptx::mma_bf16_16816(o[mt][nt], a, pb[nt][0], pb[nt][1]);
+  }
+}
+
+}  // namespace
+
+// Launch shape: CTAs per SM for the token split (several producer warps per SM keep
+// more TMA copies in flight) and for the head split, and the per-SM shared-memory
+// budget shared by their rings and merge areas (overridable at compile time for
+// tuning sweeps).
+#ifndef GQA_CTAS_TOKEN_SPLIT
+#define GQA_CTAS_TOKEN_SPLIT 2
+#endif
+#ifndef GQA_CTAS_HEAD_SPLIT
+#define GQA_CTAS_HEAD_SPLIT 1
+#endif
+#ifndef GQA_SMEM_PER_SM_KB
+#define GQA_SMEM_PER_SM_KB 200
+#endif
+template <bool SPLIT_HEADS>
+constexpr int ctas_per_sm() { return SPLIT_HEADS ? GQA_CTAS_HEAD_SPLIT : GQA_CTAS_TOKEN_SPLIT; }
+
+// D: head_dim.  NT: 8-head n-tiles per consumer.  SPLIT_HEADS: consumers split the
+// query heads (else the 64 tokens of a stage).  C: consumer warps.  S: stages.
+template <int D, int NT, bool SPLIT_HEADS, int C, int S>
+__global__ void __launch_bounds__((C + 1) * 32, ctas_per_sm<SPLIT_HEADS>())
+decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                 const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
+  using G_ = Geo<D>;
+  constexpr int MT = D / 16;
+  constexpr int NH = 8 * NT;             // heads one consumer covers
+  constexpr int NCT = C * 32;            // consumer threads
+  static_assert(SPLIT_HEADS || C == kSubChunks, "token split needs one consumer per sub-chunk");
+
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ int64_t s_wtot[kMaxWarps];
+  __shared__ int s_start_b;
+  __shared__ int64_t s_start_base;
+  __shared__ int s_prev;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int nwarps = blockDim.x >> 5;
+  const int B = p.num_seqs;
+  const int segs = p.num_kv_heads * p.n_ht;
+  const int cap = p.max_blocks * p.page_size;
+
+  // ---------------------------------------------------------------- prologue
+  // Pass 1: total block count T (and zero rows of empty sequences).
+  int64_t mine = 0;
+  for (int b = threadIdx.x; b < B; b += blockDim.x) {
+    const int L = __ldg(p.seq_lens + b);
+    const int Le = eff_len(L, cap);
+    if ((L < 0 || L > cap) && blockIdx.x == 0) atomicOr(p.err, kErrBounds);
+    if (Le == 0 && (b % gridDim.x) == blockIdx.x) {
+      uint32_t* o = reinterpret_cast<uint32_t*>(p.out + static_cast<int64_t>(b) * p.num_heads * D);
+      for (int i = 0; i < p.num_heads * D / 2; ++i) o[i] = 0u;
+    }
+    mine += static_cast<int64_t>((Le + kBlock - 1) / kBlock) * segs;
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, off);
+  if (lane == 0) s_wtot[warp] = mine;
+  if (threadIdx.x == 0) s_start_b = -1;
+  __syncthreads();
+  int64_t T = 0;
+  for (int i = 0; i < nwarps; ++i) T += s_wtot[i];
+  // Only the first T CTAs get work when there are fewer blocks than CTAs, so every
+  // CTA in use owns at least one block and a segment's pieces come from exactly the
+  // CTAs worker_of(first block) .. worker_of(last block).
+  const int64_t W = min(static_cast<int64_t>(p.num_workers), T);
+  const int64_t w = blockIdx.x;
+  if (w >= W) return;  // (also covers T == 0)
+  const int64_t x0 = worker_start(w, T, W);
+  const int64_t x1 = worker_start(w + 1, T, W);
+  __syncthreads();  // s_wtot is reused below
+
+  // Pass 2: locate the sequence holding block x0 (tiled block scan).
+  {
+    int64_t base = 0;
+    for (int t0 = 0; t0 < B && base <= x0; t0 += blockDim.x) {
+      const int b = t0 + threadIdx.x;
+      int64_t n = 0;
+      if (b < B) n = static_cast<int64_t>((eff_len(__ldg(p.seq_lens + b), cap) + kBlock - 1) / kBlock) * segs;
+      int64_t incl = n;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int64_t v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+      }
+      if (lane == 31) s_wtot[warp] = incl;
+      __syncthreads();
+      int64_t pre = 0, tot = 0;
+      for (int i = 0; i < nwarps; ++i) {
+        if (i < warp) pre += s_wtot[i];
+        tot += s_wtot[i];
+      }
+      incl += pre;
+      const int64_t lo = base + incl - n, hi = base + incl;
+      if (n > 0 && x0 >= lo && x0 < hi) {
+        s_start_b = b;
+        s_start_base = lo;
+      }
+      base += tot;
+      __syncthreads();
+    }
+  }
+
+  // ---------------------------------------------------------------- shared layout
+  const uint32_t smem0 = ptx::smem_u32(smem_raw);
+  const uint32_t pad = (1024u - (smem0 & 1023u)) & 1023u;
+  uint8_t* base_ptr = smem_raw + pad;
+  const uint32_t ring = smem0 + pad;
+  constexpr int kMergeOs = SPLIT_HEADS ? 0 : C * NH * D;     // floats
+  constexpr int kMergeMl = SPLIT_HEADS ? 0 : 2 * C * NH * 2; // floats, double-buffered
+  float* os = reinterpret_cast<float*>(base_ptr + S * G_::kStageBytes);
+  float* mls = os + kMergeOs;
+  StageInfo* info = reinterpret_cast<StageInfo*>(mls + kMergeMl);
+  const uint32_t full_bar = ptx::smem_u32(info + S);
+  const uint32_t empty_bar = full_bar + 8 * S;
+
+  const int start_b = s_start_b;
+  const int64_t start_base = s_start_base;
+  if (start_b < 0) {  // cannot happen for a non-empty range; never index with it
+    if (threadIdx.x == 0) atomicOr(p.err, kErrBounds);
+    return;
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      ptx::mbar_init(full_bar + 8 * s, 1);
+      ptx::mbar_init(empty_bar + 8 * s, C);
+    }
+    ptx::fence_mbarrier_init();
+  }
+  __syncthreads();
+
+  const int64_t total = x1 - x0;
+  const uint64_t limit = p.wait_limit_ns;
+
+  Cursor cu;
+  cu.b = start_b;
+  cursor_load_seq(cu, p, cap);
+  {
+    const int64_t off = x0 - start_base;
+    cu.seg = static_cast<int>(off / cu.nblk);
+    cu.blk = static_cast<int>(off % cu.nblk);
+  }
+
+  if (warp == C) {
+    // ============================================================ producer warp
+    if (lane == 0) {
+      ptx::prefetch_tensormap(&tmap_k);
+      ptx::prefetch_tensormap(&tmap_v);
+    }
+    const uint64_t policy = ptx::policy_evict_first();
+    // Block-table rows are read 32 entries at a time (one per lane) into a register
+    // window, with the window needed next already in flight, so no TMA issue waits on
+    // a dependent global load.  Lane s < 4 owns sub-chunk s of every block.
+    const int ps = p.page_size;
+    auto load_window = [&](int b, int k) -> int {
+      const int e = 32 * k + lane;
+      return (b >= 0 && b < B && e < p.max_blocks)
+                 ? __ldg(p.block_table + static_cast<int64_t>(b) * p.max_blocks + e) : -1;
+    };
+    int wb = -1, wk = -1, wval = -1;  // window in use: row wb, entries [32 wk, 32 wk + 32)
+    int nb = -1, nk = -1, nval = -1;  // window prefetched next
+    // length of the sequence after cu.b, loaded ahead of the cursor reaching it
+    int next_len = (cu.b + 1 < B) ? __ldg(p.seq_lens + cu.b + 1) : 0;
+    auto prefetch_after = [&](const Cursor& c, int k) {
+      const int entries = (c.len + ps - 1) / ps;
+      if (32 * (k + 1) < entries) { nb = c.b; nk = k + 1; }
+      else if (c.seg + 1 < segs) { nb = c.b; nk = 0; }
+      else { nb = c.b + 1; nk = 0; }
+      nval = load_window(nb, nk);
+    };
+    auto page_of = [&](const Cursor& c) -> int {
+      const int e0 = (c.blk * kBlock) / ps;
+      const int k = e0 >> 5;
+      if (c.b != wb || k != wk) {
+        if (c.b == nb && k == nk) { wval = nval; }
+        else { wval = load_window(c.b, k); }
+        wb = c.b;
+        wk = k;
+        prefetch_after(c, k);
+      }
+      const int t = c.blk * kBlock + (lane & 3) * kChunk;
+      const int src = (t / ps) - 32 * k;  // 0..31: a block never straddles two windows
+      const int pg = __shfl_sync(0xffffffffu, wval, src);
+      return (lane < kSubChunks && t < c.len) ? pg : -1;
+    };
+    auto advance = [&](Cursor& c) {
+      if (++c.blk < c.nblk) return;
+      c.blk = 0;
+      if (++c.seg < segs) return;
+      c.seg = 0;
+      do {
+        ++c.b;
+        c.len = (c.b < B) ? eff_len(next_len, cap) : 0;
+        c.nblk = (c.len + kBlock - 1) / kBlock;
+        next_len = (c.b + 1 < B) ? __ldg(p.seq_lens + c.b + 1) : 0;
+      } while (c.nblk == 0 && c.b + 1 < B);
+    };
+    // Pull a piece's query rows into L2 ahead of the consumers that load them.
+    auto prefetch_q = [&](const Cursor& c) {
+      const int kvh = c.seg / p.n_ht, ht = c.seg % p.n_ht;
+      const int nrows = min(p.heads_per_seg, p.group - ht * p.heads_per_seg);
+      const uint8_t* q0 = reinterpret_cast<const uint8_t*>(
+          p.q + (static_cast<int64_t>(c.b) * p.num_heads + kvh * p.group + ht * p.heads_per_seg) * D);
+      for (int off = lane * 128; off < nrows * D * 2; off += 32 * 128) ptx::prefetch_l2(q0 + off);
+    };
+    int page = page_of(cu);
+    prefetch_q(cu);
+    int piece_blk0 = cu.blk;
+    bool first_piece = true;
+    int64_t seg_base = x0 - cu.blk;
+    for (int64_t i = 0; i < total; ++i) {
+      const int stage = static_cast<int>(i % S);
+      if (i >= S) {
+        const bool ok = ptx::mbar_wait_bounded(empty_bar + 8 * stage,
+                                               static_cast<uint32_t>((i / S - 1) & 1), limit);
+        if (!__all_sync(0xffffffffu, ok)) {
+          if (lane == 0) atomicOr(p.err, kErrTimeout);
+          // give copies still in flight a bounded chance to land, then leave
+          for (int64_t j = i - S; j < i; ++j)
+            ptx::mbar_wait_bounded(full_bar + 8 * (j % S), static_cast<uint32_t>((j / S) & 1), limit);
+          return;
+        }
+      }
+      const int nvalid = min(kBlock, cu.len - cu.blk * kBlock);
+      const bool want = lane < kSubChunks && lane * kChunk < nvalid;
+      const bool ok = want && page >= 0 && page < p.num_pages;
+      const uint32_t submask = __ballot_sync(0xffffffffu, ok) & 0xFu;
+      if (__any_sync(0xffffffffu, want && !ok) && lane == 0) atomicOr(p.err, kErrBounds);
+      const bool first = (i == 0) || cu.blk == 0;
+      const bool last = (i + 1 == total) || (cu.blk + 1 == cu.nblk);
+      if (first) piece_blk0 = cu.blk;
+      if (lane == 0) {
+        StageInfo& si = info[stage];
+        si.seg_base = seg_base;
+        si.b = cu.b;
+        si.seg = cu.seg;
+        si.blk = cu.blk;
+        si.nblk = cu.nblk;
+        si.nvalid = nvalid;
+        si.submask = static_cast<int>(submask);
+        si.flags = (first ? kFirstOfPiece : 0) | (last ? kLastOfPiece : 0) |
+                   ((last && piece_blk0 == 0 && cu.blk + 1 == cu.nblk) ? kSole : 0) |
+                   (first_piece ? kFirstPieceOfCta : 0);
+        const uint32_t bytes = static_cast<uint32_t>(__popc(submask)) * 2u * G_::kSubBytes;
+        if (bytes) ptx::mbar_arrive_expect_tx(full_bar + 8 * stage, bytes);
+        else ptx::mbar_arrive(full_bar + 8 * stage);
+      }
+      __syncwarp();
+      if (ok && !p.arm_without_copy) {
+        const int kvh = cu.seg / p.n_ht;
+        const int row = (page * p.num_kv_heads + kvh) * p.page_size +
+                        (cu.blk * kBlock + lane * kChunk) % p.page_size;
+        const uint32_t kdst = ring + stage * G_::kStageBytes + lane * G_::kSubBytes;
+        const uint32_t vdst = kdst + G_::kTileBytes;
+        const uint32_t bar = full_bar + 8 * stage;
+        // one copy per tensor brings all head_dim/64 column boxes of the 16 rows
+        ptx::tma_load_3d(kdst, &tmap_k, bar, 0, row, 0, policy);
+        ptx::tma_load_3d(vdst, &tmap_v, bar, 0, row, 0, policy);
+      }
+      if (last) first_piece = false;
+      if (i + 1 < total) {
+        advance(cu);
+        if (cu.blk == 0) {
+          seg_base = x0 + i + 1;
+          prefetch_q(cu);
+        }
+        page = page_of(cu);
+      }
+    }
+    return;
+  }
+
+  // ============================================================== consumer warps
+  const int j = warp;
+  const int g = lane >> 2;
+  const int q = lane & 3;
+  const int tid = threadIdx.x;  // 0 .. NCT-1
+  uint32_t kofs[4], vofs[4];
+  {
+    // K as the A operand: matrices (t0-7, d), (t8-15, d), (t0-7, d+8), (t8-15, d+8).
+    const int tokK = (lane & 7) + (((lane >> 3) & 1) << 3);
+    const int yK = (lane >> 4) ^ (lane & 7);
+    // V^T as the A operand: matrices (t0-7, d), (t0-7, d+8), (t8-15, d), (t8-15, d+8).
+    const int tokV = (lane & 7) + ((lane >> 4) << 3);
+    const int yV = ((lane >> 3) & 1) ^ (lane & 7);
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      kofs[jj] = static_cast<uint32_t>(tokK * 128 + (((2 * jj) ^ yK) << 4));
+      vofs[jj] = static_cast<uint32_t>(tokV * 128 + (((2 * jj) ^ yV) << 4));
+    }
+  }
+
+  uint32_t qf[MT][NT][2];
+  float o[MT][NT][4];
+  float mref[NT][2], lsum[NT][2];
+  int nrows_seg = 0;  // valid heads of the segment
+  int nrows_c = 0;    // valid heads of this consumer's tile
+  int hoff_c = 0;     // first segment-relative head of this consumer's tile
+  const float sl2 = p.scale_log2;
+  int piece_parity = 0;
+
+  auto load_q = [&](int b, int seg) {
+    const int kvh = seg / p.n_ht;
+    const int ht = seg % p.n_ht;
+    nrows_seg = min(p.heads_per_seg, p.group - ht * p.heads_per_seg);
+    hoff_c = SPLIT_HEADS ? j * NH : 0;
+    nrows_c = max(0, min(NH, nrows_seg - hoff_c));
+    const int head0 = kvh * p.group + ht * p.heads_per_seg + hoff_c;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int h = nt * 8 + g;
+      const bool v = h < nrows_c;
+      const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
+          p.q + (static_cast<int64_t>(b) * p.num_heads + head0 + (v ? h : 0)) * D);
+#pragma unroll
+      for (int ks = 0; ks < MT; ++ks) {
+        qf[ks][nt][0] = v ? __ldg(qrow + ks * 8 + q) : 0u;
+        qf[ks][nt][1] = v ? __ldg(qrow + ks * 8 + 4 + q) : 0u;
+      }
+    }
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) o[mt][nt][0] = o[mt][nt][1] = o[mt][nt][2] = o[mt][nt][3] = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      mref[nt][0] = mref[nt][1] = -INFINITY;
+      lsum[nt][0] = lsum[nt][1] = 0.f;
+    }
+  };
+
+  // Cross-CTA step of a piece that is not the whole segment: all consumer threads have
+  // stored this CTA's piece; the last CTA to arrive merges every piece into out.
+  auto cross_cta = [&](const StageInfo& si) {
+    __threadfence();
+    ptx::named_barrier_sync(1, NCT);
+    const int64_t segid = static_cast<int64_t>(si.b) * segs + si.seg;
+    if (tid == 0) s_prev = atomicAdd(p.counters + segid, 1);
+    ptx::named_barrier_sync(1, NCT);
+    const int prev = s_prev;
+    const int64_t wf = worker_of(si.seg_base, T, W);
+    const int64_t wl = worker_of(si.seg_base + si.nblk - 1, T, W);
+    if (prev != static_cast<int>(wl - wf)) return;
+    __threadfence();
+    const int hps = p.heads_per_seg;
+    const int kvh = si.seg / p.n_ht;
+    const int ht = si.seg % p.n_ht;
+    const int64_t row0 = static_cast<int64_t>(si.b) * p.num_heads + kvh * p.group + ht * hps;
+    for (int idx = tid; idx < nrows_seg * D; idx += NCT) {
+      const int h = idx / D, d = idx - (idx / D) * D;
+      float M = -INFINITY, L = 0.f, acc = 0.f;
+      int64_t ww = wf;
+      for (; ww + 3 <= wl; ww += 4) {
+        float2 ml[4];
+        float ov[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int sl = piece_slot(ww + k, si.seg_base, T, W);
+          ml[k] = __ldcg(reinterpret_cast<const float2*>(p.part_ml + (static_cast<int64_t>(sl) * hps + h) * 2));
+          ov[k] = __ldcg(p.part_o + (static_cast<int64_t>(sl) * hps + h) * D + d);
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float mn = fmaxf(M, ml[k].x);
+          const float mu = (mn == -INFINITY) ? 0.f : mn;
+          const float a = ptx::ex2(M - mu), bw = ptx::ex2(ml[k].x - mu);
+          L = L * a + ml[k].y * bw;
+          acc = acc * a + ov[k] * bw;
+          M = mn;
+        }
+      }
+      for (; ww <= wl; ++ww) {
+        const int sl = piece_slot(ww, si.seg_base, T, W);
+        const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.part_ml + (static_cast<int64_t>(sl) * hps + h) * 2));
+        const float ov = __ldcg(p.part_o + (static_cast<int64_t>(sl) * hps + h) * D + d);
+        const float mn = fmaxf(M, ml.x);
+        const float mu = (mn == -INFINITY) ? 0.f : mn;
+        const float a = ptx::ex2(M - mu), bw = ptx::ex2(ml.x - mu);
+        L = L * a + ml.y * bw;
+        acc = acc * a + ov * bw;
+        M = mn;
+      }
+      reinterpret_cast<__nv_bfloat16*>(p.out)[(row0 + h) * D + d] =
+          __float2bfloat16_rn(L > 0.f ? acc / L : 0.f);
+    }
+    if (tid == 0) p.counters[segid] = 0;
+  };
+
+  for (int64_t i = 0; i < total; ++i) {
+    const int stage = static_cast<int>(i % S);
+    const bool arrived = ptx::mbar_wait_bounded(full_bar + 8 * stage, static_cast<uint32_t>((i / S) & 1), limit);
+    if (!__all_sync(0xffffffffu, arrived)) {
+      if (lane == 0) atomicOr(p.err, kErrTimeout);
+      return;
+    }
+    const StageInfo si = info[stage];
+    if (si.flags & kFirstOfPiece) load_q(si.b, si.seg);
+
+    const uint32_t kst = ring + stage * G_::kStageBytes;
+    if constexpr (SPLIT_HEADS) {
+      if (nrows_c > 0) {
+#pragma unroll 1
+        for (int sc = 0; sc < kSubChunks; ++sc) {
+          if ((si.submask >> sc) & 1) {
+            const uint32_t kb = kst + sc * G_::kSubBytes;
+            attend_subchunk<D, NT>(kb, kb + G_::kTileBytes, min(kChunk, si.nvalid - sc * kChunk),
+                                   kofs, vofs, qf, o, mref, lsum, sl2, g, q);
+          }
+        }
+      }
+    } else {
+      if ((si.submask >> j) & 1) {
+        const uint32_t kb = kst + j * G_::kSubBytes;
+        attend_subchunk<D, NT>(kb, kb + G_::kTileBytes, min(kChunk, si.nvalid - j * kChunk),
+                               kofs, vofs, qf, o, mref, lsum, sl2, g, q);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(empty_bar + 8 * stage);
+
+    if (!(si.flags & kLastOfPiece)) continue;
+
+    // ------------------------------------------------------------ end of a piece
+    float lt[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        float l = lsum[nt][e];
+        l += __shfl_xor_sync(0xffffffffu, l, 4);
+        l += __shfl_xor_sync(0xffffffffu, l, 8);
+        l += __shfl_xor_sync(0xffffffffu, l, 16);
+        lt[nt][e] = l;
+      }
+    const bool sole = si.flags & kSole;
+    const int hps = p.heads_per_seg;
+    const int kvh = si.seg / p.n_ht;
+    const int ht = si.seg % p.n_ht;
+    const int64_t row0 = static_cast<int64_t>(si.b) * p.num_heads + kvh * p.group + ht * hps;
+    const int slot = static_cast<int>(w * 2 + ((si.flags & kFirstPieceOfCta) ? 0 : 1));
+
+    if constexpr (SPLIT_HEADS) {
+      // Each consumer owns its heads over every token: write them directly.
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int h = nt * 8 + 2 * q + e;  // within this consumer's tile
+          if (h < nrows_c) {
+            const int hs = hoff_c + h;         // within the segment
+            if (sole) {
+              const float inv = lt[nt][e] > 0.f ? 1.f / lt[nt][e] : 0.f;
+              __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + (row0 + hs) * D;
+#pragma unroll
+              for (int mt = 0; mt < MT; ++mt) {
+                dst[mt * 16 + g] = __float2bfloat16_rn(o[mt][nt][e] * inv);
+                dst[mt * 16 + g + 8] = __float2bfloat16_rn(o[mt][nt][e + 2] * inv);
+              }
+            } else {
+              float* po = p.part_o + (static_cast<int64_t>(slot) * hps + hs) * D;
+#pragma unroll
+              for (int mt = 0; mt < MT; ++mt) {
+                po[mt * 16 + g] = o[mt][nt][e];
+                po[mt * 16 + g + 8] = o[mt][nt][e + 2];
+              }
+              if (g == 0)
+                *reinterpret_cast<float2*>(p.part_ml + (static_cast<int64_t>(slot) * hps + hs) * 2) =
+                    make_float2(mref[nt][e], lt[nt][e]);
+            }
+          }
+        }
+      if (!sole) cross_cta(si);
+    } else {
+      // Token split: combine the C consumers' partial states in shared memory.
+      float* ml = mls + piece_parity * (C * NH * 2);
+      piece_parity ^= 1;
+      if (g == 0) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int h = nt * 8 + 2 * q + e;
+            ml[(j * NH + h) * 2] = mref[nt][e];
+            ml[(j * NH + h) * 2 + 1] = lt[nt][e];
+          }
+      }
+      ptx::named_barrier_sync(1, NCT);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int h = nt * 8 + 2 * q + e;
+          float M = -INFINITY;
+#pragma unroll
+          for (int jj = 0; jj < C; ++jj) M = fmaxf(M, ml[(jj * NH + h) * 2]);
+          const float wgt = (mref[nt][e] == -INFINITY) ? 0.f : ptx::ex2(mref[nt][e] - M);
+          float* dst = os + (j * NH + h) * D;
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt) {
+            dst[mt * 16 + g] = o[mt][nt][e] * wgt;
+            dst[mt * 16 + g + 8] = o[mt][nt][e + 2] * wgt;
+          }
+        }
+      ptx::named_barrier_sync(1, NCT);
+      for (int idx = tid; idx < nrows_seg * D; idx += NCT) {
+        const int h = idx / D, d = idx - (idx / D) * D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int jj = 0; jj < C; ++jj) M = fmaxf(M, ml[(jj * NH + h) * 2]);
+        float L = 0.f, acc = 0.f;
+#pragma unroll
+        for (int jj = 0; jj < C; ++jj) {
+          const float mj = ml[(jj * NH + h) * 2];
+          if (mj != -INFINITY) L += ml[(jj * NH + h) * 2 + 1] * ptx::ex2(mj - M);
+          acc += os[(jj * NH + h) * D + d];
+        }
+        if (sole) {
+          reinterpret_cast<__nv_bfloat16*>(p.out)[(row0 + h) * D + d] =
+              __float2bfloat16_rn(L > 0.f ? acc / L : 0.f);
+        } else {
+          p.part_o[(static_cast<int64_t>(slot) * hps + h) * D + d] = acc;
+          if (d == 0)
+            *reinterpret_cast<float2*>(p.part_ml + (static_cast<int64_t>(slot) * hps + h) * 2) =
+                make_float2(M, L);
+        }
+      }
+      if (!sole) cross_cta(si);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ host side
+namespace {
+
+
+template <int D, int NT, bool SPLIT_HEADS, int C>
+struct Cfg {
+  static constexpr int kNH = 8 * NT;
+  static constexpr size_t kMerge =
+      SPLIT_HEADS ? 0 : (static_cast<size_t>(C) * kNH * D + 2 * C * kNH * 2) * sizeof(float);
+  static constexpr size_t kBudget =
+      static_cast<size_t>(GQA_SMEM_PER_SM_KB) * 1024 / ctas_per_sm<SPLIT_HEADS>();
+  static constexpr int kStagesRaw = static_cast<int>((kBudget - kMerge) / Geo<D>::kStageBytes);
+  static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+  static constexpr size_t kSmem = 1024 + static_cast<size_t>(kStages) * Geo<D>::kStageBytes + kMerge +
+                                  kStages * (sizeof(StageInfo) + 16);
+};
+
+template <int D, int NT, bool SH, int C>
+cudaError_t launch_t(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int grid,
+                     cudaStream_t stream) {
+  using CF = Cfg<D, NT, SH, C>;
+  auto kern = decode_ws_kernel<D, NT, SH, C, CF::kStages>;
+  static thread_local int configured_device = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_device != dev) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(CF::kSmem));
+    if (e != cudaSuccess) return e;
+    configured_device = dev;
+  }
+  kern<<<grid, (C + 1) * 32, CF::kSmem, stream>>>(tk, tv, p);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_d(const DecodeParams& p, const DecodePlan& pl, const CUtensorMap& tk,
+                     const CUtensorMap& tv, int grid, cudaStream_t s) {
+  if (!pl.split_heads)
+    return pl.n_tiles == 1 ? launch_t<D, 1, false, 4>(p, tk, tv, grid, s)
+                           : launch_t<D, 2, false, 4>(p, tk, tv, grid, s);
+  if (pl.n_tiles == 1) {
+    switch (pl.consumers) {
+      case 3: return launch_t<D, 1, true, 3>(p, tk, tv, grid, s);
+      default: return launch_t<D, 1, true, 4>(p, tk, tv, grid, s);
+    }
+  }
+  switch (pl.consumers) {
+    case 3: return launch_t<D, 2, true, 3>(p, tk, tv, grid, s);
+    case 4: return launch_t<D, 2, true, 4>(p, tk, tv, grid, s);
+    case 5: return launch_t<D, 2, true, 5>(p, tk, tv, grid, s);
+    case 6: return launch_t<D, 2, true, 6>(p, tk, tv, grid, s);
+    case 7: return launch_t<D, 2, true, 7>(p, tk, tv, grid, s);
+    default: return launch_t<D, 2, true, 8>(p, tk, tv, grid, s);
+  }
+}
+
+template <int D, int NT, bool SH, int C>
+void fill(DecodePlan& pl) {
+  using CF = Cfg<D, NT, SH, C>;
+  pl.stages = CF::kStages;
+  pl.smem_bytes = CF::kSmem;
+}
+
+}  // namespace
+
+// Small groups (G <= 16): token split, 4 consumers, one 8- or 16-head tile per segment.
+// Larger groups: head split; 8 heads per consumer up to G = 32, else 16, and up to 8
+// consumers, so one segment covers up to 128 query heads of its kv head.
+DecodePlan plan_decode(int head_dim, int group) {
+  DecodePlan pl{};
+  if (group <= 16) {
+    pl.split_heads = 0;
+    pl.n_tiles = group <= 8 ? 1 : 2;
+    pl.consumers = 4;
+    pl.heads_per_seg = 8 * pl.n_tiles;
+  } else {
+    pl.split_heads = 1;
+    pl.n_tiles = group <= 32 ? 1 : 2;
+    const int hg = 8 * pl.n_tiles;
+    int c = (group + hg - 1) / hg;
+    if (pl.n_tiles == 1) c = c <= 3 ? 3 : 4;   // 17..24 -> 3, 25..32 -> 4
+    else c = c < 3 ? 3 : (c > 8 ? 8 : c);
+    pl.consumers = c;
+    pl.heads_per_seg = hg * c;
+  }
+  pl.n_ht = (group + pl.heads_per_seg - 1) / pl.heads_per_seg;
+  pl.ctas_per_sm = pl.split_heads ? ctas_per_sm<true>() : ctas_per_sm<false>();
+  const bool sh = pl.split_heads;
+  const int nt = pl.n_tiles, c = pl.consumers;
+  if (head_dim == 64) {
+    if (!sh) { if (nt == 1) fill<64, 1, false, 4>(pl); else fill<64, 2, false, 4>(pl); }
+    else if (nt == 1) { if (c == 3) fill<64, 1, true, 3>(pl); else fill<64, 1, true, 4>(pl); }
+    else fill<64, 2, true, 8>(pl);  // stage count does not depend on C for the head split
+  } else {
+    if (!sh) { if (nt == 1) fill<128, 1, false, 4>(pl); else fill<128, 2, false, 4>(pl); }
+    else if (nt == 1) { if (c == 3) fill<128, 1, true, 3>(pl); else fill<128, 1, true, 4>(pl); }
+    else fill<128, 2, true, 8>(pl);
+  }
+  return pl;
+}
+
+cudaError_t launch_decode(const DecodeParams& p, const DecodePlan& pl, const CUtensorMap& tk,
+                          const CUtensorMap& tv, int grid, cudaStream_t stream) {
+  if (p.head_dim == 64) return launch_d<64>(p, pl, tk, tv, grid, stream);
+  return launch_d<128>(p, pl, tk, tv, grid, stream);
+}
+
+}  // namespace gqa

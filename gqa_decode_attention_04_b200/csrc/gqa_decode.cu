@@ -48,7 +48,8 @@ struct DeviceState {
   size_t counters_cap = 0;  // entries
   float* part_o = nullptr;
   float* part_ml = nullptr;
-  size_t slots_cap = 0;     // partial slots (each kHeadTile rows x 128 floats)
+  size_t part_o_cap = 0;    // floats
+  size_t part_ml_cap = 0;   // floats
 };
 
 std::mutex g_mu;
@@ -75,7 +76,8 @@ gqa_status get_state(DeviceState** out, int* dev_out) {
 
 // Grow-only decode workspace.  Counters must be zero between launches: they are
 // zeroed when allocated and every launch leaves them zero.
-gqa_status ensure_workspace(DeviceState& s, size_t counters, size_t slots, cudaStream_t stream) {
+gqa_status ensure_workspace(DeviceState& s, size_t counters, size_t part_o_floats,
+                            size_t part_ml_floats, cudaStream_t stream) {
   std::lock_guard<std::mutex> lk(g_mu);
   cudaError_t e;
   if (counters > s.counters_cap) {
@@ -89,16 +91,21 @@ gqa_status ensure_workspace(DeviceState& s, size_t counters, size_t slots, cudaS
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(split counters)");
     s.counters_cap = n;
   }
-  if (slots > s.slots_cap) {
+  if (part_o_floats > s.part_o_cap) {
     if (s.part_o) cudaFree(s.part_o);
+    s.part_o = nullptr;
+    s.part_o_cap = 0;
+    e = cudaMalloc(&s.part_o, part_o_floats * sizeof(float));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(split partials)");
+    s.part_o_cap = part_o_floats;
+  }
+  if (part_ml_floats > s.part_ml_cap) {
     if (s.part_ml) cudaFree(s.part_ml);
-    s.part_o = s.part_ml = nullptr;
-    s.slots_cap = 0;
-    e = cudaMalloc(&s.part_o, slots * gqa::kHeadTile * 128 * sizeof(float));
+    s.part_ml = nullptr;
+    s.part_ml_cap = 0;
+    e = cudaMalloc(&s.part_ml, part_ml_floats * sizeof(float));
     if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(split partials)");
-    e = cudaMalloc(&s.part_ml, slots * gqa::kHeadTile * 2 * sizeof(float));
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMalloc(split partials)");
-    s.slots_cap = slots;
+    s.part_ml_cap = part_ml_floats;
   }
   return GQA_OK;
 }
@@ -122,8 +129,10 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// The pool [num_pages, Hk, ps, D] viewed as a 2-D bf16 tensor of P*Hk*ps rows and D
-// columns; one box is 16 rows (one chunk) x 64 columns (128 bytes), 128-byte swizzle.
+// The pool [num_pages, Hk, ps, D] viewed as a 3-D bf16 tensor: 64 columns (128 bytes)
+// x P*Hk*ps rows x D/64 column groups (stride 128 bytes).  One box is 64 columns x 16
+// rows (one sub-chunk) x all D/64 groups, 128-byte swizzle; in shared memory it lands
+// as D/64 consecutive [16, 64] tiles.
 struct MapKey {
   const void* ptr;
   int64_t rows;
@@ -146,11 +155,11 @@ gqa_status make_pool_map(CUtensorMap* m, const void* pool, int64_t rows, int d, 
     }
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return fail(GQA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
-  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(gqa::kChunk)};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(pool), dims, strides,
+  cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(d / 64)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, 128};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(gqa::kChunk), static_cast<cuuint32_t>(d / 64)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(pool), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(GQA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
@@ -266,21 +275,22 @@ gqa_status gqa_paged_decode_attn(const void* q, const void* k_pages, const void*
   cudaStream_t strm = static_cast<cudaStream_t>(stream);
 
   const int group = num_heads / num_kv_heads;
-  const int n_ht = (group + gqa::kHeadTile - 1) / gqa::kHeadTile;
-  const gqa::DecodeLaunch cfg = gqa::decode_launch_config(head_dim, group);
-  // Upper bound on the chunk count (seq_lens are device data).
-  const int64_t chunks_per_seq =
-      static_cast<int64_t>(max_blocks_per_seq) * (page_size / gqa::kChunk);
-  const int64_t max_chunks = static_cast<int64_t>(num_seqs) * num_kv_heads * n_ht * chunks_per_seq;
-  int64_t workers = static_cast<int64_t>(st->sms) * cfg.ctas_per_sm * cfg.warps_per_cta;
+  const gqa::DecodePlan plan = gqa::plan_decode(head_dim, group);
+  // Upper bound on the block count (seq_lens are device data).
+  const int64_t blocks_per_seq =
+      (static_cast<int64_t>(max_blocks_per_seq) * page_size + gqa::kBlock - 1) / gqa::kBlock;
+  const int64_t max_blocks = static_cast<int64_t>(num_seqs) * num_kv_heads * plan.n_ht * blocks_per_seq;
+  int64_t workers = static_cast<int64_t>(st->sms) * plan.ctas_per_sm;
   const int forced = g_num_workers.load();
   if (forced > 0) workers = forced;
-  if (workers > max_chunks) workers = max_chunks;
+  if (workers > max_blocks) workers = max_blocks;
   if (workers < 1) workers = 1;
-  const int grid = static_cast<int>((workers + cfg.warps_per_cta - 1) / cfg.warps_per_cta);
+  const int grid = static_cast<int>(workers);
 
-  const size_t segments = static_cast<size_t>(num_seqs) * num_kv_heads * n_ht;
-  s = ensure_workspace(*st, segments, static_cast<size_t>(2 * workers), strm);
+  const size_t segments = static_cast<size_t>(num_seqs) * num_kv_heads * plan.n_ht;
+  const size_t slots = static_cast<size_t>(2 * workers);
+  s = ensure_workspace(*st, segments, slots * plan.heads_per_seg * head_dim,
+                       slots * plan.heads_per_seg * 2, strm);
   if (s != GQA_OK) return s;
 
   CUtensorMap tk, tv;
@@ -302,7 +312,8 @@ gqa_status gqa_paged_decode_attn(const void* q, const void* k_pages, const void*
   p.num_heads = num_heads;
   p.num_kv_heads = num_kv_heads;
   p.group = group;
-  p.n_ht = n_ht;
+  p.n_ht = plan.n_ht;
+  p.heads_per_seg = plan.heads_per_seg;
   p.page_size = page_size;
   p.max_blocks = max_blocks_per_seq;
   p.num_pages = num_pages;
@@ -311,7 +322,7 @@ gqa_status gqa_paged_decode_attn(const void* q, const void* k_pages, const void*
   p.num_workers = static_cast<int>(workers);
   p.wait_limit_ns = static_cast<uint64_t>(g_wait_limit_ns.load());
   p.arm_without_copy = g_arm_without_copy.load();
-  cudaError_t e = gqa::launch_decode(p, tk, tv, grid, strm);
+  cudaError_t e = gqa::launch_decode(p, plan, tk, tv, grid, strm);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   g_launches.fetch_add(1);
   return GQA_OK;

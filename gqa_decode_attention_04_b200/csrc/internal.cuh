@@ -13,27 +13,30 @@ enum : uint32_t {
   kErrTimeout = 2u,  // a bounded wait ran out: work skipped
 };
 
-// Tokens per pipeline chunk: every supported page size is a multiple of it, so a
-// chunk never straddles two pages and is one contiguous [16, head_dim] tile of
+// Tokens per TMA sub-chunk: every supported page size is a multiple of it, so a
+// sub-chunk never straddles two pages and is one contiguous [16, head_dim] tile of
 // one (page, kv head).
 constexpr int kChunk = 16;
-
-// Query heads handled per head tile (the M dimension of one m16n8k16 MMA).
-constexpr int kHeadTile = 16;
+// Tokens per pipeline stage (four sub-chunks): the unit the work list is cut into.
+constexpr int kBlock = 64;
+constexpr int kSubChunks = kBlock / kChunk;
+// Most query heads one segment (kv head x head tile) covers; partial slots hold this many.
+constexpr int kMaxSegHeads = 128;
 
 struct DecodeParams {
   const uint16_t* q;          // [B, H, D] bf16
   uint16_t* out;              // [B, H, D] bf16
   const int32_t* block_table; // [B, MB]
   const int32_t* seq_lens;    // [B]
-  float* part_o;              // [2 * num_workers, kHeadTile, D] fp32 (unnormalised)
-  float* part_ml;             // [2 * num_workers, kHeadTile, 2] fp32 (max, sum), log2 domain
+  float* part_o;              // [2 * num_workers, heads_per_seg, D] fp32 (unnormalised)
+  float* part_ml;             // [2 * num_workers, heads_per_seg, 2] fp32 (ref max, sum), log2
   int32_t* counters;          // [B * Hk * n_ht], zero between launches
   uint32_t* err;              // device error word
   int num_seqs, num_heads, num_kv_heads, group, n_ht, page_size, max_blocks, num_pages;
   int head_dim;
+  int heads_per_seg;          // query heads one segment covers
   float scale_log2;           // scale * log2(e)
-  int num_workers;
+  int num_workers;            // CTAs the work list is split over
   uint64_t wait_limit_ns;
   int arm_without_copy;
 };
@@ -52,15 +55,20 @@ struct AppendParams {
 // Launchers (return the cudaError_t of the launch).
 cudaError_t launch_kv_append(const AppendParams& p, cudaStream_t stream);
 
-struct DecodeLaunch {
-  int warps_per_cta;
+// How a (head_dim, group) problem is mapped onto the decode kernel.
+struct DecodePlan {
+  int split_heads;    // 0: consumers split the 64-token stage by tokens; 1: by query heads
+  int n_tiles;        // 8-head MMA n-tiles per consumer
+  int consumers;      // consumer (MMA) warps per CTA; one producer warp is added
+  int heads_per_seg;  // query heads a segment covers
+  int n_ht;           // segments per kv head
+  int stages;         // pipeline stages per CTA
   int ctas_per_sm;
   size_t smem_bytes;
 };
 
-// Kernel configuration for a head_dim / group combination.
-DecodeLaunch decode_launch_config(int head_dim, int group);
-cudaError_t launch_decode(const DecodeParams& p, const CUtensorMap& tmap_k,
+DecodePlan plan_decode(int head_dim, int group);
+cudaError_t launch_decode(const DecodeParams& p, const DecodePlan& plan, const CUtensorMap& tmap_k,
                           const CUtensorMap& tmap_v, int grid, cudaStream_t stream);
 
 }  // namespace gqa
