@@ -22,6 +22,7 @@ __all__ = [
     "load_library",
     "kv_append",
     "paged_decode_attn",
+    "paged_decode_attn_noalloc",
     "check_device_error",
     "kv_cache_bytes",
     "set_num_workers",
@@ -41,6 +42,7 @@ STATUS_NAMES = {0: "GQA_OK", -1: "GQA_ERR_INVALID_ARG", -2: "GQA_ERR_UNSUPPORTED
 EXPORTED_SYMBOLS = (
     "gqa_kv_append",
     "gqa_paged_decode_attn",
+    "gqa_paged_decode_attn_noalloc",
     "gqa_check_device_error",
     "gqa_last_error_string",
     "gqa_kv_cache_bytes",
@@ -81,6 +83,8 @@ def load_library() -> ctypes.CDLL:
     lib.gqa_paged_decode_attn.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32,
                                           i32, i32, vp]
     lib.gqa_paged_decode_attn.restype = i32
+    lib.gqa_paged_decode_attn_noalloc.argtypes = lib.gqa_paged_decode_attn.argtypes
+    lib.gqa_paged_decode_attn_noalloc.restype = i32
     lib.gqa_check_device_error.argtypes = [vp]
     lib.gqa_check_device_error.restype = i32
     lib.gqa_last_error_string.argtypes = []
@@ -174,6 +178,37 @@ def paged_decode_attn(q, k_pages, v_pages, block_table, seq_lens, out: Optional[
                                          block_table.data_ptr(), seq_lens.data_ptr(), out.data_ptr(),
                                          B, H, Hk, D, ps, float(scale), block_table.shape[1], P,
                                          _stream_ptr(stream)))
+    return out
+
+
+def paged_decode_attn_noalloc(q, k_pages, v_pages, block_table, seq_lens, out: torch.Tensor,
+                              scale: Optional[float] = None, stream=None) -> torch.Tensor:
+    """paged_decode_attn without any device allocation, for callers that cannot allocate
+    (their engine owns all device memory, or allocation's synchronisation is too costly).
+
+    Scratch is a fixed array inside the library, shared by every call: calls that
+    overlap on the GPU race, and the first call on a device should come before any
+    stream capture.  `out` must be given.  Device-side range errors are not reported.
+    """
+    dev = q.device
+    for t, n, dt in ((q, "q", torch.bfloat16), (k_pages, "k_pages", torch.bfloat16),
+                     (v_pages, "v_pages", torch.bfloat16), (block_table, "block_table", torch.int32),
+                     (seq_lens, "seq_lens", torch.int32), (out, "out", torch.bfloat16)):
+        _need(t, n, dt, dev)
+    B, H, D = q.shape
+    P, Hk, ps, D2 = k_pages.shape
+    if D2 != D or tuple(v_pages.shape) != (P, Hk, ps, D) or tuple(out.shape) != (B, H, D):
+        raise ValueError("shapes must match paged_decode_attn's")
+    if block_table.dim() != 2 or block_table.shape[0] != B or tuple(seq_lens.shape) != (B,):
+        raise ValueError("block_table must be [num_seqs, max_blocks], seq_lens [num_seqs]")
+    if scale is None:
+        scale = 1.0 / (D ** 0.5)
+    lib = load_library()
+    with torch.cuda.device(dev):
+        _check(lib.gqa_paged_decode_attn_noalloc(
+            q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(), block_table.data_ptr(),
+            seq_lens.data_ptr(), out.data_ptr(), B, H, Hk, D, ps, float(scale),
+            block_table.shape[1], P, _stream_ptr(stream)))
     return out
 
 

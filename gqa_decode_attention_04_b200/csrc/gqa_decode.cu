@@ -171,6 +171,46 @@ gqa_status make_pool_map(CUtensorMap* m, const void* pool, int64_t rows, int d, 
 
 }  // namespace
 
+// ------------------------------------------------------------------ allocation-free decode
+// Scratch of gqa_paged_decode_attn_noalloc: a fixed array in the library's device
+// image, present on every GPU that loads the library until the process exits, so the
+// call never has to allocate.  Layout per call: the device error word (first 256
+// bytes), one arrival counter per segment, then the split partials (reference max and
+// sum, then unnormalised O) of two slots per worker.
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t{16} << 20;  // 16 MiB
+constexpr size_t kNoAllocHeaderBytes = 256;
+constexpr size_t kNoAllocMaxSegments = 16384;             // num_seqs * num_kv_heads * head tiles
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+std::mutex g_noalloc_mu;
+std::unordered_map<int, std::pair<unsigned char*, int>> g_noalloc_dev;  // device -> (address, SMs)
+
+// Host code only holds a stand-in for g_noalloc_scratch; its device address is looked
+// up once per device, with that device current.
+gqa_status noalloc_scratch(int dev, unsigned char** ptr, int* sms) {
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  auto it = g_noalloc_dev.find(dev);
+  if (it == g_noalloc_dev.end()) {
+    void* addr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&addr, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(allocation-free scratch)");
+    int n = 0;
+    e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    it = g_noalloc_dev.emplace(dev, std::make_pair(static_cast<unsigned char*>(addr), n)).first;
+  }
+  *ptr = it->second.first;
+  *sms = it->second.second;
+  return GQA_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t{255}; }
+}  // namespace
+
 extern "C" {
 
 const char* gqa_last_error_string(void) { return g_err_msg; }
@@ -323,6 +363,116 @@ gqa_status gqa_paged_decode_attn(const void* q, const void* k_pages, const void*
   p.wait_limit_ns = static_cast<uint64_t>(g_wait_limit_ns.load());
   p.arm_without_copy = g_arm_without_copy.load();
   cudaError_t e = gqa::launch_decode(p, plan, tk, tv, grid, strm);
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  g_launches.fetch_add(1);
+  return GQA_OK;
+}
+
+gqa_status gqa_paged_decode_attn_noalloc(const void* q, const void* k_pages, const void* v_pages,
+                                         const int32_t* block_table, const int32_t* seq_lens,
+                                         void* out, int num_seqs, int num_heads, int num_kv_heads,
+                                         int head_dim, int page_size, float scale,
+                                         int max_blocks_per_seq, int num_pages, void* stream) {
+  if (num_seqs < 0) return fail(GQA_ERR_INVALID_ARG, "num_seqs < 0");
+  if (num_heads < 1 || num_kv_heads < 1 || head_dim < 1 || page_size < 1 ||
+      max_blocks_per_seq < 1 || num_pages < 1)
+    return fail(GQA_ERR_INVALID_ARG, "sizes must be positive");
+  if (num_heads % num_kv_heads != 0)
+    return fail(GQA_ERR_INVALID_ARG, "num_heads (%d) is not a multiple of num_kv_heads (%d)",
+                num_heads, num_kv_heads);
+  if (head_dim != 64 && head_dim != 128)
+    return fail(GQA_ERR_UNSUPPORTED, "head_dim %d not built (64, 128)", head_dim);
+  if (page_size % gqa::kChunk != 0 || page_size > 256)
+    return fail(GQA_ERR_UNSUPPORTED, "page_size %d not built (multiple of 16, <= 256)", page_size);
+  if (!std::isfinite(scale)) return fail(GQA_ERR_INVALID_ARG, "scale is not finite");
+  const int64_t rows = static_cast<int64_t>(num_pages) * num_kv_heads * page_size;
+  if (rows >= (int64_t{1} << 31))
+    return fail(GQA_ERR_UNSUPPORTED, "num_pages * num_kv_heads * page_size exceeds 2^31");
+  if (static_cast<int64_t>(max_blocks_per_seq) * page_size >= (int64_t{1} << 31))
+    return fail(GQA_ERR_UNSUPPORTED, "max_blocks_per_seq * page_size exceeds 2^31");
+  if (num_seqs == 0) return GQA_OK;
+  if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !out)
+    return fail(GQA_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned(k_pages, 16) || !aligned(v_pages, 16))
+    return fail(GQA_ERR_INVALID_ARG, "k_pages / v_pages must be 16-byte aligned");
+  if (!aligned(q, 4) || !aligned(out, 8))
+    return fail(GQA_ERR_INVALID_ARG, "q must be 4-byte and out 8-byte aligned");
+
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  unsigned char* scratch = nullptr;
+  int sms = 0;
+  gqa_status s = noalloc_scratch(dev, &scratch, &sms);
+  if (s != GQA_OK) return s;
+  cudaStream_t strm = static_cast<cudaStream_t>(stream);
+
+  const int group = num_heads / num_kv_heads;
+  const gqa::DecodePlan plan = gqa::plan_decode(head_dim, group);
+  const size_t segments = static_cast<size_t>(num_seqs) * num_kv_heads * plan.n_ht;
+  if (segments > kNoAllocMaxSegments)
+    return fail(GQA_ERR_UNSUPPORTED,
+                "allocation-free decode holds at most %zu segments (num_seqs * num_kv_heads * "
+                "head tiles); this call needs %zu",
+                kNoAllocMaxSegments, segments);
+  const int64_t blocks_per_seq =
+      (static_cast<int64_t>(max_blocks_per_seq) * page_size + gqa::kBlock - 1) / gqa::kBlock;
+  const int64_t max_blocks = static_cast<int64_t>(num_seqs) * num_kv_heads * plan.n_ht * blocks_per_seq;
+  int64_t workers = static_cast<int64_t>(sms) * plan.ctas_per_sm;
+  const int forced = g_num_workers.load();
+  if (forced > 0) workers = forced;
+  if (workers > max_blocks) workers = max_blocks;
+  if (workers < 1) workers = 1;
+  // Fewer workers when the split partials of every worker would not fit the array.
+  const size_t fixed = kNoAllocHeaderBytes + align256(segments * sizeof(int32_t));
+  const size_t per_worker = 2 * static_cast<size_t>(plan.heads_per_seg) *
+                            (static_cast<size_t>(head_dim) + 2) * sizeof(float) + 512;
+  const int64_t fit = static_cast<int64_t>((kNoAllocScratchBytes - fixed) / per_worker);
+  if (fit < 1)
+    return fail(GQA_ERR_UNSUPPORTED, "allocation-free scratch (%zu bytes) is too small for this call",
+                kNoAllocScratchBytes);
+  if (workers > fit) workers = fit;
+  const size_t slots = static_cast<size_t>(2 * workers);
+  unsigned char* counters = scratch + kNoAllocHeaderBytes;
+  unsigned char* part_ml = scratch + fixed;
+  unsigned char* part_o = part_ml + align256(slots * plan.heads_per_seg * 2 * sizeof(float));
+  if (part_o + slots * plan.heads_per_seg * head_dim * sizeof(float) > scratch + kNoAllocScratchBytes)
+    return fail(GQA_ERR_UNSUPPORTED, "allocation-free scratch layout does not fit");
+  // The array keeps the previous call's contents: the error word and the arrival
+  // counters must start at zero.
+  e = cudaMemsetAsync(scratch, 0, kNoAllocHeaderBytes + segments * sizeof(int32_t), strm);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(allocation-free scratch)");
+
+  CUtensorMap tk, tv;
+  s = make_pool_map(&tk, k_pages, rows, head_dim, dev);
+  if (s != GQA_OK) return s;
+  s = make_pool_map(&tv, v_pages, rows, head_dim, dev);
+  if (s != GQA_OK) return s;
+
+  gqa::DecodeParams p;
+  p.q = static_cast<const uint16_t*>(q);
+  p.out = static_cast<uint16_t*>(out);
+  p.block_table = block_table;
+  p.seq_lens = seq_lens;
+  p.part_o = reinterpret_cast<float*>(part_o);
+  p.part_ml = reinterpret_cast<float*>(part_ml);
+  p.counters = reinterpret_cast<int32_t*>(counters);
+  p.err = reinterpret_cast<uint32_t*>(scratch);
+  p.num_seqs = num_seqs;
+  p.num_heads = num_heads;
+  p.num_kv_heads = num_kv_heads;
+  p.group = group;
+  p.n_ht = plan.n_ht;
+  p.heads_per_seg = plan.heads_per_seg;
+  p.page_size = page_size;
+  p.max_blocks = max_blocks_per_seq;
+  p.num_pages = num_pages;
+  p.head_dim = head_dim;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.num_workers = static_cast<int>(workers);
+  p.wait_limit_ns = static_cast<uint64_t>(g_wait_limit_ns.load());
+  p.arm_without_copy = g_arm_without_copy.load();
+  e = gqa::launch_decode(p, plan, tk, tv, static_cast<int>(workers), strm);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   g_launches.fetch_add(1);
   return GQA_OK;

@@ -121,6 +121,40 @@ gqa_status gqa_paged_decode_attn(const void* q, const void* k_pages, const void*
                                  int num_pages, void* stream);
 
 /*
+ * gqa_paged_decode_attn_noalloc -- the same decode attention as gqa_paged_decode_attn
+ * (same arguments, layouts and result), for callers that cannot allocate device memory:
+ * an engine that has already reserved nearly all of the GPU for its own caching
+ * allocator or KV pool (an extra cudaMalloc would fail or fragment it), a step loop that
+ * cannot afford the device-wide synchronisation cudaMalloc/cudaFree imply, or a plugin
+ * whose host framework hands it no workspace.  The pages describe no such variant; it
+ * exists only for these callers.
+ *
+ * Scratch: instead of the per-device workspace, the call uses a fixed 16 MiB array
+ * compiled into the library's device image.  Every GPU that loads the library holds
+ * that array until the process exits.  This call never allocates: no cudaMalloc, no
+ * cudaFree, no allocating library routine.
+ *   - Set-up: the first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call before any
+ *     stream capture.
+ *   - Sharing: all calls use the same array and it keeps the last call's contents; each
+ *     call clears the part that must start at zero (error word, split counters) on
+ *     `stream`.  Calls whose execution overlaps on the GPU (other streams, other host
+ *     threads) race on the array and must be ordered by the caller.
+ *   - Limits: at most 16384 segments (num_seqs * num_kv_heads * head tiles; a head tile
+ *     holds 8 or 16 query heads for groups up to 16, up to 128 otherwise); when the
+ *     split partials of the default number of workers do not fit, fewer workers are
+ *     used.  A call beyond the limits returns GQA_ERR_UNSUPPORTED and launches nothing.
+ *   - Device-side range errors (bad page ids, lengths) are skipped as in
+ *     gqa_paged_decode_attn but recorded only in the array, so
+ *     gqa_check_device_error does not report them.
+ */
+gqa_status gqa_paged_decode_attn_noalloc(const void* q, const void* k_pages, const void* v_pages,
+                                         const int32_t* block_table, const int32_t* seq_lens,
+                                         void* out, int num_seqs, int num_heads, int num_kv_heads,
+                                         int head_dim, int page_size, float scale,
+                                         int max_blocks_per_seq, int num_pages, void* stream);
+
+/*
  * gqa_check_device_error -- synchronise `stream`, then read and clear the current
  * device's error word.  Returns GQA_OK, GQA_ERR_DEVICE_BOUNDS, GQA_ERR_TIMEOUT (takes
  * precedence when both are set; it also resets the decode workspace counters a
