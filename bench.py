@@ -168,6 +168,12 @@ def setup_dist(n_gpus: int):
     return 0, 1, 0
 
 
+def rank_seed(workload: int, rank: int) -> int:
+    """Seed of the batch rank `rank` runs: rank 0 runs the workload's own batch, the
+    others independent batches of the same shape (weak scaling, no data exchange)."""
+    return 1000 + workload + 7919 * rank
+
+
 def reduce_max_sum(t_ms: float, units: float, device):
     """Max of the per-rank times and sum of the per-rank units (whole-job figures)."""
     if not dist.is_initialized():
@@ -302,7 +308,7 @@ def run_ours(args, rank, world, local):
 
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    seed = 1000 + args.workload + 7919 * rank
+    seed = rank_seed(args.workload, rank)
     inp_cpu = _with_append(make_inputs(args.workload, seed=seed, poison=False), seed)
     nbytes = algorithmic_bytes(inp_cpu, with_append=True)
 
