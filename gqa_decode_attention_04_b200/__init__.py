@@ -22,6 +22,7 @@ __all__ = [
     "load_library",
     "kv_append",
     "paged_decode_attn",
+    "decode_step",
     "paged_decode_attn_noalloc",
     "check_device_error",
     "kv_cache_bytes",
@@ -42,6 +43,7 @@ STATUS_NAMES = {0: "GQA_OK", -1: "GQA_ERR_INVALID_ARG", -2: "GQA_ERR_UNSUPPORTED
 EXPORTED_SYMBOLS = (
     "gqa_kv_append",
     "gqa_paged_decode_attn",
+    "gqa_decode_step",
     "gqa_paged_decode_attn_noalloc",
     "gqa_check_device_error",
     "gqa_last_error_string",
@@ -83,6 +85,9 @@ def load_library() -> ctypes.CDLL:
     lib.gqa_paged_decode_attn.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32,
                                           i32, i32, vp]
     lib.gqa_paged_decode_attn.restype = i32
+    lib.gqa_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
+                                    f32, i32, i32, vp]
+    lib.gqa_decode_step.restype = i32
     lib.gqa_paged_decode_attn_noalloc.argtypes = lib.gqa_paged_decode_attn.argtypes
     lib.gqa_paged_decode_attn_noalloc.restype = i32
     lib.gqa_check_device_error.argtypes = [vp]
@@ -178,6 +183,42 @@ def paged_decode_attn(q, k_pages, v_pages, block_table, seq_lens, out: Optional[
                                          block_table.data_ptr(), seq_lens.data_ptr(), out.data_ptr(),
                                          B, H, Hk, D, ps, float(scale), block_table.shape[1], P,
                                          _stream_ptr(stream)))
+    return out
+
+
+def decode_step(q, k_new, v_new, k_pages, v_pages, block_table, positions, seq_lens,
+                out: Optional[torch.Tensor] = None, scale: Optional[float] = None,
+                stream=None) -> torch.Tensor:
+    """One decode step: append k_new/v_new at positions, then attend over seq_lens tokens."""
+    dev = q.device
+    for t, n, dt in ((q, "q", torch.bfloat16), (k_new, "k_new", torch.bfloat16),
+                     (v_new, "v_new", torch.bfloat16), (k_pages, "k_pages", torch.bfloat16),
+                     (v_pages, "v_pages", torch.bfloat16), (block_table, "block_table", torch.int32),
+                     (positions, "positions", torch.int32), (seq_lens, "seq_lens", torch.int32)):
+        _need(t, n, dt, dev)
+    B, H, D = q.shape
+    P, Hk, ps, D2 = k_pages.shape
+    if D2 != D or tuple(v_pages.shape) != (P, Hk, ps, D):
+        raise ValueError("page pools must be [num_pages, num_kv_heads, page_size, head_dim]")
+    if tuple(k_new.shape) != (B, Hk, D) or tuple(v_new.shape) != (B, Hk, D):
+        raise ValueError("k_new / v_new must be [num_seqs, num_kv_heads, head_dim]")
+    if (block_table.dim() != 2 or block_table.shape[0] != B or tuple(seq_lens.shape) != (B,)
+            or tuple(positions.shape) != (B,)):
+        raise ValueError("block_table must be [num_seqs, max_blocks]; seq_lens, positions [num_seqs]")
+    if out is None:
+        out = torch.empty((B, H, D), dtype=torch.bfloat16, device=dev)
+    else:
+        _need(out, "out", torch.bfloat16, dev)
+        if tuple(out.shape) != (B, H, D):
+            raise ValueError("out must be [num_seqs, num_heads, head_dim]")
+    if scale is None:
+        scale = 1.0 / (D ** 0.5)
+    lib = load_library()
+    with torch.cuda.device(dev):
+        _check(lib.gqa_decode_step(q.data_ptr(), k_new.data_ptr(), v_new.data_ptr(), k_pages.data_ptr(),
+                                   v_pages.data_ptr(), block_table.data_ptr(), positions.data_ptr(),
+                                   seq_lens.data_ptr(), out.data_ptr(), B, H, Hk, D, ps, float(scale),
+                                   block_table.shape[1], P, _stream_ptr(stream)))
     return out
 
 

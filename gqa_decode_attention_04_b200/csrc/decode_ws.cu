@@ -443,6 +443,7 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
         if (bytes) ptx::mbar_arrive_expect_tx(full_bar + 8 * stage, bytes);
         else ptx::mbar_arrive(full_bar + 8 * stage);
       }
+      if (i == 0) ptx::pdl_wait_prerequisites();  // K/V may still be written by the previous kernel
       __syncwarp();
       if (ok && !p.arm_without_copy) {
         const int kvh = cu.seg / p.n_ht;
@@ -544,42 +545,50 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int kvh = si.seg / p.n_ht;
     const int ht = si.seg % p.n_ht;
     const int64_t row0 = static_cast<int64_t>(si.b) * p.num_heads + kvh * p.group + ht * hps;
-    for (int idx = tid; idx < nrows_seg * D; idx += NCT) {
-      const int h = idx / D, d = idx - (idx / D) * D;
-      float M = -INFINITY, L = 0.f, acc = 0.f;
-      int64_t ww = wf;
-      for (; ww + 3 <= wl; ww += 4) {
-        float2 ml[4];
-        float ov[4];
+    // Outputs in batches of 8 per thread; for each piece the 8 (max, sum) pairs and 8
+    // partial values are loaded together, so a piece costs one L2 round trip per batch.
+    const int total_out = nrows_seg * D;
+    for (int base = 0; base < total_out; base += 8 * NCT) {
+      float M[8], L[8], acc[8];
+      int off_o[8], off_ml[8];
+      bool act[8];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int sl = piece_slot(ww + k, si.seg_base, T, W);
-          ml[k] = __ldcg(reinterpret_cast<const float2*>(p.part_ml + (static_cast<int64_t>(sl) * hps + h) * 2));
-          ov[k] = __ldcg(p.part_o + (static_cast<int64_t>(sl) * hps + h) * D + d);
+      for (int k = 0; k < 8; ++k) {
+        const int idx = base + tid + k * NCT;
+        act[k] = idx < total_out;
+        const int h = act[k] ? idx / D : 0;
+        off_o[k] = act[k] ? h * D + (idx - h * D) : 0;
+        off_ml[k] = h * 2;
+        M[k] = -INFINITY;
+        L[k] = 0.f;
+        acc[k] = 0.f;
+      }
+      for (int64_t ww = wf; ww <= wl; ++ww) {
+        const int64_t sl = piece_slot(ww, si.seg_base, T, W);
+        const float* po = p.part_o + sl * hps * D;
+        const float* pm = p.part_ml + sl * hps * 2;
+        float2 ml[8];
+        float ov[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          ml[k] = act[k] ? __ldcg(reinterpret_cast<const float2*>(pm + off_ml[k])) : make_float2(-INFINITY, 0.f);
+          ov[k] = act[k] ? __ldcg(po + off_o[k]) : 0.f;
         }
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float mn = fmaxf(M, ml[k].x);
+        for (int k = 0; k < 8; ++k) {
+          const float mn = fmaxf(M[k], ml[k].x);
           const float mu = (mn == -INFINITY) ? 0.f : mn;
-          const float a = ptx::ex2(M - mu), bw = ptx::ex2(ml[k].x - mu);
-          L = L * a + ml[k].y * bw;
-          acc = acc * a + ov[k] * bw;
-          M = mn;
+          const float a = ptx::ex2(M[k] - mu), bw = ptx::ex2(ml[k].x - mu);
+          L[k] = L[k] * a + ml[k].y * bw;
+          acc[k] = acc[k] * a + ov[k] * bw;
+          M[k] = mn;
         }
       }
-      for (; ww <= wl; ++ww) {
-        const int sl = piece_slot(ww, si.seg_base, T, W);
-        const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.part_ml + (static_cast<int64_t>(sl) * hps + h) * 2));
-        const float ov = __ldcg(p.part_o + (static_cast<int64_t>(sl) * hps + h) * D + d);
-        const float mn = fmaxf(M, ml.x);
-        const float mu = (mn == -INFINITY) ? 0.f : mn;
-        const float a = ptx::ex2(M - mu), bw = ptx::ex2(ml.x - mu);
-        L = L * a + ml.y * bw;
-        acc = acc * a + ov * bw;
-        M = mn;
-      }
-      reinterpret_cast<__nv_bfloat16*>(p.out)[(row0 + h) * D + d] =
-          __float2bfloat16_rn(L > 0.f ? acc / L : 0.f);
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        if (act[k])
+          reinterpret_cast<__nv_bfloat16*>(p.out)[row0 * D + off_o[k]] =
+              __float2bfloat16_rn(L[k] > 0.f ? acc[k] / L[k] : 0.f);
     }
     if (tid == 0) p.counters[segid] = 0;
   };
@@ -746,7 +755,7 @@ struct Cfg {
 
 template <int D, int NT, bool SH, int C>
 cudaError_t launch_t(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int grid,
-                     cudaStream_t stream) {
+                     cudaStream_t stream, bool overlap) {
   using CF = Cfg<D, NT, SH, C>;
   auto kern = decode_ws_kernel<D, NT, SH, C, CF::kStages>;
   static thread_local int configured_device = -1;
@@ -758,29 +767,42 @@ cudaError_t launch_t(const DecodeParams& p, const CUtensorMap& tk, const CUtenso
     if (e != cudaSuccess) return e;
     configured_device = dev;
   }
-  kern<<<grid, (C + 1) * 32, CF::kSmem, stream>>>(tk, tv, p);
-  return cudaGetLastError();
+  if (!overlap) {
+    kern<<<grid, (C + 1) * 32, CF::kSmem, stream>>>(tk, tv, p);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3((C + 1) * 32);
+  cfg.dynamicSmemBytes = CF::kSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tk, tv, p);
 }
 
 template <int D>
 cudaError_t launch_d(const DecodeParams& p, const DecodePlan& pl, const CUtensorMap& tk,
-                     const CUtensorMap& tv, int grid, cudaStream_t s) {
+                     const CUtensorMap& tv, int grid, cudaStream_t s, bool o) {
   if (!pl.split_heads)
-    return pl.n_tiles == 1 ? launch_t<D, 1, false, 4>(p, tk, tv, grid, s)
-                           : launch_t<D, 2, false, 4>(p, tk, tv, grid, s);
+    return pl.n_tiles == 1 ? launch_t<D, 1, false, 4>(p, tk, tv, grid, s, o)
+                           : launch_t<D, 2, false, 4>(p, tk, tv, grid, s, o);
   if (pl.n_tiles == 1) {
     switch (pl.consumers) {
-      case 3: return launch_t<D, 1, true, 3>(p, tk, tv, grid, s);
-      default: return launch_t<D, 1, true, 4>(p, tk, tv, grid, s);
+      case 3: return launch_t<D, 1, true, 3>(p, tk, tv, grid, s, o);
+      default: return launch_t<D, 1, true, 4>(p, tk, tv, grid, s, o);
     }
   }
   switch (pl.consumers) {
-    case 3: return launch_t<D, 2, true, 3>(p, tk, tv, grid, s);
-    case 4: return launch_t<D, 2, true, 4>(p, tk, tv, grid, s);
-    case 5: return launch_t<D, 2, true, 5>(p, tk, tv, grid, s);
-    case 6: return launch_t<D, 2, true, 6>(p, tk, tv, grid, s);
-    case 7: return launch_t<D, 2, true, 7>(p, tk, tv, grid, s);
-    default: return launch_t<D, 2, true, 8>(p, tk, tv, grid, s);
+    case 3: return launch_t<D, 2, true, 3>(p, tk, tv, grid, s, o);
+    case 4: return launch_t<D, 2, true, 4>(p, tk, tv, grid, s, o);
+    case 5: return launch_t<D, 2, true, 5>(p, tk, tv, grid, s, o);
+    case 6: return launch_t<D, 2, true, 6>(p, tk, tv, grid, s, o);
+    case 7: return launch_t<D, 2, true, 7>(p, tk, tv, grid, s, o);
+    default: return launch_t<D, 2, true, 8>(p, tk, tv, grid, s, o);
   }
 }
 
@@ -830,9 +852,9 @@ DecodePlan plan_decode(int head_dim, int group) {
 }
 
 cudaError_t launch_decode(const DecodeParams& p, const DecodePlan& pl, const CUtensorMap& tk,
-                          const CUtensorMap& tv, int grid, cudaStream_t stream) {
-  if (p.head_dim == 64) return launch_d<64>(p, pl, tk, tv, grid, stream);
-  return launch_d<128>(p, pl, tk, tv, grid, stream);
+                          const CUtensorMap& tv, int grid, cudaStream_t stream, bool overlap) {
+  if (p.head_dim == 64) return launch_d<64>(p, pl, tk, tv, grid, stream, overlap);
+  return launch_d<128>(p, pl, tk, tv, grid, stream, overlap);
 }
 
 }  // namespace gqa

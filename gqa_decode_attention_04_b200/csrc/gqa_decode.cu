@@ -209,79 +209,12 @@ gqa_status noalloc_scratch(int dev, unsigned char** ptr, int* sms) {
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t{255}; }
-}  // namespace
 
-extern "C" {
-
-const char* gqa_last_error_string(void) { return g_err_msg; }
-
-int gqa_abi_version(void) { return 1; }
-
-uint64_t gqa_launch_count(void) { return g_launches.load(); }
-
-size_t gqa_kv_cache_bytes(int num_layers, int num_kv_heads, int head_dim, int64_t seq_len) {
-  if (num_layers < 0 || num_kv_heads < 0 || head_dim < 0 || seq_len < 0) return 0;
-  return static_cast<size_t>(2) * num_layers * num_kv_heads * head_dim *
-         static_cast<size_t>(seq_len) * 2;
-}
-
-gqa_status gqa_set_num_workers(int n) {
-  if (n < 0 || n > (1 << 20)) return fail(GQA_ERR_INVALID_ARG, "num_workers must be in [0, 2^20]");
-  g_num_workers.store(n);
-  return GQA_OK;
-}
-
-gqa_status gqa_set_wait_limit_ns(int64_t limit_ns, int arm_without_copy) {
-  if (limit_ns <= 0) return fail(GQA_ERR_INVALID_ARG, "wait limit must be positive");
-  g_wait_limit_ns.store(limit_ns);
-  g_arm_without_copy.store(arm_without_copy ? 1 : 0);
-  return GQA_OK;
-}
-
-gqa_status gqa_kv_append(const void* k_new, const void* v_new, void* k_pages, void* v_pages,
-                         const int32_t* block_table, const int32_t* positions, int num_seqs,
-                         int num_kv_heads, int head_dim, int page_size, int max_blocks_per_seq,
-                         int num_pages, void* stream) {
-  if (num_seqs < 0) return fail(GQA_ERR_INVALID_ARG, "num_seqs < 0");
-  if (num_kv_heads < 1 || head_dim < 1 || page_size < 1 || max_blocks_per_seq < 1 || num_pages < 1)
-    return fail(GQA_ERR_INVALID_ARG, "sizes must be positive");
-  if (head_dim % 8 != 0) return fail(GQA_ERR_UNSUPPORTED, "head_dim must be a multiple of 8");
-  if (static_cast<int64_t>(max_blocks_per_seq) * page_size > INT32_MAX)
-    return fail(GQA_ERR_UNSUPPORTED, "max_blocks_per_seq * page_size exceeds 2^31");
-  if (num_seqs == 0) return GQA_OK;
-  if (!k_new || !v_new || !k_pages || !v_pages || !block_table || !positions)
-    return fail(GQA_ERR_INVALID_ARG, "null pointer argument");
-  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_pages, 16) || !aligned(v_pages, 16))
-    return fail(GQA_ERR_INVALID_ARG, "bf16 tensors must be 16-byte aligned");
-  DeviceState* st;
-  int dev;
-  gqa_status s = get_state(&st, &dev);
-  if (s != GQA_OK) return s;
-  gqa::AppendParams p;
-  p.k_new = static_cast<const uint4*>(k_new);
-  p.v_new = static_cast<const uint4*>(v_new);
-  p.k_pages = static_cast<uint4*>(k_pages);
-  p.v_pages = static_cast<uint4*>(v_pages);
-  p.block_table = block_table;
-  p.positions = positions;
-  p.err = st->err;
-  p.num_seqs = num_seqs;
-  p.num_kv_heads = num_kv_heads;
-  p.vec_per_row = head_dim / 8;
-  p.page_size = page_size;
-  p.max_blocks = max_blocks_per_seq;
-  p.num_pages = num_pages;
-  cudaError_t e = gqa::launch_kv_append(p, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "kv_append launch");
-  g_launches.fetch_add(1);
-  return GQA_OK;
-}
-
-gqa_status gqa_paged_decode_attn(const void* q, const void* k_pages, const void* v_pages,
-                                 const int32_t* block_table, const int32_t* seq_lens, void* out,
-                                 int num_seqs, int num_heads, int num_kv_heads, int head_dim,
-                                 int page_size, float scale, int max_blocks_per_seq,
-                                 int num_pages, void* stream) {
+gqa_status decode_impl(const void* q, const void* k_pages, const void* v_pages,
+                       const int32_t* block_table, const int32_t* seq_lens, void* out,
+                       int num_seqs, int num_heads, int num_kv_heads, int head_dim, int page_size,
+                       float scale, int max_blocks_per_seq, int num_pages, void* stream,
+                       bool overlap_previous) {
   if (num_seqs < 0) return fail(GQA_ERR_INVALID_ARG, "num_seqs < 0");
   if (num_seqs > 65536) return fail(GQA_ERR_UNSUPPORTED, "num_seqs > 65536");
   if (num_heads < 1 || num_kv_heads < 1 || head_dim < 1 || page_size < 1 ||
@@ -362,10 +295,104 @@ gqa_status gqa_paged_decode_attn(const void* q, const void* k_pages, const void*
   p.num_workers = static_cast<int>(workers);
   p.wait_limit_ns = static_cast<uint64_t>(g_wait_limit_ns.load());
   p.arm_without_copy = g_arm_without_copy.load();
-  cudaError_t e = gqa::launch_decode(p, plan, tk, tv, grid, strm);
+  cudaError_t e = gqa::launch_decode(p, plan, tk, tv, grid, strm, overlap_previous);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   g_launches.fetch_add(1);
   return GQA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* gqa_last_error_string(void) { return g_err_msg; }
+
+int gqa_abi_version(void) { return 1; }
+
+uint64_t gqa_launch_count(void) { return g_launches.load(); }
+
+size_t gqa_kv_cache_bytes(int num_layers, int num_kv_heads, int head_dim, int64_t seq_len) {
+  if (num_layers < 0 || num_kv_heads < 0 || head_dim < 0 || seq_len < 0) return 0;
+  return static_cast<size_t>(2) * num_layers * num_kv_heads * head_dim *
+         static_cast<size_t>(seq_len) * 2;
+}
+
+gqa_status gqa_set_num_workers(int n) {
+  if (n < 0 || n > (1 << 20)) return fail(GQA_ERR_INVALID_ARG, "num_workers must be in [0, 2^20]");
+  g_num_workers.store(n);
+  return GQA_OK;
+}
+
+gqa_status gqa_set_wait_limit_ns(int64_t limit_ns, int arm_without_copy) {
+  if (limit_ns <= 0) return fail(GQA_ERR_INVALID_ARG, "wait limit must be positive");
+  g_wait_limit_ns.store(limit_ns);
+  g_arm_without_copy.store(arm_without_copy ? 1 : 0);
+  return GQA_OK;
+}
+
+gqa_status gqa_kv_append(const void* k_new, const void* v_new, void* k_pages, void* v_pages,
+                         const int32_t* block_table, const int32_t* positions, int num_seqs,
+                         int num_kv_heads, int head_dim, int page_size, int max_blocks_per_seq,
+                         int num_pages, void* stream) {
+  if (num_seqs < 0) return fail(GQA_ERR_INVALID_ARG, "num_seqs < 0");
+  if (num_kv_heads < 1 || head_dim < 1 || page_size < 1 || max_blocks_per_seq < 1 || num_pages < 1)
+    return fail(GQA_ERR_INVALID_ARG, "sizes must be positive");
+  if (head_dim % 8 != 0) return fail(GQA_ERR_UNSUPPORTED, "head_dim must be a multiple of 8");
+  if (static_cast<int64_t>(max_blocks_per_seq) * page_size > INT32_MAX)
+    return fail(GQA_ERR_UNSUPPORTED, "max_blocks_per_seq * page_size exceeds 2^31");
+  if (num_seqs == 0) return GQA_OK;
+  if (!k_new || !v_new || !k_pages || !v_pages || !block_table || !positions)
+    return fail(GQA_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_pages, 16) || !aligned(v_pages, 16))
+    return fail(GQA_ERR_INVALID_ARG, "bf16 tensors must be 16-byte aligned");
+  DeviceState* st;
+  int dev;
+  gqa_status s = get_state(&st, &dev);
+  if (s != GQA_OK) return s;
+  gqa::AppendParams p;
+  p.k_new = static_cast<const uint4*>(k_new);
+  p.v_new = static_cast<const uint4*>(v_new);
+  p.k_pages = static_cast<uint4*>(k_pages);
+  p.v_pages = static_cast<uint4*>(v_pages);
+  p.block_table = block_table;
+  p.positions = positions;
+  p.err = st->err;
+  p.num_seqs = num_seqs;
+  p.num_kv_heads = num_kv_heads;
+  p.vec_per_row = head_dim / 8;
+  p.page_size = page_size;
+  p.max_blocks = max_blocks_per_seq;
+  p.num_pages = num_pages;
+  cudaError_t e = gqa::launch_kv_append(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "kv_append launch");
+  g_launches.fetch_add(1);
+  return GQA_OK;
+}
+
+gqa_status gqa_paged_decode_attn(const void* q, const void* k_pages, const void* v_pages,
+                                 const int32_t* block_table, const int32_t* seq_lens, void* out,
+                                 int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                 int page_size, float scale, int max_blocks_per_seq,
+                                 int num_pages, void* stream) {
+  return decode_impl(q, k_pages, v_pages, block_table, seq_lens, out, num_seqs, num_heads,
+                     num_kv_heads, head_dim, page_size, scale, max_blocks_per_seq, num_pages,
+                     stream, false);
+}
+
+gqa_status gqa_decode_step(const void* q, const void* k_new, const void* v_new, void* k_pages,
+                           void* v_pages, const int32_t* block_table, const int32_t* positions,
+                           const int32_t* seq_lens, void* out, int num_seqs, int num_heads,
+                           int num_kv_heads, int head_dim, int page_size, float scale,
+                           int max_blocks_per_seq, int num_pages, void* stream) {
+  gqa_status s = gqa_kv_append(k_new, v_new, k_pages, v_pages, block_table, positions, num_seqs,
+                               num_kv_heads, head_dim, page_size, max_blocks_per_seq, num_pages,
+                               stream);
+  if (s != GQA_OK) return s;
+  // The decode launch overlaps the append kernel's tail: the append writes only the
+  // new K/V rows, which the decode's producer reads after waiting for it.
+  return decode_impl(q, k_pages, v_pages, block_table, seq_lens, out, num_seqs, num_heads,
+                     num_kv_heads, head_dim, page_size, scale, max_blocks_per_seq, num_pages,
+                     stream, true);
 }
 
 gqa_status gqa_paged_decode_attn_noalloc(const void* q, const void* k_pages, const void* v_pages,

@@ -68,7 +68,11 @@ struct DecodePlan {
 };
 
 DecodePlan plan_decode(int head_dim, int group);
+// overlap_previous: launch with programmatic stream serialization, so the prologue
+// overlaps the preceding kernel of the stream (which must write nothing the decode reads
+// except the K/V pools); the producer waits for that kernel before its first K/V copy.
 cudaError_t launch_decode(const DecodeParams& p, const DecodePlan& plan, const CUtensorMap& tmap_k,
-                          const CUtensorMap& tmap_v, int grid, cudaStream_t stream);
+                          const CUtensorMap& tmap_v, int grid, cudaStream_t stream,
+                          bool overlap_previous = false);
 
 }  // namespace gqa

@@ -5,10 +5,14 @@
 // one 16-byte vector, so a warp writes 512 contiguous bytes of one slot row
 // (head_dim = 128: two rows per warp) and the copy is bit-exact.
 #include "internal.cuh"
+#include "ptx.cuh"
 
 namespace gqa {
 
 __global__ void __launch_bounds__(256) kv_append_kernel(const AppendParams p) {
+  // A decode kernel launched right after this one may start its prologue (it reads
+  // none of what this kernel writes until it waits for this grid to complete).
+  ptx::pdl_launch_dependents();
   const int64_t per_tensor =
       static_cast<int64_t>(p.num_seqs) * p.num_kv_heads * p.vec_per_row;
   const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;

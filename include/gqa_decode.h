@@ -121,6 +121,21 @@ gqa_status gqa_paged_decode_attn(const void* q, const void* k_pages, const void*
                                  int num_pages, void* stream);
 
 /*
+ * gqa_decode_step -- one decode step: gqa_kv_append of this step's K/V rows (at
+ * positions[b]), then gqa_paged_decode_attn over seq_lens[b] tokens, on `stream`.
+ * Same arguments, layouts, requirements and errors as the two calls.  The decode launch
+ * overlaps the append (programmatic dependent launch): its prologue and block-table
+ * reads run while the append finishes, and its first K/V copy waits for it.  This is
+ * the step tiny-llm's "优化" page describes (append position, then attention over the
+ * block table) as one call.
+ */
+gqa_status gqa_decode_step(const void* q, const void* k_new, const void* v_new, void* k_pages,
+                           void* v_pages, const int32_t* block_table, const int32_t* positions,
+                           const int32_t* seq_lens, void* out, int num_seqs, int num_heads,
+                           int num_kv_heads, int head_dim, int page_size, float scale,
+                           int max_blocks_per_seq, int num_pages, void* stream);
+
+/*
  * gqa_paged_decode_attn_noalloc -- the same decode attention as gqa_paged_decode_attn
  * (same arguments, layouts and result), for callers that cannot allocate device memory:
  * an engine that has already reserved nearly all of the GPU for its own caching

@@ -188,3 +188,45 @@ def test_workload5_append_then_attend(cuda_device):
     rows = _sample_rows(inp, n_seq=10)
     got = gpu_f64(out)[[r[0] for r in rows], [r[1] for r in rows]]
     assert_close(got, oracle_rows(h, rows), what="continuous_batch")
+
+
+# ------------------------------------------------------------------ fused decode step
+
+@pytest.mark.parametrize("case", [([1, 17, 300, 64, 2000], 32, 8, 128, 16),
+                                  ([40, 9], 4, 1, 64, 16),
+                                  ([700, 129], 96, 1, 128, 64)],
+                         ids=["gqa", "tiny_mqa", "mqa"])
+def test_decode_step_equals_append_then_attend(cuda_device, case):
+    seq_lens, H, Hk, D, ps = case
+    inp = make_custom_inputs(seq_lens, H, Hk, D, ps, seed=31, append=True, extra_pages=2)
+    d = inp.to(cuda_device)
+    out = gq.decode_step(d.q, d.k_new, d.v_new, d.k_pages, d.v_pages, d.block_table, d.positions,
+                         d.seq_lens, scale=d.scale)
+    gq.check_device_error()
+    h = host_arrays(inp)
+    k2, v2 = oracle.kv_append(h["k"], h["v"], bf16_bits(inp.k_new), bf16_bits(inp.v_new),
+                              h["bt"], inp.positions.numpy())
+    assert np.array_equal(bf16_bits(d.k_pages), k2)
+    assert np.array_equal(bf16_bits(d.v_pages), v2)
+    h["k"], h["v"] = k2, v2
+    assert_close(gpu_f64(out), oracle_out(h), what=str(case))
+
+
+def test_consecutive_steps_rewrite_what_the_previous_decode_read(cuda_device):
+    """Back-to-back steps append different rows at the same positions: each decode must
+    see its own step's rows, never a later or earlier step's."""
+    inp = make_custom_inputs([500, 33, 1], 16, 4, 128, 16, seed=32, append=True)
+    d = inp.to(cuda_device)
+    g = torch.Generator().manual_seed(5)
+    outs, rows = [], []
+    for step in range(4):
+        kn = torch.randn(d.k_new.shape, generator=g).to(torch.bfloat16)
+        vn = torch.randn(d.v_new.shape, generator=g).to(torch.bfloat16) * (step + 1)
+        rows.append((kn, vn))
+        outs.append(gq.decode_step(d.q, kn.to(cuda_device), vn.to(cuda_device), d.k_pages, d.v_pages,
+                                   d.block_table, d.positions, d.seq_lens, scale=d.scale))
+    gq.check_device_error()
+    h = host_arrays(inp)
+    for step, (kn, vn) in enumerate(rows):
+        k2, v2 = oracle.kv_append(h["k"], h["v"], bf16_bits(kn), bf16_bits(vn), h["bt"], inp.positions.numpy())
+        assert_close(gpu_f64(outs[step]), oracle_out(dict(h, k=k2, v=v2)), what=f"step {step}")
