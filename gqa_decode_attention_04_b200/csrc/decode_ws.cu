@@ -84,6 +84,22 @@ __device__ __forceinline__ void cursor_load_seq(Cursor& cu, const DecodeParams& 
   cu.nblk = (cu.len + kBlock - 1) / kBlock;
 }
 
+// Step a cursor to the next block of the work list (only while blocks remain).
+// next_len holds seq_lens[c.b + 1], loaded ahead of the cursor reaching it.
+__device__ __forceinline__ void walk_next(Cursor& c, int& next_len, const DecodeParams& p, int segs,
+                                          int cap) {
+  if (++c.blk < c.nblk) return;
+  c.blk = 0;
+  if (++c.seg < segs) return;
+  c.seg = 0;
+  do {
+    ++c.b;
+    c.len = (c.b < p.num_seqs) ? eff_len(next_len, cap) : 0;
+    c.nblk = (c.len + kBlock - 1) / kBlock;
+    next_len = (c.b + 1 < p.num_seqs) ? __ldg(p.seq_lens + c.b + 1) : 0;
+  } while (c.nblk == 0 && c.b + 1 < p.num_seqs);
+}
+
 __device__ __forceinline__ int64_t worker_start(int64_t w, int64_t T, int64_t W) { return w * T / W; }
 // The worker (CTA) whose range holds linear block x.
 __device__ __forceinline__ int64_t worker_of(int64_t x, int64_t T, int64_t W) {
@@ -208,7 +224,7 @@ __device__ __forceinline__ void attend_subchunk(uint32_t kb, uint32_t vb, int nv
 #define GQA_CTAS_HEAD_SPLIT 1
 #endif
 #ifndef GQA_SMEM_PER_SM_KB
-#define GQA_SMEM_PER_SM_KB 200
+#define GQA_SMEM_PER_SM_KB 212
 #endif
 template <bool SPLIT_HEADS>
 constexpr int ctas_per_sm() { return SPLIT_HEADS ? GQA_CTAS_HEAD_SPLIT : GQA_CTAS_TOKEN_SPLIT; }
@@ -216,7 +232,7 @@ constexpr int ctas_per_sm() { return SPLIT_HEADS ? GQA_CTAS_HEAD_SPLIT : GQA_CTA
 // D: head_dim.  NT: 8-head n-tiles per consumer.  SPLIT_HEADS: consumers split the
 // query heads (else the 64 tokens of a stage).  C: consumer warps.  S: stages.
 template <int D, int NT, bool SPLIT_HEADS, int C, int S>
-__global__ void __launch_bounds__((C + 1) * 32, ctas_per_sm<SPLIT_HEADS>())
+__global__ void __launch_bounds__((C + (SPLIT_HEADS ? 1 : 2)) * 32, ctas_per_sm<SPLIT_HEADS>())
 decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
                  const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
   using G_ = Geo<D>;
@@ -239,7 +255,8 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
   const int cap = p.max_blocks * p.page_size;
 
   // ---------------------------------------------------------------- prologue
-  // Pass 1: total block count T (and zero rows of empty sequences).
+  // Pass 1: block counts per sequence, their total T (and zero rows of empty sequences).
+  int64_t n_first = 0;  // this thread's count in the first tile of sequences
   int64_t mine = 0;
   for (int b = threadIdx.x; b < B; b += blockDim.x) {
     const int L = __ldg(p.seq_lens + b);
@@ -249,54 +266,73 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
       uint32_t* o = reinterpret_cast<uint32_t*>(p.out + static_cast<int64_t>(b) * p.num_heads * D);
       for (int i = 0; i < p.num_heads * D / 2; ++i) o[i] = 0u;
     }
-    mine += static_cast<int64_t>((Le + kBlock - 1) / kBlock) * segs;
+    const int64_t n = static_cast<int64_t>((Le + kBlock - 1) / kBlock) * segs;
+    if (b == static_cast<int>(threadIdx.x)) n_first = n;
+    mine += n;
   }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, off);
-  if (lane == 0) s_wtot[warp] = mine;
   if (threadIdx.x == 0) s_start_b = -1;
-  __syncthreads();
-  int64_t T = 0;
-  for (int i = 0; i < nwarps; ++i) T += s_wtot[i];
-  // Only the first T CTAs get work when there are fewer blocks than CTAs, so every
-  // CTA in use owns at least one block and a segment's pieces come from exactly the
-  // CTAs worker_of(first block) .. worker_of(last block).
-  const int64_t W = min(static_cast<int64_t>(p.num_workers), T);
+  // Inclusive block-wide scan of one value per thread; returns (inclusive, tile total).
+  auto block_scan = [&](int64_t n, int64_t& tot) -> int64_t {
+    int64_t incl = n;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int64_t v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    if (lane == 31) s_wtot[warp] = incl;
+    __syncthreads();
+    int64_t pre = 0;
+    tot = 0;
+    for (int i = 0; i < nwarps; ++i) {
+      if (i < warp) pre += s_wtot[i];
+      tot += s_wtot[i];
+    }
+    __syncthreads();  // s_wtot is reused by the next scan
+    return incl + pre;
+  };
+  int64_t T = 0, W = 0, x0 = 0, x1 = 0;
   const int64_t w = blockIdx.x;
-  if (w >= W) return;  // (also covers T == 0)
-  const int64_t x0 = worker_start(w, T, W);
-  const int64_t x1 = worker_start(w + 1, T, W);
-  __syncthreads();  // s_wtot is reused below
-
-  // Pass 2: locate the sequence holding block x0 (tiled block scan).
-  {
+  if (B <= static_cast<int>(blockDim.x)) {
+    // One tile holds every sequence: the scan gives T and the start in one pass.
+    const int64_t incl = block_scan(n_first, T);
+    // Only the first T CTAs get work when there are fewer blocks than CTAs, so every
+    // CTA in use owns at least one block and a segment's pieces come from exactly the
+    // CTAs worker_of(first block) .. worker_of(last block).
+    W = min(static_cast<int64_t>(p.num_workers), T);
+    if (w >= W) return;  // (also covers T == 0)
+    x0 = worker_start(w, T, W);
+    x1 = worker_start(w + 1, T, W);
+    if (n_first > 0 && x0 >= incl - n_first && x0 < incl) {
+      s_start_b = threadIdx.x;
+      s_start_base = incl - n_first;
+    }
+    __syncthreads();
+  } else {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, off);
+    if (lane == 0) s_wtot[warp] = mine;
+    __syncthreads();
+    for (int i = 0; i < nwarps; ++i) T += s_wtot[i];
+    W = min(static_cast<int64_t>(p.num_workers), T);
+    if (w >= W) return;
+    x0 = worker_start(w, T, W);
+    x1 = worker_start(w + 1, T, W);
+    __syncthreads();  // s_wtot is reused below
+    // Pass 2: locate the sequence holding block x0 (tiled block scan).
     int64_t base = 0;
     for (int t0 = 0; t0 < B && base <= x0; t0 += blockDim.x) {
       const int b = t0 + threadIdx.x;
       int64_t n = 0;
       if (b < B) n = static_cast<int64_t>((eff_len(__ldg(p.seq_lens + b), cap) + kBlock - 1) / kBlock) * segs;
-      int64_t incl = n;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int64_t v = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += v;
-      }
-      if (lane == 31) s_wtot[warp] = incl;
-      __syncthreads();
-      int64_t pre = 0, tot = 0;
-      for (int i = 0; i < nwarps; ++i) {
-        if (i < warp) pre += s_wtot[i];
-        tot += s_wtot[i];
-      }
-      incl += pre;
-      const int64_t lo = base + incl - n, hi = base + incl;
-      if (n > 0 && x0 >= lo && x0 < hi) {
+      int64_t tot = 0;
+      const int64_t incl = base + block_scan(n, tot);
+      if (n > 0 && x0 >= incl - n && x0 < incl) {
         s_start_b = b;
-        s_start_base = lo;
+        s_start_base = incl - n;
       }
       base += tot;
-      __syncthreads();
     }
+    __syncthreads();
   }
 
   // ---------------------------------------------------------------- shared layout
@@ -304,13 +340,19 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
   const uint32_t pad = (1024u - (smem0 & 1023u)) & 1023u;
   uint8_t* base_ptr = smem_raw + pad;
   const uint32_t ring = smem0 + pad;
-  constexpr int kMergeOs = SPLIT_HEADS ? 0 : C * NH * D;     // floats
-  constexpr int kMergeMl = SPLIT_HEADS ? 0 : 2 * C * NH * 2; // floats, double-buffered
-  float* os = reinterpret_cast<float*>(base_ptr + S * G_::kStageBytes);
-  float* mls = os + kMergeOs;
-  StageInfo* info = reinterpret_cast<StageInfo*>(mls + kMergeMl);
+  // Token split: at a piece end each consumer leaves its partial O^T in the part of the
+  // stage only it read (its sub-chunk's K tile, and V tile for a second n-tile) and its
+  // (max, sum) pairs in cml[stage]; the epilogue warp combines them and releases the stage.
+  static_assert(SPLIT_HEADS || 8 * D * 4 == G_::kSubBytes, "an 8-head partial fills one sub-chunk tile");
+  constexpr int kCml = SPLIT_HEADS ? 0 : S * C * NH * 2;  // floats
+  float* cml = reinterpret_cast<float*>(base_ptr + S * G_::kStageBytes);
+  // Token split: the query rows of a piece arrive with its first block (bulk copy).
+  constexpr int kQBytes = SPLIT_HEADS ? 0 : NH * D * 2;
+  uint8_t* qbuf = reinterpret_cast<uint8_t*>(cml + kCml);
+  StageInfo* info = reinterpret_cast<StageInfo*>(qbuf + S * kQBytes);
   const uint32_t full_bar = ptx::smem_u32(info + S);
   const uint32_t empty_bar = full_bar + 8 * S;
+  const uint32_t comb_bar = empty_bar + 8 * S;  // token split: consumers -> epilogue
 
   const int start_b = s_start_b;
   const int64_t start_base = s_start_base;
@@ -322,6 +364,7 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
     for (int s = 0; s < S; ++s) {
       ptx::mbar_init(full_bar + 8 * s, 1);
       ptx::mbar_init(empty_bar + 8 * s, C);
+      if (!SPLIT_HEADS) ptx::mbar_init(comb_bar + 8 * s, C);
     }
     ptx::fence_mbarrier_init();
   }
@@ -381,17 +424,10 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
       const int pg = __shfl_sync(0xffffffffu, wval, src);
       return (lane < kSubChunks && t < c.len) ? pg : -1;
     };
-    auto advance = [&](Cursor& c) {
-      if (++c.blk < c.nblk) return;
-      c.blk = 0;
-      if (++c.seg < segs) return;
-      c.seg = 0;
-      do {
-        ++c.b;
-        c.len = (c.b < B) ? eff_len(next_len, cap) : 0;
-        c.nblk = (c.len + kBlock - 1) / kBlock;
-        next_len = (c.b + 1 < B) ? __ldg(p.seq_lens + c.b + 1) : 0;
-      } while (c.nblk == 0 && c.b + 1 < B);
+    // Bytes of a piece's query rows (contiguous in q): the token split stages them.
+    auto q_rows_bytes = [&](const Cursor& c) -> uint32_t {
+      const int ht = c.seg % p.n_ht;
+      return static_cast<uint32_t>(min(NH, p.group - ht * NH)) * D * 2u;
     };
     // Pull a piece's query rows into L2 ahead of the consumers that load them.
     auto prefetch_q = [&](const Cursor& c) {
@@ -402,7 +438,7 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
       for (int off = lane * 128; off < nrows * D * 2; off += 32 * 128) ptx::prefetch_l2(q0 + off);
     };
     int page = page_of(cu);
-    prefetch_q(cu);
+    if (SPLIT_HEADS) prefetch_q(cu);
     int piece_blk0 = cu.blk;
     bool first_piece = true;
     int64_t seg_base = x0 - cu.blk;
@@ -439,12 +475,18 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
         si.flags = (first ? kFirstOfPiece : 0) | (last ? kLastOfPiece : 0) |
                    ((last && piece_blk0 == 0 && cu.blk + 1 == cu.nblk) ? kSole : 0) |
                    (first_piece ? kFirstPieceOfCta : 0);
-        const uint32_t bytes = static_cast<uint32_t>(__popc(submask)) * 2u * G_::kSubBytes;
+        uint32_t bytes = static_cast<uint32_t>(__popc(submask)) * 2u * G_::kSubBytes;
+        if (!SPLIT_HEADS && first && !p.arm_without_copy) bytes += q_rows_bytes(cu);
         if (bytes) ptx::mbar_arrive_expect_tx(full_bar + 8 * stage, bytes);
         else ptx::mbar_arrive(full_bar + 8 * stage);
       }
       if (i == 0) ptx::pdl_wait_prerequisites();  // K/V may still be written by the previous kernel
       __syncwarp();
+      if (!SPLIT_HEADS && first && lane == kSubChunks && !p.arm_without_copy) {
+        const int kvh = cu.seg / p.n_ht, ht = cu.seg % p.n_ht;
+        const uint16_t* src = p.q + (static_cast<int64_t>(cu.b) * p.num_heads + kvh * p.group + ht * NH) * D;
+        ptx::bulk_load(ptx::smem_u32(qbuf + stage * kQBytes), src, q_rows_bytes(cu), full_bar + 8 * stage);
+      }
       if (ok && !p.arm_without_copy) {
         const int kvh = cu.seg / p.n_ht;
         const int row = (page * p.num_kv_heads + kvh) * p.page_size +
@@ -458,13 +500,162 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
       }
       if (last) first_piece = false;
       if (i + 1 < total) {
-        advance(cu);
+        walk_next(cu, next_len, p, segs, cap);
         if (cu.blk == 0) {
           seg_base = x0 + i + 1;
-          prefetch_q(cu);
+          if (SPLIT_HEADS) prefetch_q(cu);
         }
         page = page_of(cu);
       }
+    }
+    return;
+  }
+
+  if (!SPLIT_HEADS && warp == C + 1) {
+    // ============================================================ epilogue warp
+    // Walks the same block list.  At each piece end it waits for the C consumers' states
+    // in the stage, combines them, writes out (or this CTA's piece of the segment),
+    // releases the stage to the producer, and runs the cross-CTA step; the consumers
+    // meanwhile go on with the next blocks.
+    constexpr int CPL = D / 32;  // columns per lane
+    const int d0 = lane * CPL;
+    const int hps = p.heads_per_seg;
+    int next_len = (cu.b + 1 < B) ? __ldg(p.seq_lens + cu.b + 1) : 0;
+    uint32_t comb_phase = 0;  // bit s: parity of the next completion of comb_bar[s]
+    for (int64_t i = 0; i < total; ++i) {
+      if ((cu.blk + 1 == cu.nblk) || (i + 1 == total)) {
+        const int stage = static_cast<int>(i % S);
+        const bool ok = ptx::mbar_wait_bounded(comb_bar + 8 * stage, (comb_phase >> stage) & 1u, limit);
+        comb_phase ^= 1u << stage;
+        if (!__all_sync(0xffffffffu, ok)) {
+          if (lane == 0) atomicOr(p.err, kErrTimeout);
+          return;
+        }
+        const StageInfo si = info[stage];
+        const float* ml = cml + stage * C * NH * 2;  // [C][NH][2]
+        const uint8_t* st = base_ptr + stage * G_::kStageBytes;
+        const int kvh = si.seg / p.n_ht, ht = si.seg % p.n_ht;
+        const int nrows = min(hps, p.group - ht * hps);
+        const int64_t row0 = static_cast<int64_t>(si.b) * p.num_heads + kvh * p.group + ht * hps;
+        const bool sole = si.flags & kSole;
+        const int64_t slot = w * 2 + ((si.flags & kFirstPieceOfCta) ? 0 : 1);
+        for (int h = 0; h < nrows; ++h) {
+          float mj[C], wj[C];
+          float M = -INFINITY, L = 0.f;
+#pragma unroll
+          for (int jj = 0; jj < C; ++jj) {
+            mj[jj] = ml[(jj * NH + h) * 2];
+            M = fmaxf(M, mj[jj]);
+          }
+#pragma unroll
+          for (int jj = 0; jj < C; ++jj) {
+            wj[jj] = (mj[jj] == -INFINITY) ? 0.f : ptx::ex2(mj[jj] - M);
+            L += wj[jj] * ml[(jj * NH + h) * 2 + 1];
+          }
+          float acc[CPL];
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) acc[c] = 0.f;
+#pragma unroll
+          for (int jj = 0; jj < C; ++jj) {
+            const float* src = reinterpret_cast<const float*>(st + (h >= 8 ? G_::kTileBytes : 0) +
+                                                              jj * G_::kSubBytes) + (h & 7) * D + d0;
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) acc[c] += wj[jj] * src[c];
+          }
+          if (sole) {
+            const float inv = L > 0.f ? 1.f / L : 0.f;
+            uint16_t* dst = p.out + (row0 + h) * D + d0;
+            if constexpr (CPL == 4) {
+              uint2 v;
+              v.x = ptx::pack_bf16x2(acc[0] * inv, acc[1] * inv);
+              v.y = ptx::pack_bf16x2(acc[2] * inv, acc[3] * inv);
+              *reinterpret_cast<uint2*>(dst) = v;
+            } else {
+              *reinterpret_cast<uint32_t*>(dst) = ptx::pack_bf16x2(acc[0] * inv, acc[1] * inv);
+            }
+          } else {
+            float* dst = p.part_o + (slot * hps + h) * D + d0;
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) dst[c] = acc[c];
+            if (lane == 0)
+              *reinterpret_cast<float2*>(p.part_ml + (slot * hps + h) * 2) = make_float2(M, L);
+          }
+        }
+        // The stage is free again: all lanes are done reading it.
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive_cnt(empty_bar + 8 * stage, C);
+
+        if (!sole) {
+          // Cross-CTA step: the last CTA to finish its piece merges every piece.
+          __threadfence();
+          __syncwarp();
+          const int64_t segid = static_cast<int64_t>(si.b) * segs + si.seg;
+          int prev = 0;
+          if (lane == 0) prev = atomicAdd(p.counters + segid, 1);
+          prev = __shfl_sync(0xffffffffu, prev, 0);
+          const int64_t wf = worker_of(si.seg_base, T, W);
+          const int64_t wl = worker_of(si.seg_base + si.nblk - 1, T, W);
+          if (prev == static_cast<int>(wl - wf)) {
+            __threadfence();
+            for (int h0 = 0; h0 < nrows; h0 += 8) {
+              float M[8], L[8], acc[8][CPL];
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                M[k] = -INFINITY;
+                L[k] = 0.f;
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) acc[k][c] = 0.f;
+              }
+              for (int64_t ww = wf; ww <= wl; ++ww) {
+                const int64_t sl = piece_slot(ww, si.seg_base, T, W);
+                float2 mlv[8];
+                float v[8][CPL];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                  const int h = min(h0 + k, nrows - 1);
+                  mlv[k] = __ldcg(reinterpret_cast<const float2*>(p.part_ml + (sl * hps + h) * 2));
+                  const float* src = p.part_o + (sl * hps + h) * D + d0;
+                  if constexpr (CPL == 4) {
+                    const float4 t4 = __ldcg(reinterpret_cast<const float4*>(src));
+                    v[k][0] = t4.x; v[k][1] = t4.y; v[k][2] = t4.z; v[k][3] = t4.w;
+                  } else {
+                    const float2 t2 = __ldcg(reinterpret_cast<const float2*>(src));
+                    v[k][0] = t2.x; v[k][1] = t2.y;
+                  }
+                }
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                  const float mn = fmaxf(M[k], mlv[k].x);
+                  const float mu = (mn == -INFINITY) ? 0.f : mn;
+                  const float a = ptx::ex2(M[k] - mu), bw = ptx::ex2(mlv[k].x - mu);
+                  L[k] = L[k] * a + mlv[k].y * bw;
+#pragma unroll
+                  for (int c = 0; c < CPL; ++c) acc[k][c] = acc[k][c] * a + v[k][c] * bw;
+                  M[k] = mn;
+                }
+              }
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                if (h0 + k < nrows) {
+                  const float inv = L[k] > 0.f ? 1.f / L[k] : 0.f;
+                  uint16_t* dst = p.out + (row0 + h0 + k) * D + d0;
+                  if constexpr (CPL == 4) {
+                    uint2 u;
+                    u.x = ptx::pack_bf16x2(acc[k][0] * inv, acc[k][1] * inv);
+                    u.y = ptx::pack_bf16x2(acc[k][2] * inv, acc[k][3] * inv);
+                    *reinterpret_cast<uint2*>(dst) = u;
+                  } else {
+                    *reinterpret_cast<uint32_t*>(dst) = ptx::pack_bf16x2(acc[k][0] * inv, acc[k][1] * inv);
+                  }
+                }
+              }
+            }
+            if (lane == 0) p.counters[segid] = 0;
+          }
+        }
+      }
+      if (i + 1 < total) walk_next(cu, next_len, p, segs, cap);
     }
     return;
   }
@@ -496,9 +687,8 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
   int nrows_c = 0;    // valid heads of this consumer's tile
   int hoff_c = 0;     // first segment-relative head of this consumer's tile
   const float sl2 = p.scale_log2;
-  int piece_parity = 0;
 
-  auto load_q = [&](int b, int seg) {
+  auto load_q = [&](int b, int seg, int stage) {
     const int kvh = seg / p.n_ht;
     const int ht = seg % p.n_ht;
     nrows_seg = min(p.heads_per_seg, p.group - ht * p.heads_per_seg);
@@ -509,12 +699,15 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
     for (int nt = 0; nt < NT; ++nt) {
       const int h = nt * 8 + g;
       const bool v = h < nrows_c;
-      const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
-          p.q + (static_cast<int64_t>(b) * p.num_heads + head0 + (v ? h : 0)) * D);
+      // token split: from the rows staged with the piece's first block; else from HBM/L2
+      const uint32_t* qrow =
+          SPLIT_HEADS ? reinterpret_cast<const uint32_t*>(
+                            p.q + (static_cast<int64_t>(b) * p.num_heads + head0 + (v ? h : 0)) * D)
+                      : reinterpret_cast<const uint32_t*>(qbuf + stage * kQBytes) + (v ? h : 0) * (D / 2);
 #pragma unroll
       for (int ks = 0; ks < MT; ++ks) {
-        qf[ks][nt][0] = v ? __ldg(qrow + ks * 8 + q) : 0u;
-        qf[ks][nt][1] = v ? __ldg(qrow + ks * 8 + 4 + q) : 0u;
+        qf[ks][nt][0] = v ? (SPLIT_HEADS ? __ldg(qrow + ks * 8 + q) : qrow[ks * 8 + q]) : 0u;
+        qf[ks][nt][1] = v ? (SPLIT_HEADS ? __ldg(qrow + ks * 8 + 4 + q) : qrow[ks * 8 + 4 + q]) : 0u;
       }
     }
 #pragma unroll
@@ -601,7 +794,7 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
       return;
     }
     const StageInfo si = info[stage];
-    if (si.flags & kFirstOfPiece) load_q(si.b, si.seg);
+    if (si.flags & kFirstOfPiece) load_q(si.b, si.seg, stage);
 
     const uint32_t kst = ring + stage * G_::kStageBytes;
     if constexpr (SPLIT_HEADS) {
@@ -622,10 +815,13 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
                                kofs, vofs, qf, o, mref, lsum, sl2, g, q);
       }
     }
+    const bool piece_end = si.flags & kLastOfPiece;
     __syncwarp();
-    if (lane == 0) ptx::mbar_arrive(empty_bar + 8 * stage);
+    // A token-split piece end keeps the stage: the epilogue warp releases it after the
+    // combine (it arrives for all C consumers).
+    if (lane == 0 && (SPLIT_HEADS || !piece_end)) ptx::mbar_arrive(empty_bar + 8 * stage);
 
-    if (!(si.flags & kLastOfPiece)) continue;
+    if (!piece_end) continue;
 
     // ------------------------------------------------------------ end of a piece
     float lt[NT][2];
@@ -678,60 +874,37 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
         }
       if (!sole) cross_cta(si);
     } else {
-      // Token split: combine the C consumers' partial states in shared memory.
-      float* ml = mls + piece_parity * (C * NH * 2);
-      piece_parity ^= 1;
+      // Token split: hand the piece to the epilogue warp.  This consumer's partial O^T
+      // (relative to its own reference max) goes into the tiles of its sub-chunk, which
+      // only it read; its (max, sum) pairs into cml[stage][j].
+      float* mlj = cml + (stage * C + j) * NH * 2;
       if (g == 0) {
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
             const int h = nt * 8 + 2 * q + e;
-            ml[(j * NH + h) * 2] = mref[nt][e];
-            ml[(j * NH + h) * 2 + 1] = lt[nt][e];
+            mlj[h * 2] = mref[nt][e];
+            mlj[h * 2 + 1] = lt[nt][e];
           }
       }
-      ptx::named_barrier_sync(1, NCT);
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
+      for (int nt = 0; nt < NT; ++nt) {
+        float* reg = reinterpret_cast<float*>(base_ptr + stage * G_::kStageBytes +
+                                              (nt ? G_::kTileBytes : 0) + j * G_::kSubBytes);
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          const int h = nt * 8 + 2 * q + e;
-          float M = -INFINITY;
-#pragma unroll
-          for (int jj = 0; jj < C; ++jj) M = fmaxf(M, ml[(jj * NH + h) * 2]);
-          const float wgt = (mref[nt][e] == -INFINITY) ? 0.f : ptx::ex2(mref[nt][e] - M);
-          float* dst = os + (j * NH + h) * D;
+          float* row = reg + (2 * q + e) * D;
 #pragma unroll
           for (int mt = 0; mt < MT; ++mt) {
-            dst[mt * 16 + g] = o[mt][nt][e] * wgt;
-            dst[mt * 16 + g + 8] = o[mt][nt][e + 2] * wgt;
+            row[mt * 16 + g] = o[mt][nt][e];
+            row[mt * 16 + g + 8] = o[mt][nt][e + 2];
           }
         }
-      ptx::named_barrier_sync(1, NCT);
-      for (int idx = tid; idx < nrows_seg * D; idx += NCT) {
-        const int h = idx / D, d = idx - (idx / D) * D;
-        float M = -INFINITY;
-#pragma unroll
-        for (int jj = 0; jj < C; ++jj) M = fmaxf(M, ml[(jj * NH + h) * 2]);
-        float L = 0.f, acc = 0.f;
-#pragma unroll
-        for (int jj = 0; jj < C; ++jj) {
-          const float mj = ml[(jj * NH + h) * 2];
-          if (mj != -INFINITY) L += ml[(jj * NH + h) * 2 + 1] * ptx::ex2(mj - M);
-          acc += os[(jj * NH + h) * D + d];
-        }
-        if (sole) {
-          reinterpret_cast<__nv_bfloat16*>(p.out)[(row0 + h) * D + d] =
-              __float2bfloat16_rn(L > 0.f ? acc / L : 0.f);
-        } else {
-          p.part_o[(static_cast<int64_t>(slot) * hps + h) * D + d] = acc;
-          if (d == 0)
-            *reinterpret_cast<float2*>(p.part_ml + (static_cast<int64_t>(slot) * hps + h) * 2) =
-                make_float2(M, L);
-        }
       }
-      if (!sole) cross_cta(si);
+      ptx::fence_proxy_async_smem();  // the stage will be refilled by TMA later
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(comb_bar + 8 * stage);
     }
   }
 }
@@ -743,14 +916,16 @@ namespace {
 template <int D, int NT, bool SPLIT_HEADS, int C>
 struct Cfg {
   static constexpr int kNH = 8 * NT;
-  static constexpr size_t kMerge =
-      SPLIT_HEADS ? 0 : (static_cast<size_t>(C) * kNH * D + 2 * C * kNH * 2) * sizeof(float);
+  // token split: per-stage (max, sum) hand-off area, sized for up to 8 stages
+  static constexpr size_t kMerge = SPLIT_HEADS ? 0 : static_cast<size_t>(8 * C * kNH * 2) * sizeof(float);
   static constexpr size_t kBudget =
       static_cast<size_t>(GQA_SMEM_PER_SM_KB) * 1024 / ctas_per_sm<SPLIT_HEADS>();
-  static constexpr int kStagesRaw = static_cast<int>((kBudget - kMerge) / Geo<D>::kStageBytes);
+  static constexpr size_t kQBytes = SPLIT_HEADS ? 0 : static_cast<size_t>(kNH) * D * 2;
+  static constexpr int kStagesRaw =
+      static_cast<int>((kBudget - kMerge) / (Geo<D>::kStageBytes + kQBytes));
   static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
-  static constexpr size_t kSmem = 1024 + static_cast<size_t>(kStages) * Geo<D>::kStageBytes + kMerge +
-                                  kStages * (sizeof(StageInfo) + 16);
+  static constexpr size_t kSmem = 1024 + static_cast<size_t>(kStages) * (Geo<D>::kStageBytes + kQBytes) + kMerge +
+                                  kStages * (sizeof(StageInfo) + 24);
 };
 
 template <int D, int NT, bool SH, int C>
@@ -767,13 +942,14 @@ cudaError_t launch_t(const DecodeParams& p, const CUtensorMap& tk, const CUtenso
     if (e != cudaSuccess) return e;
     configured_device = dev;
   }
+  const int threads = (C + (SH ? 1 : 2)) * 32;  // consumers, producer, (epilogue)
   if (!overlap) {
-    kern<<<grid, (C + 1) * 32, CF::kSmem, stream>>>(tk, tv, p);
+    kern<<<grid, threads, CF::kSmem, stream>>>(tk, tv, p);
     return cudaGetLastError();
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3((C + 1) * 32);
+  cfg.blockDim = dim3(threads);
   cfg.dynamicSmemBytes = CF::kSmem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -820,6 +996,17 @@ void fill(DecodePlan& pl) {
 // consumers, so one segment covers up to 128 query heads of its kv head.
 DecodePlan plan_decode(int head_dim, int group) {
   DecodePlan pl{};
+  if (group > 32) {
+    // Dense enough for the 5th-generation tensor cores: one 128-row MMA tile of heads.
+    pl.tensor_cores = 1;
+    pl.split_heads = 1;
+    pl.heads_per_seg = group < 128 ? group : 128;
+    pl.n_ht = (group + pl.heads_per_seg - 1) / pl.heads_per_seg;
+    pl.ctas_per_sm = 1;
+    pl.consumers = 4;
+    pl.smem_bytes = decode_tc_smem_bytes(head_dim);
+    return pl;
+  }
   if (group <= 16) {
     pl.split_heads = 0;
     pl.n_tiles = group <= 8 ? 1 : 2;

@@ -138,16 +138,24 @@ struct MapKey {
   int64_t rows;
   int d;
   int dev;
+  int box_rows;
+  int box_groups;
   bool operator==(const MapKey& o) const {
-    return ptr == o.ptr && rows == o.rows && d == o.d && dev == o.dev;
+    return ptr == o.ptr && rows == o.rows && d == o.d && dev == o.dev && box_rows == o.box_rows &&
+           box_groups == o.box_groups;
   }
 };
 
-gqa_status make_pool_map(CUtensorMap* m, const void* pool, int64_t rows, int d, int dev) {
+// A [rows, d] bf16 matrix viewed as a 3-D tensor: 64 columns (128 bytes) x rows x d/64
+// column groups (stride 128 bytes).  One box is 64 columns x box_rows rows x box_groups
+// groups, 128-byte swizzle; it lands as box_groups consecutive [box_rows, 64] tiles.
+// Used for the page pools ([P * Hk * ps, D]) and for q ([B * H, D]).
+gqa_status make_map(CUtensorMap* m, const void* base, int64_t rows, int d, int dev, int box_rows,
+                    int box_groups) {
   static thread_local MapKey keys[8];
   static thread_local CUtensorMap maps[8];
   static thread_local int next = 0;
-  MapKey k{pool, rows, d, dev};
+  MapKey k{base, rows, d, dev, box_rows, box_groups};
   for (int i = 0; i < 8; ++i)
     if (keys[i] == k) {
       *m = maps[i];
@@ -157,9 +165,9 @@ gqa_status make_pool_map(CUtensorMap* m, const void* pool, int64_t rows, int d, 
   if (!enc) return fail(GQA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
   cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(d / 64)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, 128};
-  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(gqa::kChunk), static_cast<cuuint32_t>(d / 64)};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), static_cast<cuuint32_t>(box_groups)};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(pool), dims, strides,
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(GQA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
@@ -167,6 +175,27 @@ gqa_status make_pool_map(CUtensorMap* m, const void* pool, int64_t rows, int d, 
   maps[next] = *m;
   next = (next + 1) % 8;
   return GQA_OK;
+}
+
+// Tensor maps of one decode launch and the launch itself (both kernels).
+cudaError_t launch_with_maps(const gqa::DecodeParams& p, const gqa::DecodePlan& plan,
+                             const void* q, const void* k_pages, const void* v_pages, int64_t rows,
+                             int dev, int grid, cudaStream_t strm, bool overlap, gqa_status* st) {
+  CUtensorMap tk, tv, tq;
+  const int hd = p.head_dim;
+  if (plan.tensor_cores) {
+    const int br = p.page_size < 64 ? p.page_size : 64;
+    *st = make_map(&tk, k_pages, rows, hd, dev, br, 1);
+    if (*st == GQA_OK) *st = make_map(&tv, v_pages, rows, hd, dev, br, 1);
+    if (*st == GQA_OK)
+      *st = make_map(&tq, q, static_cast<int64_t>(p.num_seqs) * p.num_heads, hd, dev, 128, 1);
+    if (*st != GQA_OK) return cudaSuccess;
+    return gqa::launch_decode_tc(p, tk, tv, tq, grid, strm, overlap);
+  }
+  *st = make_map(&tk, k_pages, rows, hd, dev, gqa::kChunk, hd / 64);
+  if (*st == GQA_OK) *st = make_map(&tv, v_pages, rows, hd, dev, gqa::kChunk, hd / 64);
+  if (*st != GQA_OK) return cudaSuccess;
+  return gqa::launch_decode(p, plan, tk, tv, grid, strm, overlap);
 }
 
 }  // namespace
@@ -238,8 +267,8 @@ gqa_status decode_impl(const void* q, const void* k_pages, const void* v_pages,
     return fail(GQA_ERR_INVALID_ARG, "null pointer argument");
   if (!aligned(k_pages, 16) || !aligned(v_pages, 16))
     return fail(GQA_ERR_INVALID_ARG, "k_pages / v_pages must be 16-byte aligned");
-  if (!aligned(q, 4) || !aligned(out, 8))
-    return fail(GQA_ERR_INVALID_ARG, "q must be 4-byte and out 8-byte aligned");
+  if (!aligned(q, 16) || !aligned(out, 8))
+    return fail(GQA_ERR_INVALID_ARG, "q must be 16-byte and out 8-byte aligned");
 
   DeviceState* st;
   int dev;
@@ -266,11 +295,6 @@ gqa_status decode_impl(const void* q, const void* k_pages, const void* v_pages,
                        slots * plan.heads_per_seg * 2, strm);
   if (s != GQA_OK) return s;
 
-  CUtensorMap tk, tv;
-  s = make_pool_map(&tk, k_pages, rows, head_dim, dev);
-  if (s != GQA_OK) return s;
-  s = make_pool_map(&tv, v_pages, rows, head_dim, dev);
-  if (s != GQA_OK) return s;
 
   gqa::DecodeParams p;
   p.q = static_cast<const uint16_t*>(q);
@@ -295,7 +319,9 @@ gqa_status decode_impl(const void* q, const void* k_pages, const void* v_pages,
   p.num_workers = static_cast<int>(workers);
   p.wait_limit_ns = static_cast<uint64_t>(g_wait_limit_ns.load());
   p.arm_without_copy = g_arm_without_copy.load();
-  cudaError_t e = gqa::launch_decode(p, plan, tk, tv, grid, strm, overlap_previous);
+  cudaError_t e = launch_with_maps(p, plan, q, k_pages, v_pages, rows, dev, grid, strm,
+                                   overlap_previous, &s);
+  if (s != GQA_OK) return s;
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   g_launches.fetch_add(1);
   return GQA_OK;
@@ -422,8 +448,8 @@ gqa_status gqa_paged_decode_attn_noalloc(const void* q, const void* k_pages, con
     return fail(GQA_ERR_INVALID_ARG, "null pointer argument");
   if (!aligned(k_pages, 16) || !aligned(v_pages, 16))
     return fail(GQA_ERR_INVALID_ARG, "k_pages / v_pages must be 16-byte aligned");
-  if (!aligned(q, 4) || !aligned(out, 8))
-    return fail(GQA_ERR_INVALID_ARG, "q must be 4-byte and out 8-byte aligned");
+  if (!aligned(q, 16) || !aligned(out, 8))
+    return fail(GQA_ERR_INVALID_ARG, "q must be 16-byte and out 8-byte aligned");
 
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -470,11 +496,6 @@ gqa_status gqa_paged_decode_attn_noalloc(const void* q, const void* k_pages, con
   e = cudaMemsetAsync(scratch, 0, kNoAllocHeaderBytes + segments * sizeof(int32_t), strm);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(allocation-free scratch)");
 
-  CUtensorMap tk, tv;
-  s = make_pool_map(&tk, k_pages, rows, head_dim, dev);
-  if (s != GQA_OK) return s;
-  s = make_pool_map(&tv, v_pages, rows, head_dim, dev);
-  if (s != GQA_OK) return s;
 
   gqa::DecodeParams p;
   p.q = static_cast<const uint16_t*>(q);
@@ -499,7 +520,9 @@ gqa_status gqa_paged_decode_attn_noalloc(const void* q, const void* k_pages, con
   p.num_workers = static_cast<int>(workers);
   p.wait_limit_ns = static_cast<uint64_t>(g_wait_limit_ns.load());
   p.arm_without_copy = g_arm_without_copy.load();
-  e = gqa::launch_decode(p, plan, tk, tv, static_cast<int>(workers), strm);
+  e = launch_with_maps(p, plan, q, k_pages, v_pages, rows, dev, static_cast<int>(workers), strm,
+                       false, &s);
+  if (s != GQA_OK) return s;
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   g_launches.fetch_add(1);
   return GQA_OK;

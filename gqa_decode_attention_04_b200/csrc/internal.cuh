@@ -57,6 +57,7 @@ cudaError_t launch_kv_append(const AppendParams& p, cudaStream_t stream);
 
 // How a (head_dim, group) problem is mapped onto the decode kernel.
 struct DecodePlan {
+  int tensor_cores;   // 1: tcgen05 kernel (large groups), 0: mma.sync warp-specialized kernel
   int split_heads;    // 0: consumers split the 64-token stage by tokens; 1: by query heads
   int n_tiles;        // 8-head MMA n-tiles per consumer
   int consumers;      // consumer (MMA) warps per CTA; one producer warp is added
@@ -71,6 +72,12 @@ DecodePlan plan_decode(int head_dim, int group);
 // overlap_previous: launch with programmatic stream serialization, so the prologue
 // overlaps the preceding kernel of the stream (which must write nothing the decode reads
 // except the K/V pools); the producer waits for that kernel before its first K/V copy.
+// tcgen05 kernel: K/V maps with boxes of min(page_size, 64) rows x 64 columns, one
+// column group per copy; Q map over [num_seqs * num_heads, head_dim] with 128-row boxes.
+cudaError_t launch_decode_tc(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
+                             const CUtensorMap& tq, int grid, cudaStream_t stream, bool overlap);
+size_t decode_tc_smem_bytes(int head_dim);
+
 cudaError_t launch_decode(const DecodeParams& p, const DecodePlan& plan, const CUtensorMap& tmap_k,
                           const CUtensorMap& tmap_v, int grid, cudaStream_t stream,
                           bool overlap_previous = false);

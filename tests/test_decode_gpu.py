@@ -230,3 +230,33 @@ def test_consecutive_steps_rewrite_what_the_previous_decode_read(cuda_device):
     for step, (kn, vn) in enumerate(rows):
         k2, v2 = oracle.kv_append(h["k"], h["v"], bf16_bits(kn), bf16_bits(vn), h["bt"], inp.positions.numpy())
         assert_close(gpu_f64(outs[step]), oracle_out(dict(h, k=k2, v=v2)), what=f"step {step}")
+
+
+# ------------------------------------------------------------------ large groups (tcgen05 path)
+
+TC_CASES = [
+    ([70], 96, 1, 128, 64),                   # MQA, one partial block
+    ([1000, 63, 129], 96, 1, 128, 64),        # MQA, several blocks, ragged tails
+    ([500, 17], 64, 1, 64, 16),               # head_dim 64, page 16 (16-row copies)
+    ([300, 1, 65], 128, 2, 128, 32),          # G = 64 per kv head, page 32
+    ([200, 33], 128, 1, 128, 128),            # G = 128 (full tile), page 128
+    ([150], 200, 1, 64, 16),                  # G = 200: two head tiles per kv head
+    ([257, 2, 31], 48, 1, 128, 16),           # G = 48 (tile partly padding)
+]
+
+
+@pytest.mark.parametrize("case", TC_CASES, ids=lambda c: f"L{len(c[0])}_H{c[1]}_Hk{c[2]}_D{c[3]}_ps{c[4]}")
+def test_large_group_parity(cuda_device, case):
+    seq_lens, H, Hk, D, ps = case
+    inp = make_custom_inputs(seq_lens, H, Hk, D, ps, seed=sum(seq_lens) + H, extra_pages=2)
+    d, out = _run(inp, cuda_device)
+    assert_close(gpu_f64(out), oracle_out(host_arrays(inp)), what=str(case))
+
+
+@pytest.mark.parametrize("workers", [1, 2, 5, 40, 500])
+def test_large_group_forced_splits(cuda_device, workers):
+    """Pieces of one MQA segment spread over many CTAs and merged by log-sum-exp."""
+    inp = make_custom_inputs([3000, 640], 96, 1, 128, 64, seed=44, spike_fraction=0.01)
+    gq.set_num_workers(workers)
+    d, out = _run(inp, cuda_device)
+    assert_close(gpu_f64(out), oracle_out(host_arrays(inp)), what=f"workers={workers}")
