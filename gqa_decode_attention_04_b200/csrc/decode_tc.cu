@@ -2,9 +2,9 @@
 // on the 5th-generation tensor cores (tcgen05, TMEM accumulators).
 //
 // Same result as decode_ws.cu (page "TensorRT对Multi-Query Attention的专项优化支持": decode
-// re-reads all cached K/V; with MQA every query head shares one K/V head, which the plugin
-// computes "without unnecessary copying and broadcasting" of K/V, on tensor cores for QK^T
-// and AV with tiled shared-memory prefetch; tiny-llm "优化" page: paged KV by block table,
+// re-reads all cached K/V; with MQA every query head shares one K/V head, and the plugin
+// never duplicates K/V per query head; QK^T and AV run on tensor cores with K/V tiles
+// prefetched into shared memory; tiny-llm "优化" page: paged KV by block table,
 // FlashDecoding for long contexts).  With G query heads per K/V head the contraction is
 // G flop per cached byte; for G = 96 this is a dense GEMM that CUDA-core or mma.sync code
 // cannot keep up with at HBM speed, so it runs on tcgen05:
@@ -12,19 +12,23 @@
 //   * Work list and split: as decode_ws.cu, with 64-token blocks; one contiguous range of
 //     the (sequence, segment, block) list per CTA, one CTA per SM; a segment covers up to
 //     128 query heads (the MMA's M = 128 rows), more heads use more segments.
-//   * Producer warp: TMA copies of each block's K and V ([64 tokens, 64 dims] boxes,
-//     128-byte swizzle, K-major for K, MN-major use for V) into a ring of stages, and of
-//     the segment's 128 query rows into a double-buffered Q tile at each piece start.
-//   * MMA warp (one thread issues): S_j = Q K_j^T (M=128 heads, N=64 tokens, K=head_dim)
-//     into one of two TMEM buffers; then O += P_{j-1} V_{j-1} with P read from TMEM
-//     (M=128, N=head_dim, K=64 tokens).  Completion is signalled with tcgen05.commit.
-//   * Softmax warpgroup (128 threads, thread r = query head r): reads its S row from TMEM,
-//     online softmax in the log2 domain with a lazily moved reference (O rescaled in TMEM
-//     only when the row maximum rises by more than 8), writes P (bf16) over S in TMEM.
-//     At a piece end it reads its O row, normalises it and writes out, or stores the
-//     piece for the cross-CTA log-sum-exp merge (last CTA to finish merges).
+//   * Producer warp: TMA copies of each block's K and V into a ring of stages (boxes of
+//     the largest power of two rows dividing the page size, at most 64; a 64-row box
+//     carries every column group), block-table entries read ahead through a register
+//     window, and the segment's 128 query rows (one box) at each piece start.
+//   * S warp (one thread issues): S_j = Q K_j^T (M = 128 heads, N = 64 tokens,
+//     K = head_dim) into one of four TMEM buffers, as soon as K_j has landed and the
+//     buffer's previous P V is done.
+//   * P V warp (one thread issues): O_g += P_j[:, half g] V_j[half g] for the two token
+//     halves, P read from TMEM, once both softmax warpgroups have written P_j.
+//   * Two softmax warpgroups (256 threads; warpgroup g owns tokens [32 g, 32 g + 32) of
+//     every block, thread = head row): each runs its own online softmax in the log2
+//     domain over its half with its own O accumulator (rescaled in TMEM only when its
+//     reference rises by more than 8), writing P (bf16) over its half of S.  At a piece
+//     end the two (max, sum, O) are combined; the result is normalised and written out,
+//     or stored for the cross-CTA log-sum-exp merge (the last CTA to finish merges).
 //   * Safety: every wait is bounded; on a timeout all warps leave their loops, the MMA
-//     warp waits for its issued MMAs, and TMEM is released before exit.
+//     warps wait for their issued MMAs, and TMEM is released before exit.
 #include "internal.cuh"
 #include "ptx.cuh"
 
@@ -34,7 +38,14 @@ namespace {
 
 constexpr int kTcBlk = 64;      // tokens per stage
 constexpr int kTcRows = 128;    // MMA M: query-head rows per segment
-constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kTcBufs = 4;      // S/P buffers in TMEM (blocks in flight between the MMAs and the softmax)
+// Warp roles: 0-7 softmax (two warpgroups, each owning half of a block's 64 tokens for all
+// 128 head rows), 8 producer, 9 S MMA issuer (and TMEM owner), 10 P V MMA issuer.
+constexpr int kTcSoftThreads = 256;
+constexpr int kTcWarps = 11;
+constexpr int kTcThreads = 32 * kTcWarps;
+constexpr int kWarpProducer = 8, kWarpS = 9, kWarpPV = 10;
 constexpr float kTcRescale = 8.0f;
 
 template <int D>
@@ -45,10 +56,12 @@ struct TcGeo {
   static constexpr int kStage = 2 * kTile;
   static constexpr int kQGroup = kTcRows * 128;
   static constexpr int kQTile = kGroups * kQGroup;
-  static constexpr int kStages = D == 128 ? 4 : 8;
-  // TMEM columns: S/P buffers 0 and 1 at 0 and 64 (64 fp32 columns each; P, bf16 pairs,
-  // overwrites the first 32), O at 128 (D columns).
-  static constexpr uint32_t kS0 = 0, kS1 = 64, kO = 128;
+  static constexpr int kStages = D == 128 ? 5 : 10;
+  // TMEM columns: S/P buffer k at 64 k (64 fp32 columns each; the bf16 pairs of P of
+  // tokens 0-31 overwrite columns 0-15, of tokens 32-63 columns 32-47), then one O
+  // accumulator (D columns) per softmax warpgroup.
+  static constexpr uint32_t kO0 = 64 * kTcBufs, kO1 = kO0 + D;
+  static_assert(kO1 + D <= kTmemCols, "TMEM columns");
 };
 
 struct TcStageInfo {
@@ -69,13 +82,15 @@ struct TcCursor {
 }  // namespace
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kTcThreads, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                  const __grid_constant__ CUtensorMap tmap_q, const DecodeParams p) {
   using GE = TcGeo<D>;
   constexpr int S = GE::kStages;
   extern __shared__ uint8_t smem_raw[];
-  __shared__ int64_t s_wtot[6];
+  __shared__ int64_t s_wtot[kTcWarps];
+  __shared__ float s_xmax[2][kTcRows];  // per-piece row references of each warpgroup
+  __shared__ float s_xsum[2][kTcRows];  // per-piece row sums of each warpgroup
   __shared__ int s_start_b;
   __shared__ int64_t s_start_base;
   __shared__ uint32_t s_tmem;
@@ -109,7 +124,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
   }
   __syncthreads();
   int64_t T = 0;
-  for (int i = 0; i < 6; ++i) T += s_wtot[i];
+  for (int i = 0; i < kTcWarps; ++i) T += s_wtot[i];
   const int64_t W = min(static_cast<int64_t>(p.num_workers), T);
   const int64_t w = blockIdx.x;
   if (w >= W) return;
@@ -130,7 +145,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
       if (lane == 31) s_wtot[warp] = incl;
       __syncthreads();
       int64_t pre = 0, tot = 0;
-      for (int i = 0; i < 6; ++i) {
+      for (int i = 0; i < kTcWarps; ++i) {
         if (i < warp) pre += s_wtot[i];
         tot += s_wtot[i];
       }
@@ -153,39 +168,39 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
   const uint32_t pad = (1024u - (smem0 & 1023u)) & 1023u;
   uint8_t* base_ptr = smem_raw + pad;
   const uint32_t ring = smem0 + pad;                        // S stages of K | V
-  const uint32_t qbuf = ring + S * GE::kStage;              // 2 Q tiles
+  const uint32_t qbuf = ring + S * GE::kStage;              // Q tile of the current piece
   uint8_t* vring = base_ptr;                                // generic view of the ring
-  TcStageInfo* info = reinterpret_cast<TcStageInfo*>(base_ptr + S * GE::kStage + 2 * GE::kQTile);
+  TcStageInfo* info = reinterpret_cast<TcStageInfo*>(base_ptr + S * GE::kStage + GE::kQTile);
   const uint32_t bar0 = ptx::smem_u32(info + S);
   const uint32_t full_bar = bar0;                 // [S] producer -> MMA (K/V landed)
   const uint32_t empty_bar = full_bar + 8 * S;    // [S] MMA commit -> producer
-  const uint32_t qfull_bar = empty_bar + 8 * S;   // [2]
-  const uint32_t qempty_bar = qfull_bar + 16;     // [2]
-  const uint32_t sfull_bar = qempty_bar + 16;     // [2] MMA commit -> softmax
-  const uint32_t pfull_bar = sfull_bar + 16;      // [2] softmax (128) -> MMA
-  const uint32_t pv_bar = pfull_bar + 16;         // MMA commit after each PV
-  const uint32_t ofree_bar = pv_bar + 8;          // softmax (128) -> MMA, after a piece's O is read
+  const uint32_t qfull_bar = empty_bar + 8 * S;   // producer -> S warp (piece k: phase k)
+  const uint32_t qempty_bar = qfull_bar + 8;      // S warp commit -> producer
+  const uint32_t sfull_bar = qempty_bar + 8;             // [kTcBufs] S warp commit -> softmax
+  const uint32_t pfull_bar = sfull_bar + 8 * kTcBufs;    // [kTcBufs] softmax (256) -> P V warp
+  const uint32_t pv_bar = pfull_bar + 8 * kTcBufs;       // [kTcBufs] P V warp commit after block j's P V
+  const uint32_t ofree_bar = pv_bar + 8 * kTcBufs;       // softmax (256) -> P V warp, a piece's O is read
   const uint32_t drain_bar = ofree_bar + 8;       // MMA commit at exit
-  const uint32_t wg_bar = drain_bar + 8;          // softmax warpgroup rendezvous (128)
+  const uint32_t wg_bar = drain_bar + 8;          // rendezvous of both softmax warpgroups (256)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       ptx::mbar_init(full_bar + 8 * s, 1);
       ptx::mbar_init(empty_bar + 8 * s, 1);
     }
-    for (int k = 0; k < 2; ++k) {
-      ptx::mbar_init(qfull_bar + 8 * k, 1);
-      ptx::mbar_init(qempty_bar + 8 * k, 1);
+    ptx::mbar_init(qfull_bar, 1);
+    ptx::mbar_init(qempty_bar, 1);
+    for (int k = 0; k < kTcBufs; ++k) {
       ptx::mbar_init(sfull_bar + 8 * k, 1);
-      ptx::mbar_init(pfull_bar + 8 * k, 128);
+      ptx::mbar_init(pfull_bar + 8 * k, kTcSoftThreads);
+      ptx::mbar_init(pv_bar + 8 * k, 1);
     }
-    ptx::mbar_init(pv_bar, 1);
-    ptx::mbar_init(ofree_bar, 128);
-    ptx::mbar_init(drain_bar, 1);
-    ptx::mbar_init(wg_bar, 128);
+    ptx::mbar_init(ofree_bar, kTcSoftThreads);
+    ptx::mbar_init(drain_bar, 2);  // both MMA-issuing warps
+    ptx::mbar_init(wg_bar, kTcSoftThreads);
     ptx::fence_mbarrier_init();
   }
-  if (warp == 5) ptx::tmem_alloc(ptx::smem_u32(&s_tmem), kTmemCols);
+  if (warp == kWarpS) ptx::tmem_alloc(ptx::smem_u32(&s_tmem), kTmemCols);
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
@@ -208,23 +223,83 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
     atomicExch(&s_abort, 1);
   };
 
-  if (warp == 4) {
+  if (warp == kWarpProducer) {
     // ============================================================ producer warp
+    // One iteration per 64-token block.  The loop is a single warp's serial instruction
+    // stream, so it carries no integer division and no 64-bit index arithmetic: page
+    // positions advance incrementally and divisions happen once per piece.
+    if (lane == 0) {
+      ptx::prefetch_tensormap(&tmap_k);
+      ptx::prefetch_tensormap(&tmap_v);
+      ptx::prefetch_tensormap(&tmap_q);
+    }
     const uint64_t policy = ptx::policy_evict_first();
     const int ps = p.page_size;
-    const int R = ps < kTcBlk ? ps : kTcBlk;   // rows per TMA box (one page or one block)
-    const int nchunks = kTcBlk / R;           // lanes < nchunks each copy one box row range
+    const int R = tc_box_rows(ps);           // rows per TMA box: divides both 64 and ps
+    const int nchunks = kTcBlk / R;          // boxes (page pieces) per block and tensor
+    // A 64-row box carries every 64-column group at once (its shared-memory image is the
+    // [group][64 rows][128 B] tile the MMAs read); shorter boxes carry one group each.
+    const int box_groups = R == kTcBlk ? GE::kGroups : 1;
+    const int gsteps = GE::kGroups / box_groups;
+    const int nops = 2 * nchunks * gsteps;   // copies per block, one per lane
+    // This lane's copy: tensor (K or V), chunk and column group.
+    const int op_t = lane / (nchunks * gsteps);
+    const int op_c = (lane % (nchunks * gsteps)) / gsteps;
+    const int op_g = (lane % gsteps) * box_groups;
+    const int cl = lane & (nchunks - 1);     // chunk whose page this lane tracks
+    const uint32_t tile_bytes = 2u * GE::kGroups * R * 128u;  // K + V bytes of one chunk
+    // Block-table rows are read 32 entries at a time (one per lane) into a register window,
+    // with the window needed next already in flight, so no copy waits on a dependent load.
+    // Window boundaries (entry 32 k starts at token 32 k ps, a multiple of 512) fall on
+    // block boundaries, so one block's entries share a window.
+    auto load_window = [&](int b, int k) -> int {
+      const int e = 32 * k + lane;
+      return (b >= 0 && b < B && e < p.max_blocks)
+                 ? __ldg(p.block_table + static_cast<int64_t>(b) * p.max_blocks + e) : -1;
+    };
+    int wb = -1, wk = -1, wval = -1;  // window in use: row wb, entries [32 wk, 32 wk + 32)
+    int nb = -1, nk = -1, nval = -1;  // window prefetched next
     int next_len = (cu.b + 1 < B) ? __ldg(p.seq_lens + cu.b + 1) : 0;
+    // Chunk cl of the cursor's block starts at token t = 64 blk + cl R: block-table entry
+    // pe = t / ps, row po = t % ps inside that page.
+    int pe = 0, po = 0, kvh = 0, ht = 0, q_row0 = 0;
+    auto start_piece = [&]() {
+      const int t = cu.blk * kTcBlk + cl * R;
+      pe = t / ps;
+      po = t - pe * ps;
+      kvh = cu.seg / p.n_ht;
+      ht = cu.seg - kvh * p.n_ht;
+      q_row0 = cu.b * p.num_heads + kvh * p.group + ht * hps;
+    };
+    auto page_of = [&]() -> int {  // this lane's chunk page, -1 past the sequence end
+      const int k = pe >> 5;
+      if (cu.b != wb || k != wk) {
+        wval = (cu.b == nb && k == nk) ? nval : load_window(cu.b, k);
+        wb = cu.b;
+        wk = k;
+        const int entries = (cu.len + ps - 1) / ps;
+        if (32 * (k + 1) < entries) { nb = cu.b; nk = k + 1; }
+        else if (cu.seg + 1 < segs) { nb = cu.b; nk = 0; }
+        else { nb = cu.b + 1; nk = 0; }
+        nval = load_window(nb, nk);
+      }
+      const int pg = __shfl_sync(0xffffffffu, wval, pe & 31);
+      return (lane < nchunks && cu.blk * kTcBlk + cl * R < cu.len) ? pg : -1;
+    };
+    start_piece();
     int64_t seg_base = x0 - cu.blk;
     int piece = 0;
     bool first_piece = true;
     int piece_blk0 = cu.blk;
+    int page = page_of();
+    int stage = 0;
+    uint32_t round = 0;  // times the ring has wrapped
     int64_t i = 0;
+    ptx::pdl_wait_prerequisites();  // K/V pools may be written by the previous kernel
     for (; i < total; ++i) {
       if (__any_sync(0xffffffffu, aborted())) break;  // warp-uniform
-      const int stage = static_cast<int>(i % S);
-      if (i >= S) {
-        const bool ok = ptx::mbar_wait_bounded(empty_bar + 8 * stage, static_cast<uint32_t>((i / S - 1) & 1), limit);
+      if (round > 0) {
+        const bool ok = ptx::mbar_wait_bounded(empty_bar + 8 * stage, (round - 1) & 1u, limit);
         if (!__all_sync(0xffffffffu, ok)) {
           if (lane == 0) abort_all(kErrTimeout);
           break;
@@ -232,45 +307,36 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
       }
       const bool first = (i == 0) || cu.blk == 0;
       const bool last = (i + 1 == total) || (cu.blk + 1 == cu.nblk);
-      if (first) piece_blk0 = cu.blk;
-      const int kvh = cu.seg / p.n_ht, ht = cu.seg % p.n_ht;
       if (first) {
-        // Q rows of this piece's segment into buffer piece & 1 (freed by the MMA warp).
-        const int qb = piece & 1;
+        piece_blk0 = cu.blk;
+        // Q rows of this piece's segment (the previous piece's S MMAs must be done with it).
         bool ok = true;
-        if (piece >= 2)
-          ok = ptx::mbar_wait_bounded(qempty_bar + 8 * qb, static_cast<uint32_t>((piece / 2 - 1) & 1), limit);
+        if (piece >= 1)
+          ok = ptx::mbar_wait_bounded(qempty_bar, static_cast<uint32_t>((piece - 1) & 1), limit);
         if (!__all_sync(0xffffffffu, ok)) {
           if (lane == 0) abort_all(kErrTimeout);
           break;
         }
         if (lane == 0) {
-          if (i == 0) ptx::pdl_wait_prerequisites();
-          ptx::mbar_arrive_expect_tx(qfull_bar + 8 * qb, p.arm_without_copy ? 1u : GE::kQTile);
-          if (!p.arm_without_copy) {
-            const int row0 = cu.b * p.num_heads + kvh * p.group + ht * hps;
-#pragma unroll
-            for (int g = 0; g < GE::kGroups; ++g)
-              ptx::tma_load_3d(qbuf + qb * GE::kQTile + g * GE::kQGroup, &tmap_q, qfull_bar + 8 * qb, 0, row0, g, 0);
-          }
+          ptx::mbar_arrive_expect_tx(qfull_bar, p.arm_without_copy ? 1u : GE::kQTile);
+          if (!p.arm_without_copy)  // one box: 128 rows x every column group
+            ptx::tma_load_3d(qbuf, &tmap_q, qfull_bar, 0, q_row0, 0, 0);
         }
       }
       const int nvalid = min(kTcBlk, cu.len - cu.blk * kTcBlk);
-      int page = -1;
       const bool want = lane < nchunks && lane * R < nvalid;
-      if (want) {
-        const int t = cu.blk * kTcBlk + lane * R;
-        page = __ldg(p.block_table + static_cast<int64_t>(cu.b) * p.max_blocks + t / ps);
-      }
       const bool ok = want && page >= 0 && page < p.num_pages;
-      if (__any_sync(0xffffffffu, want && !ok) && lane == 0) atomicOr(p.err, kErrBounds);
+      const uint32_t wantbits = __ballot_sync(0xffffffffu, want);
       const uint32_t okbits = __ballot_sync(0xffffffffu, ok);
-      const uint32_t nload = __popc(okbits);
-      uint64_t vmask = 0;
-      for (int c = 0; c < nchunks; ++c)
-        if ((okbits >> c) & 1u) vmask |= (R >= 64 ? ~0ull : ((1ull << R) - 1ull)) << (c * R);
-      if (nvalid < kTcBlk) vmask &= (1ull << nvalid) - 1ull;
+      const int op_page = __shfl_sync(0xffffffffu, page, op_c);
+      const int op_po = __shfl_sync(0xffffffffu, po, op_c);
       if (lane == 0) {
+        if (wantbits != okbits) atomicOr(p.err, kErrBounds);
+        uint64_t vmask = 0;
+        const uint64_t chunk_mask = R >= 64 ? ~0ull : ((1ull << R) - 1ull);
+        for (int c = 0; c < nchunks; ++c)
+          if ((okbits >> c) & 1u) vmask |= chunk_mask << (c * R);
+        if (nvalid < kTcBlk) vmask &= (1ull << nvalid) - 1ull;
         TcStageInfo& si = info[stage];
         si.seg_base = seg_base;
         si.vmask = vmask;
@@ -283,30 +349,33 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
         si.flags = (first ? kTcFirst : 0) | (last ? kTcLast : 0) |
                    ((last && piece_blk0 == 0 && cu.blk + 1 == cu.nblk) ? kTcSole : 0) |
                    (first_piece ? kTcFirstPieceOfCta : 0);
-        const uint32_t bytes = p.arm_without_copy ? 0u : nload * 2u * GE::kGroups * R * 128u;
+        const uint32_t bytes = p.arm_without_copy ? 0u : __popc(okbits) * tile_bytes;
         if (bytes) ptx::mbar_arrive_expect_tx(full_bar + 8 * stage, bytes);
         else if (p.arm_without_copy) ptx::mbar_arrive_expect_tx(full_bar + 8 * stage, 1u);
         else ptx::mbar_arrive(full_bar + 8 * stage);
       }
-      if (i == 0 && lane == 0 && !first) ptx::pdl_wait_prerequisites();
       __syncwarp();
-      if (ok && !p.arm_without_copy) {
-        const int t = cu.blk * kTcBlk + lane * R;
-        const int row = (page * p.num_kv_heads + kvh) * ps + t % ps;
-        const uint32_t kdst = ring + stage * GE::kStage + lane * R * 128;
-        const uint32_t vdst = kdst + GE::kTile;
-#pragma unroll
-        for (int g = 0; g < GE::kGroups; ++g) {
-          ptx::tma_load_3d(kdst + g * GE::kGroupBytes, &tmap_k, full_bar + 8 * stage, 0, row, g, policy);
-          ptx::tma_load_3d(vdst + g * GE::kGroupBytes, &tmap_v, full_bar + 8 * stage, 0, row, g, policy);
-        }
+      if (lane < nops && ((okbits >> op_c) & 1u) && !p.arm_without_copy) {
+        const int row = (op_page * p.num_kv_heads + kvh) * ps + op_po;
+        const uint32_t dst = ring + stage * GE::kStage + op_t * GE::kTile + op_g * GE::kGroupBytes + op_c * R * 128;
+        ptx::tma_load_3d(dst, op_t ? &tmap_v : &tmap_k, full_bar + 8 * stage, 0, row, op_g, policy);
+      }
+      if (++stage == S) {
+        stage = 0;
+        ++round;
       }
       if (last) {
         first_piece = false;
         ++piece;
       }
       if (i + 1 < total) {
-        if (++cu.blk >= cu.nblk) {
+        if (++cu.blk < cu.nblk) {
+          po += kTcBlk;  // next block of the same piece
+          while (po >= ps) {
+            po -= ps;
+            ++pe;
+          }
+        } else {
           cu.blk = 0;
           if (++cu.seg >= segs) {
             cu.seg = 0;
@@ -318,28 +387,74 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
             } while (cu.nblk == 0 && cu.b + 1 < B);
           }
           seg_base = x0 + i + 1;
+          start_piece();
         }
+        page = page_of();
       }
     }
     // Let copies still in flight land before the CTA can exit.
     for (int64_t j = (i > S ? i - S : 0); j < i; ++j)
       ptx::mbar_wait_bounded(full_bar + 8 * (j % S), static_cast<uint32_t>((j / S) & 1), limit);
-  } else if (warp == 5) {
-    // ============================================================ MMA warp
+  } else if (warp == kWarpS) {
+    // ============================================================ S warp
+    // S_n = Q K_n^T into TMEM buffer n % kTcBufs once block n's K has landed and the P V of
+    // block n - kTcBufs (issued by the P V warp, reading P from the same buffer) is complete.
     constexpr uint32_t idS = ptx::umma_idesc_bf16(kTcRows, kTcBlk, false);
+    for (int64_t n = 0; n < total; ++n) {
+      if (__any_sync(0xffffffffu, aborted())) break;  // warp-uniform
+      const int stage = static_cast<int>(n % S);
+      bool ok = ptx::mbar_wait_bounded(full_bar + 8 * stage, static_cast<uint32_t>((n / S) & 1), limit);
+      const TcStageInfo si = info[stage];
+      if (ok && (si.flags & kTcFirst))
+        ok = ptx::mbar_wait_bounded(qfull_bar, static_cast<uint32_t>(si.piece & 1), limit);
+      if (ok && n >= kTcBufs)
+        ok = ptx::mbar_wait_bounded(pv_bar + 8 * (n % kTcBufs),
+                                    static_cast<uint32_t>(((n - kTcBufs) / kTcBufs) & 1), limit);
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) abort_all(kErrTimeout);
+        break;
+      }
+      ptx::tc_fence_after();
+      if (lane == 0) {
+        const int sb = static_cast<int>(n % kTcBufs);
+        const uint32_t kb = ring + stage * GE::kStage;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint64_t a = ptx::umma_desc_sw128(qbuf + (ks >> 2) * GE::kQGroup + (ks & 3) * 32, 16, 1024);
+          const uint64_t b = ptx::umma_desc_sw128(kb + (ks >> 2) * GE::kGroupBytes + (ks & 3) * 32, 16, 1024);
+          ptx::umma_ss(tmem + 64 * sb, a, b, idS, ks > 0 ? 1u : 0u);
+        }
+        ptx::umma_commit(sfull_bar + 8 * sb);
+        if (si.flags & kTcLast) ptx::umma_commit(qempty_bar);  // Q tile no longer read
+      }
+      __syncwarp();
+    }
+    // Every MMA issued by this warp completes before TMEM can be released.
+    if (lane == 0) ptx::umma_commit(drain_bar);
+    __syncwarp();
+    ptx::mbar_wait_bounded(drain_bar, 0, limit);
+  } else if (warp == kWarpPV) {
+    // ============================================================ P V warp
+    // O += P_m V_m as soon as the softmax has written P_m (and, at a piece start, has read
+    // the previous piece's O out).
     constexpr uint32_t idPV = ptx::umma_idesc_bf16(kTcRows, D, true);
-    int64_t pend = -1;            // block whose P V is not issued yet
-    int pend_stage = 0, pend_first = 0, pend_piece = 0;
-    uint64_t pend_vmask = 0;
-    bool failed = false;
-    // O += P_j V_j for a pending block j.
-    auto issue_pv = [&](int64_t j, int stage, uint64_t vmask, int first, int piece) -> bool {
-      const int sb = static_cast<int>(j & 1);
-      bool ok = ptx::mbar_wait_bounded(pfull_bar + 8 * sb, static_cast<uint32_t>((j / 2) & 1), limit);
-      if (ok && first && piece > 0)  // the previous piece's O has been read out
-        ok = ptx::mbar_wait_bounded(ofree_bar, static_cast<uint32_t>((piece - 1) & 1), limit);
-      if (!__all_sync(0xffffffffu, ok)) return false;
-      if (vmask != ~0ull) {
+    for (int64_t m = 0; m < total; ++m) {
+      if (__any_sync(0xffffffffu, aborted())) break;  // warp-uniform
+      const int k = static_cast<int>(m % kTcBufs);
+      const int stage = static_cast<int>(m % S);
+      bool ok = ptx::mbar_wait_bounded(pfull_bar + 8 * k, static_cast<uint32_t>((m / kTcBufs) & 1), limit);
+      // V_m landed before S_m was issued; observing the copy barrier here as well orders
+      // the TMA writes before this warp's own stores and MMAs (it has already completed).
+      if (ok) ok = ptx::mbar_wait_bounded(full_bar + 8 * stage, static_cast<uint32_t>((m / S) & 1), limit);
+      const TcStageInfo si = info[stage];  // the stage is held until this P V completes
+      const bool first = si.flags & kTcFirst;
+      if (ok && first && si.piece > 0)
+        ok = ptx::mbar_wait_bounded(ofree_bar, static_cast<uint32_t>((si.piece - 1) & 1), limit);
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) abort_all(kErrTimeout);
+        break;
+      }
+      if (si.vmask != ~0ull) {
         // Rows of tokens past the sequence end (or of pages that failed the range check)
         // may hold any bits, NaN included: zero them in V so 0 * NaN cannot reach O.
         // (Their scores are masked to -inf by the softmax.)
@@ -347,7 +462,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
         for (int idx = lane; idx < kTcBlk * 8 * GE::kGroups; idx += 32) {
           const int g = idx / (kTcBlk * 8);
           const int r = (idx / 8) % kTcBlk, c = idx % 8;
-          if (!((vmask >> r) & 1ull))
+          if (!((si.vmask >> r) & 1ull))
             *reinterpret_cast<uint4*>(v + g * GE::kGroupBytes + r * 128 + c * 16) = make_uint4(0, 0, 0, 0);
         }
         ptx::fence_proxy_async_smem();
@@ -356,104 +471,63 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
       ptx::tc_fence_after();
       if (lane == 0) {
         const uint32_t vb = ring + stage * GE::kStage + GE::kTile;
-        const uint32_t pt = tmem + (sb ? GE::kS1 : GE::kS0);
+        const uint32_t pt = tmem + 64 * k;
 #pragma unroll
         for (int ks = 0; ks < kTcBlk / 16; ++ks) {
           const uint64_t bdesc = ptx::umma_desc_sw128(vb + ks * 16 * 128, GE::kGroupBytes, 1024);
-          ptx::umma_ts(tmem + GE::kO, pt + ks * 8, bdesc, idPV, (first && ks == 0) ? 0u : 1u);
+          // Tokens 0-31 accumulate into warpgroup 0's O, tokens 32-63 into warpgroup 1's;
+          // P of tokens 16 ks .. 16 ks + 15 sits at column 32 (ks / 2) + 8 (ks % 2).
+          ptx::umma_ts(tmem + (ks < 2 ? GE::kO0 : GE::kO1), pt + (ks >> 1) * 32 + (ks & 1) * 8, bdesc,
+                       idPV, (first && (ks & 1) == 0) ? 0u : 1u);
         }
-        ptx::umma_commit(empty_bar + 8 * stage);  // K_j and V_j are consumed
-        ptx::umma_commit(pv_bar);
+        ptx::umma_commit(empty_bar + 8 * stage);  // K_m and V_m are consumed
+        ptx::umma_commit(pv_bar + 8 * k);
       }
       __syncwarp();
-      return true;
-    };
-    for (int64_t i = 0; i < total && !failed; ++i) {
-      if (__any_sync(0xffffffffu, aborted())) break;  // warp-uniform
-      const int stage = static_cast<int>(i % S);
-      bool ok = ptx::mbar_wait_bounded(full_bar + 8 * stage, static_cast<uint32_t>((i / S) & 1), limit);
-      const TcStageInfo si = info[stage];
-      const int qb = si.piece & 1;
-      if (ok && (si.flags & kTcFirst))
-        ok = ptx::mbar_wait_bounded(qfull_bar + 8 * qb, static_cast<uint32_t>((si.piece / 2) & 1), limit);
-      if (!__all_sync(0xffffffffu, ok)) {
-        if (lane == 0) abort_all(kErrTimeout);
-        failed = true;
-        break;
-      }
-      ptx::tc_fence_after();
-      const int sb = static_cast<int>(i & 1);
-      if (lane == 0) {
-        const uint32_t kb = ring + stage * GE::kStage;
-        const uint32_t qt = qbuf + qb * GE::kQTile;
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const uint64_t a = ptx::umma_desc_sw128(qt + (ks >> 2) * GE::kQGroup + (ks & 3) * 32, 16, 1024);
-          const uint64_t b = ptx::umma_desc_sw128(kb + (ks >> 2) * GE::kGroupBytes + (ks & 3) * 32, 16, 1024);
-          ptx::umma_ss(tmem + (sb ? GE::kS1 : GE::kS0), a, b, idS, ks > 0 ? 1u : 0u);
-        }
-        ptx::umma_commit(sfull_bar + 8 * sb);
-        if (si.flags & kTcLast) ptx::umma_commit(qempty_bar + 8 * qb);  // Q tile no longer read
-      }
-      __syncwarp();
-      if (pend >= 0) {
-        if (!issue_pv(pend, pend_stage, pend_vmask, pend_first, pend_piece)) {
-          if (lane == 0) abort_all(kErrTimeout);
-          failed = true;
-          break;
-        }
-        pend = -1;
-      }
-      pend = i;
-      pend_stage = stage;
-      pend_vmask = si.vmask;
-      pend_first = (si.flags & kTcFirst) ? 1 : 0;
-      pend_piece = si.piece;
-      if (si.flags & kTcLast) {  // finish the piece now so its O can be read out
-        if (!issue_pv(pend, pend_stage, pend_vmask, pend_first, pend_piece)) {
-          if (lane == 0) abort_all(kErrTimeout);
-          failed = true;
-          break;
-        }
-        pend = -1;
-      }
     }
-    // Every MMA issued by this warp completes before TMEM can be released.
     if (lane == 0) ptx::umma_commit(drain_bar);
     __syncwarp();
     ptx::mbar_wait_bounded(drain_bar, 0, limit);
   } else {
-    // ============================================================ softmax warpgroup
-    const int r = threadIdx.x;              // query-head row of the segment tile
-    const uint32_t lane_off = static_cast<uint32_t>(32 * warp) << 16;
+    // ============================================================ softmax warpgroups
+    // Thread t: warpgroup g = t / 128 owns tokens [32 g, 32 g + 32) of every block and its
+    // own O accumulator in TMEM; row r = t % 128 is query head r of the segment tile
+    // (TMEM lane r).  The two warpgroups run independent online softmaxes over their
+    // halves (no per-block exchange) and combine the two (max, sum, O) at a piece end.
+    const int t = threadIdx.x;
+    const int g = t >> 7, r = t & (kTcRows - 1);
+    const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+    const uint32_t o_mine = tmem + lane_off + (g ? GE::kO1 : GE::kO0);
     const float sl2 = p.scale_log2;
+    const bool pos = sl2 >= 0.f;  // a negative scale turns the row maximum into a minimum
+    constexpr int HD = D / 2;     // output columns each warpgroup finishes at a piece end
     float mref = -INFINITY, lsum = 0.f;
-    int64_t pv_seen = 0;  // PV completions consumed (one per block, in order)
     int wg_phase = 0;
     bool failed = false;
     // Every wait outcome is made warp-uniform: the TMEM loads and stores that follow are
     // warp-collective (.sync.aligned) and must never run on part of a warp.
-    auto wait_pv_upto = [&](int64_t n) -> bool {
-      while (pv_seen < n) {
-        const bool ok = ptx::mbar_wait_bounded(pv_bar, static_cast<uint32_t>(pv_seen & 1), limit);
-        if (!__all_sync(0xffffffffu, ok)) return false;
-        ++pv_seen;
-      }
-      return true;
+    // P V MMAs are issued by one thread and complete in order, so "the P V of block j is
+    // complete" (phase j / kTcBufs of pv_bar[j % kTcBufs]) covers every earlier block.  It
+    // is only waited for at block i with j >= i - 1: the barrier's next phase (block
+    // j + kTcBufs) needs a P this warpgroup has not written yet, so parity is unambiguous.
+    auto wait_pv_done = [&](int64_t j) -> bool {
+      const bool ok = ptx::mbar_wait_bounded(pv_bar + 8 * (j % kTcBufs),
+                                             static_cast<uint32_t>((j / kTcBufs) & 1), limit);
+      return __all_sync(0xffffffffu, ok);
     };
-    auto wg_sync = [&]() -> bool {  // all 128 threads (bounded)
+    auto wg_sync = [&]() -> bool {  // all 256 softmax threads (bounded)
       ptx::mbar_arrive(wg_bar);
       const bool ok = ptx::mbar_wait_bounded(wg_bar, static_cast<uint32_t>(wg_phase & 1), limit);
       ++wg_phase;
       return __all_sync(0xffffffffu, ok);
     };
     for (int64_t i = 0; i < total && !failed; ++i) {
-      if (__any_sync(0xffffffffu, aborted())) break;  // warp-uniform
-      const int sb = static_cast<int>(i & 1);
-      bool ok = __all_sync(0xffffffffu,
-                           ptx::mbar_wait_bounded(sfull_bar + 8 * sb, static_cast<uint32_t>((i / 2) & 1), limit));
-      if (ok && i > 0) ok = wait_pv_upto(i);  // P_{i-1} V_{i-1} is in O
-      if (!ok) {
+      // Another warp's failed wait ends the CTA; checked every 8 blocks (each wait here is
+      // bounded, so a stale flag only costs time).
+      if ((i & 7) == 0 && __any_sync(0xffffffffu, aborted())) break;
+      const int sb = static_cast<int>(i % kTcBufs);
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait_bounded(sfull_bar + 8 * sb,
+                                                          static_cast<uint32_t>((i / kTcBufs) & 1), limit))) {
         abort_all(kErrTimeout);
         failed = true;
         break;
@@ -465,34 +539,62 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
         mref = -INFINITY;
         lsum = 0.f;
       }
-      const uint32_t st = tmem + lane_off + (sb ? GE::kS1 : GE::kS0);
-      uint32_t u0[32], u1[32];
-      ptx::tmem_ld32(st, u0);
-      ptx::tmem_ld32(st + 32, u1);
+      const uint32_t st = tmem + lane_off + 64 * sb;
+      uint32_t u[32];
+      ptx::tmem_ld32(st + 32 * g, u);
       ptx::tmem_wait_ld();
-      float s[64];
+      // Scores of tokens outside the sequence (or of pages that failed the range check)
+      // may be anything, NaN included: they take the raw value that scales to -inf.
+      const uint32_t vm = static_cast<uint32_t>(si.vmask >> (32 * g));
+      const bool full = vm == 0xffffffffu;
+      if (!full) {
+        const uint32_t off = pos ? 0xff800000u : 0x7f800000u;  // -inf / +inf
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        s[c] = ((si.vmask >> c) & 1ull) ? __uint_as_float(u0[c]) * sl2 : -INFINITY;
-        s[32 + c] = ((si.vmask >> (32 + c)) & 1ull) ? __uint_as_float(u1[c]) * sl2 : -INFINITY;
+        for (int c = 0; c < 32; ++c)
+          if (!((vm >> c) & 1u)) u[c] = off;
       }
-      float mx = -INFINITY;
+      // Row maximum of this half's scaled scores (log2 domain), a tree over raw scores.
+      float mx;
+      {
+        float tt[16];
+        if (pos) {
 #pragma unroll
-      for (int c = 0; c < 64; ++c) mx = fmaxf(mx, s[c]);
+          for (int c = 0; c < 16; ++c) tt[c] = fmaxf(__uint_as_float(u[c]), __uint_as_float(u[c + 16]));
+#pragma unroll
+          for (int w2 = 8; w2 > 0; w2 >>= 1)
+#pragma unroll
+            for (int c = 0; c < w2; ++c) tt[c] = fmaxf(tt[c], tt[c + w2]);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) tt[c] = fminf(__uint_as_float(u[c]), __uint_as_float(u[c + 16]));
+#pragma unroll
+          for (int w2 = 8; w2 > 0; w2 >>= 1)
+#pragma unroll
+            for (int c = 0; c < w2; ++c) tt[c] = fminf(tt[c], tt[c + w2]);
+        }
+        mx = tt[0] * sl2;
+        if (mx != mx) mx = -INFINITY;  // every token masked and a zero scale
+      }
       const bool need = mx > mref + kTcRescale;
       if (__any_sync(0xffffffffu, need)) {
         const float alpha = need ? ptx::ex2(mref - mx) : 1.f;  // 0 when mref = -inf
         if (!first) {
-          // Rescale O rows in TMEM (P V of earlier blocks are complete).  The whole warp
-          // takes part; rows that keep their reference scale by 1.
+          // Rescale this warpgroup's O rows in TMEM once every earlier P V is in.  The
+          // whole warp takes part; rows that keep their reference scale by 1.
+          if (!wait_pv_done(i - 1)) {
+            abort_all(kErrTimeout);
+            failed = true;
+            break;
+          }
+          ptx::tc_fence_after();
 #pragma unroll
           for (int c0 = 0; c0 < D; c0 += 32) {
             uint32_t ov[32];
-            ptx::tmem_ld32(tmem + lane_off + GE::kO + c0, ov);
+            ptx::tmem_ld32(o_mine + c0, ov);
             ptx::tmem_wait_ld();
 #pragma unroll
             for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
-            ptx::tmem_st32(tmem + lane_off + GE::kO + c0, ov);
+            ptx::tmem_st32(o_mine + c0, ov);
           }
           ptx::tmem_wait_st();
         }
@@ -501,63 +603,95 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
           mref = mx;
         }
       }
-      const float mu = (mref == -INFINITY) ? 0.f : mref;
-      uint32_t pk[32];
-      float ls = 0.f;
+      // P = 2^(score * scale_log2 - reference), one FFMA and one ex2 per score; bf16
+      // pairs overwrite the first 16 of this half's own 32 score columns (token 32 g + 2j,
+      // 32 g + 2j + 1 in column 32 g + j), so neither warpgroup touches the other's scores.
+      const float nmu = (mref == -INFINITY) ? 0.f : -mref;
+      uint32_t pk[16];
+      float ls0 = 0.f, ls1 = 0.f, ls2 = 0.f, ls3 = 0.f;
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float a = ptx::ex2(s[2 * c] - mu), b2 = ptx::ex2(s[2 * c + 1] - mu);
-        ls += a + b2;
-        pk[c] = ptx::pack_bf16x2(a, b2);
+      for (int c = 0; c < 32; c += 4) {
+        float a0 = ptx::ex2(fmaf(__uint_as_float(u[c]), sl2, nmu));
+        float a1 = ptx::ex2(fmaf(__uint_as_float(u[c + 1]), sl2, nmu));
+        float a2 = ptx::ex2(fmaf(__uint_as_float(u[c + 2]), sl2, nmu));
+        float a3 = ptx::ex2(fmaf(__uint_as_float(u[c + 3]), sl2, nmu));
+        if (!full) {  // masked scores are exactly 0 (with a zero scale, inf * 0 is NaN)
+          const uint32_t bits = (vm >> c) & 15u;
+          a0 = (bits & 1u) ? a0 : 0.f;
+          a1 = (bits & 2u) ? a1 : 0.f;
+          a2 = (bits & 4u) ? a2 : 0.f;
+          a3 = (bits & 8u) ? a3 : 0.f;
+        }
+        ls0 += a0;
+        ls1 += a1;
+        ls2 += a2;
+        ls3 += a3;
+        pk[c / 2] = ptx::pack_bf16x2(a0, a1);
+        pk[c / 2 + 1] = ptx::pack_bf16x2(a2, a3);
       }
-      lsum += ls;
-      ptx::tmem_st32(st, pk);
+      lsum += (ls0 + ls1) + (ls2 + ls3);
+      ptx::tmem_st16(st + 32 * g, pk);
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       ptx::mbar_arrive(pfull_bar + 8 * sb);
 
       if (!(si.flags & kTcLast)) continue;
       // ---------------------------------------------------------- end of a piece
-      if (!wait_pv_upto(i + 1)) {
+      // Combine the two halves: M = max(m0, m1), O = sum_g O_g 2^(m_g - M),
+      // L = sum_g l_g 2^(m_g - M).  Warpgroup g finishes output columns [g HD, g HD + HD).
+      if (!wait_pv_done(i)) {
         abort_all(kErrTimeout);
         failed = true;
         break;
       }
       ptx::tc_fence_after();
+      s_xmax[g][r] = mref;
+      s_xsum[g][r] = lsum;
+      if (!wg_sync()) {
+        abort_all(kErrTimeout);
+        failed = true;
+        break;
+      }
+      const float m0 = s_xmax[0][r], m1 = s_xmax[1][r];
+      const float Mx = fmaxf(m0, m1);
+      const float Mu = (Mx == -INFINITY) ? 0.f : Mx;
+      const float w0 = ptx::ex2(m0 - Mu), w1 = ptx::ex2(m1 - Mu);  // 0 for an empty half
+      const float ltot = s_xsum[0][r] * w0 + s_xsum[1][r] * w1;
       const int kvh = si.seg / p.n_ht, ht = si.seg % p.n_ht;
       const int nrows = min(hps, p.group - ht * hps);
       const int64_t row0 = static_cast<int64_t>(si.b) * p.num_heads + kvh * p.group + ht * hps;
       const bool sole = si.flags & kTcSole;
       const int64_t slot = w * 2 + ((si.flags & kTcFirstPieceOfCta) ? 0 : 1);
-      const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+      const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
+      const float f0 = sole ? w0 * inv : w0, f1 = sole ? w1 * inv : w1;
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t ov[32];
-        ptx::tmem_ld32(tmem + lane_off + GE::kO + c0, ov);
+      for (int c0 = 0; c0 < HD; c0 += 32) {
+        uint32_t oa[32], ob[32];
+        ptx::tmem_ld32(tmem + lane_off + GE::kO0 + g * HD + c0, oa);
+        ptx::tmem_ld32(tmem + lane_off + GE::kO1 + g * HD + c0, ob);
         ptx::tmem_wait_ld();
-        if (r < nrows) {
-          if (sole) {
-            uint4* dst = reinterpret_cast<uint4*>(p.out + (row0 + r) * D + c0);
+        float o[32];
 #pragma unroll
-            for (int c = 0; c < 32; c += 8) {
-              uint4 v;
-              v.x = ptx::pack_bf16x2(__uint_as_float(ov[c]) * inv, __uint_as_float(ov[c + 1]) * inv);
-              v.y = ptx::pack_bf16x2(__uint_as_float(ov[c + 2]) * inv, __uint_as_float(ov[c + 3]) * inv);
-              v.z = ptx::pack_bf16x2(__uint_as_float(ov[c + 4]) * inv, __uint_as_float(ov[c + 5]) * inv);
-              v.w = ptx::pack_bf16x2(__uint_as_float(ov[c + 6]) * inv, __uint_as_float(ov[c + 7]) * inv);
-              dst[c / 8] = v;
+        for (int c = 0; c < 32; ++c) o[c] = __uint_as_float(oa[c]) * f0 + __uint_as_float(ob[c]) * f1;
+        if (r < nrows) {
+          if (sole) {  // out is only 8-byte aligned: 4 columns per store
+            uint2* dst = reinterpret_cast<uint2*>(p.out + (row0 + r) * D + g * HD + c0);
+#pragma unroll
+            for (int c = 0; c < 32; c += 4) {
+              uint2 v;
+              v.x = ptx::pack_bf16x2(o[c], o[c + 1]);
+              v.y = ptx::pack_bf16x2(o[c + 2], o[c + 3]);
+              dst[c / 4] = v;
             }
           } else {
-            float4* dst = reinterpret_cast<float4*>(p.part_o + (slot * hps + r) * D + c0);
+            float4* dst = reinterpret_cast<float4*>(p.part_o + (slot * hps + r) * D + g * HD + c0);
 #pragma unroll
-            for (int c = 0; c < 32; c += 4)
-              dst[c / 4] = make_float4(__uint_as_float(ov[c]), __uint_as_float(ov[c + 1]),
-                                       __uint_as_float(ov[c + 2]), __uint_as_float(ov[c + 3]));
+            for (int c = 0; c < 32; c += 4) dst[c / 4] = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
           }
         }
       }
-      if (!sole && r < nrows)
-        *reinterpret_cast<float2*>(p.part_ml + (slot * hps + r) * 2) = make_float2(mref, lsum);
+      if (!sole && g == 0 && r < nrows)
+        *reinterpret_cast<float2*>(p.part_ml + (slot * hps + r) * 2) = make_float2(Mx, ltot);
       ptx::tc_fence_before();
       ptx::mbar_arrive(ofree_bar);  // O may be overwritten by the next piece
       if (sole) continue;
@@ -569,7 +703,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
         break;
       }
       const int64_t segid = static_cast<int64_t>(si.b) * segs + si.seg;
-      if (r == 0) s_prev = atomicAdd(p.counters + segid, 1);
+      if (t == 0) s_prev = atomicAdd(p.counters + segid, 1);
       if (!wg_sync()) {
         abort_all(kErrTimeout);
         failed = true;
@@ -580,46 +714,79 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
       const int64_t wl = tc_worker_of(si.seg_base + si.nblk - 1, T, W);
       if (prev != static_cast<int>(wl - wf)) continue;
       __threadfence();
-      if (r < nrows) {
-        uint4* dst = reinterpret_cast<uint4*>(p.out + (row0 + r) * D);
-        for (int c0 = 0; c0 < D; c0 += 64) {  // 64 columns of this row at a time
-          float M = -INFINITY, Ls = 0.f;
-          float acc[64];
+      {
+        // Piece k of the segment belongs to worker wf + k.  For k > 0 that worker's range
+        // starts inside the segment, so the piece is its first (slot 0); worker wf's piece
+        // is its first only if its range starts exactly at the segment start.
+        const int np = static_cast<int>(wl - wf + 1);
+        const int64_t slot0 = wf * 2 + (si.seg_base <= tc_wstart(wf, T, W) ? 0 : 1);
+        auto slot_of = [&](int k) -> int64_t { return k == 0 ? slot0 : (wf + k) * 2; };
+        // Lanes across columns (coalesced rows): warp q merges rows q*4 .. q*4+3, then
+        // the next 32 rows; 4 rows x 4 pieces of (max, sum) and values per round trip.
+        constexpr int CW = D / 32;  // columns per lane
+        const int q = t >> 5, ln = t & 31;
+        for (int h0 = q * 4; h0 < nrows; h0 += 32) {
+          float M[4], L[4], acc[4][CW];
 #pragma unroll
-          for (int c = 0; c < 64; ++c) acc[c] = 0.f;
-          for (int64_t ww = wf; ww <= wl; ++ww) {
-            const int64_t sl = ww * 2 + (si.seg_base <= tc_wstart(ww, T, W) ? 0 : 1);
-            const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.part_ml + (sl * hps + r) * 2));
-            const float4* src = reinterpret_cast<const float4*>(p.part_o + (sl * hps + r) * D + c0);
-            float4 v[16];
+          for (int j = 0; j < 4; ++j) {
+            M[j] = -INFINITY;
+            L[j] = 0.f;
 #pragma unroll
-            for (int k = 0; k < 16; ++k) v[k] = __ldcg(src + k);
-            const float mn = fmaxf(M, ml.x);
-            const float mu2 = (mn == -INFINITY) ? 0.f : mn;
-            const float a = ptx::ex2(M - mu2), bw = ptx::ex2(ml.x - mu2);
-            Ls = Ls * a + ml.y * bw;
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-              acc[4 * k] = acc[4 * k] * a + v[k].x * bw;
-              acc[4 * k + 1] = acc[4 * k + 1] * a + v[k].y * bw;
-              acc[4 * k + 2] = acc[4 * k + 2] * a + v[k].z * bw;
-              acc[4 * k + 3] = acc[4 * k + 3] * a + v[k].w * bw;
-            }
-            M = mn;
+            for (int c = 0; c < CW; ++c) acc[j][c] = 0.f;
           }
-          const float iv = Ls > 0.f ? 1.f / Ls : 0.f;
+          for (int k0 = 0; k0 < np; k0 += 4) {
+            float2 ml[4][4];
+            float v[4][4][CW];
 #pragma unroll
-          for (int c = 0; c < 64; c += 8) {
-            uint4 u;
-            u.x = ptx::pack_bf16x2(acc[c] * iv, acc[c + 1] * iv);
-            u.y = ptx::pack_bf16x2(acc[c + 2] * iv, acc[c + 3] * iv);
-            u.z = ptx::pack_bf16x2(acc[c + 4] * iv, acc[c + 5] * iv);
-            u.w = ptx::pack_bf16x2(acc[c + 6] * iv, acc[c + 7] * iv);
-            dst[(c0 + c) / 8] = u;
+            for (int k = 0; k < 4; ++k) {
+              const int64_t sl = slot_of(k0 + k < np ? k0 + k : 0);
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const bool act = k0 + k < np && h0 + j < nrows;
+                const int64_t e = sl * hps + min(h0 + j, nrows - 1);
+                ml[k][j] = act ? __ldcg(reinterpret_cast<const float2*>(p.part_ml + e * 2))
+                               : make_float2(-INFINITY, 0.f);
+                if constexpr (CW == 4) {
+                  const float4 x = act ? __ldcg(reinterpret_cast<const float4*>(p.part_o + e * D) + ln)
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+                  v[k][j][0] = x.x; v[k][j][1] = x.y; v[k][j][2] = x.z; v[k][j][3] = x.w;
+                } else {
+                  const float2 x = act ? __ldcg(reinterpret_cast<const float2*>(p.part_o + e * D) + ln)
+                                       : make_float2(0.f, 0.f);
+                  v[k][j][0] = x.x; v[k][j][1] = x.y;
+                }
+              }
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const float mn = fmaxf(M[j], ml[k][j].x);
+                const float mu = (mn == -INFINITY) ? 0.f : mn;
+                const float a = ptx::ex2(M[j] - mu), bw = ptx::ex2(ml[k][j].x - mu);
+                L[j] = L[j] * a + ml[k][j].y * bw;
+#pragma unroll
+                for (int c = 0; c < CW; ++c) acc[j][c] = acc[j][c] * a + v[k][j][c] * bw;
+                M[j] = mn;
+              }
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if (h0 + j >= nrows) continue;
+            const float iv = L[j] > 0.f ? 1.f / L[j] : 0.f;
+            uint16_t* dst = p.out + (row0 + h0 + j) * D + ln * CW;
+            if constexpr (CW == 4) {
+              uint2 o;
+              o.x = ptx::pack_bf16x2(acc[j][0] * iv, acc[j][1] * iv);
+              o.y = ptx::pack_bf16x2(acc[j][2] * iv, acc[j][3] * iv);
+              *reinterpret_cast<uint2*>(dst) = o;
+            } else {
+              *reinterpret_cast<uint32_t*>(dst) = ptx::pack_bf16x2(acc[j][0] * iv, acc[j][1] * iv);
+            }
           }
         }
       }
-      if (r == 0) p.counters[segid] = 0;
+      if (t == 0) p.counters[segid] = 0;
     }
   }
 
@@ -627,7 +794,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
-  if (warp == 5) ptx::tmem_dealloc(tmem, kTmemCols);
+  if (warp == kWarpS) ptx::tmem_dealloc(tmem, kTmemCols);
 }
 
 // ------------------------------------------------------------------ host side
@@ -635,8 +802,8 @@ namespace {
 template <int D>
 constexpr size_t tc_smem_bytes() {
   using GE = TcGeo<D>;
-  return 1024 + static_cast<size_t>(GE::kStages) * GE::kStage + 2 * GE::kQTile +
-         GE::kStages * sizeof(TcStageInfo) + 16 * GE::kStages + 128;
+  return 1024 + static_cast<size_t>(GE::kStages) * GE::kStage + GE::kQTile +
+         GE::kStages * sizeof(TcStageInfo) + 16 * GE::kStages + 24 * kTcBufs + 64;
 }
 
 template <int D>
@@ -654,7 +821,7 @@ cudaError_t launch_tc_t(const DecodeParams& p, const CUtensorMap& tk, const CUte
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(192);
+  cfg.blockDim = dim3(kTcThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];

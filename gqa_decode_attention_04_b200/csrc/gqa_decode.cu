@@ -184,11 +184,12 @@ cudaError_t launch_with_maps(const gqa::DecodeParams& p, const gqa::DecodePlan& 
   CUtensorMap tk, tv, tq;
   const int hd = p.head_dim;
   if (plan.tensor_cores) {
-    const int br = p.page_size < 64 ? p.page_size : 64;
-    *st = make_map(&tk, k_pages, rows, hd, dev, br, 1);
-    if (*st == GQA_OK) *st = make_map(&tv, v_pages, rows, hd, dev, br, 1);
+    const int br = gqa::tc_box_rows(p.page_size);
+    const int bg = br == 64 ? hd / 64 : 1;  // a 64-row box carries every column group
+    *st = make_map(&tk, k_pages, rows, hd, dev, br, bg);
+    if (*st == GQA_OK) *st = make_map(&tv, v_pages, rows, hd, dev, br, bg);
     if (*st == GQA_OK)
-      *st = make_map(&tq, q, static_cast<int64_t>(p.num_seqs) * p.num_heads, hd, dev, 128, 1);
+      *st = make_map(&tq, q, static_cast<int64_t>(p.num_seqs) * p.num_heads, hd, dev, 128, hd / 64);
     if (*st != GQA_OK) return cudaSuccess;
     return gqa::launch_decode_tc(p, tk, tv, tq, grid, strm, overlap);
   }

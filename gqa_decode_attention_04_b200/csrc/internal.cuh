@@ -23,6 +23,14 @@ constexpr int kSubChunks = kBlock / kChunk;
 // Most query heads one segment (kv head x head tile) covers; partial slots hold this many.
 constexpr int kMaxSegHeads = 128;
 
+// Rows of one K/V copy of the tcgen05 kernel: the largest power of two dividing the page
+// size, at most one block, so a copy never straddles two pages and a block is a whole
+// number of copies.
+__host__ __device__ __forceinline__ int tc_box_rows(int page_size) {
+  const int low = page_size & -page_size;
+  return low < kBlock ? low : kBlock;
+}
+
 struct DecodeParams {
   const uint16_t* q;          // [B, H, D] bf16
   uint16_t* out;              // [B, H, D] bf16
@@ -72,8 +80,9 @@ DecodePlan plan_decode(int head_dim, int group);
 // overlap_previous: launch with programmatic stream serialization, so the prologue
 // overlaps the preceding kernel of the stream (which must write nothing the decode reads
 // except the K/V pools); the producer waits for that kernel before its first K/V copy.
-// tcgen05 kernel: K/V maps with boxes of min(page_size, 64) rows x 64 columns, one
-// column group per copy; Q map over [num_seqs * num_heads, head_dim] with 128-row boxes.
+// tcgen05 kernel: K/V maps with boxes of tc_box_rows(page_size) rows x 64 columns and
+// every column group when that is 64 rows, one group otherwise; Q map over
+// [num_seqs * num_heads, head_dim] with boxes of 128 rows x every column group.
 cudaError_t launch_decode_tc(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
                              const CUtensorMap& tq, int grid, cudaStream_t stream, bool overlap);
 size_t decode_tc_smem_bytes(int head_dim);

@@ -110,7 +110,7 @@ gqa_status gqa_kv_append(const void* k_new, const void* v_new, void* k_pages, vo
  *   seq_lens[b]     context length of sequence b including any token appended this
  *                   step; 0 gives an all-zero output row.
  * Requirements: head_dim in {64, 128}; page_size a multiple of 16 in [16, 256];
- * num_heads % num_kv_heads == 0; q, out 4-byte aligned; k_pages, v_pages 16-byte
+ * num_heads % num_kv_heads == 0; q 16-byte and out 8-byte aligned; k_pages, v_pages 16-byte
  * aligned; num_seqs <= 65536.  Slots at or beyond seq_lens[b] and unused pages may
  * hold any bits (NaN included) without affecting out.
  */

@@ -130,6 +130,33 @@ def test_large_scale_peaked_softmax(cuda_device):
     assert_close(gpu_f64(out), oracle_out(host_arrays(inp)), what="peaked")
 
 
+@pytest.mark.parametrize("heads", [(16, 2), (96, 1)], ids=["gqa", "mqa"])
+@pytest.mark.parametrize("scale", [0.0, -0.3], ids=["zero", "negative"])
+def test_zero_and_negative_scale(cuda_device, heads, scale):
+    """Any finite scale: 0 gives the plain mean of V over each sequence; a negative scale
+    favours the smallest scores.  Poisoned slots past each length must stay masked."""
+    H, Hk = heads
+    inp = make_custom_inputs([300, 45, 130], H, Hk, 128, 16, seed=19, extra_pages=3, scale=scale)
+    _, out = _run(inp, cuda_device)
+    assert_close(gpu_f64(out), oracle_out(host_arrays(inp)), what=f"scale={scale}")
+
+
+@pytest.mark.parametrize("heads", [(8, 2), (96, 1)], ids=["gqa", "mqa"])
+def test_out_only_8_byte_aligned(cuda_device, heads):
+    """out may start on any 8-byte boundary (here 8 bytes past a 16-byte one)."""
+    H, Hk = heads
+    inp = make_custom_inputs([260, 70], H, Hk, 128, 16, seed=20)
+    d = inp.to(cuda_device)
+    n = 2 * H * 128
+    buf = torch.full((n + 8,), float("nan"), dtype=torch.bfloat16, device=cuda_device)
+    out = buf[4:4 + n].view(2, H, 128)
+    assert out.data_ptr() % 16 == 8
+    gq.paged_decode_attn(d.q, d.k_pages, d.v_pages, d.block_table, d.seq_lens, out=out, scale=d.scale)
+    torch.cuda.synchronize()
+    assert_close(gpu_f64(out), oracle_out(host_arrays(inp)), what="misaligned out")
+    assert torch.isnan(buf[:4].float()).all() and torch.isnan(buf[4 + n:].float()).all()
+
+
 def test_out_buffer_is_written_in_place(cuda_device):
     inp = make_custom_inputs([40, 9], 4, 1, 64, 16, seed=18)
     d = inp.to(cuda_device)
@@ -242,6 +269,13 @@ TC_CASES = [
     ([200, 33], 128, 1, 128, 128),            # G = 128 (full tile), page 128
     ([150], 200, 1, 64, 16),                  # G = 200: two head tiles per kv head
     ([257, 2, 31], 48, 1, 128, 16),           # G = 48 (tile partly padding)
+    ([400, 5], 64, 1, 64, 64),                # head_dim 64, page 64 (one box per block)
+    ([700, 90], 96, 1, 128, 256),             # page 256: four blocks per page
+    ([2100, 700, 3], 64, 1, 128, 16),         # block-table rows spanning several windows
+    ([1500, 47], 96, 1, 128, 48),             # page 48: blocks straddle pages (16-row copies)
+    ([900, 130], 64, 1, 128, 80),             # page 80
+    ([1100, 96], 40, 1, 64, 96),              # page 96 (32-row copies), head_dim 64
+    ([800, 193], 72, 1, 128, 192),            # page 192: 64-row copies, three blocks per page
 ]
 
 
