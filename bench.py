@@ -39,9 +39,17 @@ from workloads import WORKLOADS, make_inputs, bf16_bits  # noqa: E402
 METRIC = "paged GQA decode attn: achieved HBM TB/s (% of B200 peak), tokens/s"
 FALLBACK_HBM_GBS = 6650.0
 PROFILE_TRAFFIC = os.path.join(ROOT, "profiles", "traffic.json")
-KERNEL_SOURCES = ["gqa_decode_attention_04_b200/csrc/decode_ws.cu",
-                  "gqa_decode_attention_04_b200/csrc/ptx.cuh",
-                  "gqa_decode_attention_04_b200/csrc/internal.cuh"]
+_CSRC = "gqa_decode_attention_04_b200/csrc/"
+KERNEL_SOURCES = {
+    "decode_ws_kernel": [_CSRC + "decode_ws.cu", _CSRC + "ptx.cuh", _CSRC + "internal.cuh"],
+    "decode_tc_kernel": [_CSRC + "decode_tc.cu", _CSRC + "ptx.cuh", _CSRC + "internal.cuh"],
+}
+
+
+def decode_kernel_for(inp) -> str:
+    """The decode kernel the library picks for this head grouping: the tcgen05 kernel
+    for more than 32 query heads per kv head, the mma.sync kernel otherwise."""
+    return "decode_tc_kernel" if inp.num_heads // inp.num_kv_heads > 32 else "decode_ws_kernel"
 
 
 # ------------------------------------------------------------------ helpers
@@ -74,15 +82,15 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_sha() -> str:
+def kernel_source_sha(kernel: str) -> str:
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload_name: str, units_per_launch: int):
+def profiled_traffic(workload_name: str, kernel: str, units_per_launch: int):
     """DRAM bytes per launch from a committed ncu capture, if it was taken of the
     current kernel source; scaled to this launch's units when the capture was of a
     smaller case.  None when absent or stale."""
@@ -90,7 +98,7 @@ def profiled_traffic(workload_name: str, units_per_launch: int):
         with open(PROFILE_TRAFFIC) as f:
             j = json.load(f)
         e = j[workload_name]
-        if e.get("kernel_source_sha") != kernel_source_sha():
+        if not e.get("kernel", "").startswith(kernel) or e.get("kernel_source_sha") != kernel_source_sha(kernel):
             return None
         per_unit = e["dram_bytes_per_launch"] / e["units_per_launch"]
         return int(round(per_unit * units_per_launch))
@@ -429,10 +437,10 @@ def run_ours(args, rank, world, local):
         "e2e": {"value": e2e_tbps, "unit": "TB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms / args.steps},
         "gpu_launches": int(launches),
-        "roofline": {"bound": "hbm", "kernel": "decode_ws_kernel",
+        "roofline": {"bound": "hbm", "kernel": decode_kernel_for(inp_cpu),
                      "achieved": achieved_gbs, "peak": peak, "unit": "GB/s",
                      "frac": achieved_gbs / peak, "peak_kind": f"{peak_kind} (hbm_gbs)",
-                     "traffic": profiled_traffic(WORKLOADS[args.workload].name, units),
+                     "traffic": profiled_traffic(WORKLOADS[args.workload].name, decode_kernel_for(inp_cpu), units),
                      "algorithmic_bytes_per_launch": nbytes["decode"],
                      "decode_ms": decode_ms_local},
         "clocks": clocks.summary(),
