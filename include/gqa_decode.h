@@ -37,7 +37,9 @@
  *
  *   Token t of sequence b is slot (t % page_size) of page block_table[b][t / page_size];
  *   query head h reads kv head h / (num_heads / num_kv_heads).  Block-table entries
- *   past ceil(seq_lens[b] / page_size) are never read.
+ *   past ceil(seq_lens[b] / page_size) are never used and may hold any value (the
+ *   decode kernels load rows of the table 32 entries at a time, so such entries inside
+ *   the [num_seqs, max_blocks_per_seq] array may be loaded, never dereferenced).
  *
  *   `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  Calls
  *   only enqueue work: they never synchronise the stream and never read device data
