@@ -41,11 +41,12 @@ constexpr int kTcRows = 128;    // MMA M: query-head rows per segment
 constexpr uint32_t kTmemCols = 512;
 constexpr int kTcBufs = 4;      // S/P buffers in TMEM (blocks in flight between the MMAs and the softmax)
 // Warp roles: 0-7 softmax (two warpgroups, each owning half of a block's 64 tokens for all
-// 128 head rows), 8 producer, 9 S MMA issuer (and TMEM owner), 10 P V MMA issuer.
+// 128 head rows), 8 and 11 producers (even and odd blocks), 9 S MMA issuer (and TMEM
+// owner), 10 P V MMA issuer.
 constexpr int kTcSoftThreads = 256;
-constexpr int kTcWarps = 11;
+constexpr int kTcWarps = 12;
 constexpr int kTcThreads = 32 * kTcWarps;
-constexpr int kWarpProducer = 8, kWarpS = 9, kWarpPV = 10;
+constexpr int kWarpProducer = 8, kWarpS = 9, kWarpPV = 10, kWarpProducer2 = 11;
 constexpr float kTcRescale = 8.0f;
 
 template <int D>
@@ -223,11 +224,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
     atomicExch(&s_abort, 1);
   };
 
-  if (warp == kWarpProducer) {
-    // ============================================================ producer warp
-    // One iteration per 64-token block.  The loop is a single warp's serial instruction
-    // stream, so it carries no integer division and no 64-bit index arithmetic: page
-    // positions advance incrementally and divisions happen once per piece.
+  if (warp == kWarpProducer || warp == kWarpProducer2) {
+    // ============================================================ producer warps
+    // Both walk every 64-token block of the range; producer `pid` issues the blocks with
+    // i % 2 == pid (its stage descriptor, copy barrier, K/V copies, and the piece's Q copy
+    // when the block starts a piece), so the serial per-block issue work is split in two.
+    // The loop carries no integer division and no 64-bit index arithmetic: page positions
+    // advance incrementally and divisions happen once per piece.
+    const uint32_t pid = warp == kWarpProducer ? 0u : 1u;
     if (lane == 0) {
       ptx::prefetch_tensormap(&tmap_k);
       ptx::prefetch_tensormap(&tmap_v);
@@ -297,6 +301,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
     int64_t i = 0;
     ptx::pdl_wait_prerequisites();  // K/V pools may be written by the previous kernel
     for (; i < total; ++i) {
+      const bool mine = (static_cast<uint32_t>(i) & 1u) == pid;
+      const bool first = (i == 0) || cu.blk == 0;
+      const bool last = (i + 1 == total) || (cu.blk + 1 == cu.nblk);
+      if (first) piece_blk0 = cu.blk;
+      if (mine) {
       if (__any_sync(0xffffffffu, aborted())) break;  // warp-uniform
       if (round > 0) {
         const bool ok = ptx::mbar_wait_bounded(empty_bar + 8 * stage, (round - 1) & 1u, limit);
@@ -305,10 +314,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
           break;
         }
       }
-      const bool first = (i == 0) || cu.blk == 0;
-      const bool last = (i + 1 == total) || (cu.blk + 1 == cu.nblk);
       if (first) {
-        piece_blk0 = cu.blk;
         // Q rows of this piece's segment (the previous piece's S MMAs must be done with it).
         bool ok = true;
         if (piece >= 1)
@@ -360,6 +366,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
         const uint32_t dst = ring + stage * GE::kStage + op_t * GE::kTile + op_g * GE::kGroupBytes + op_c * R * 128;
         ptx::tma_load_3d(dst, op_t ? &tmap_v : &tmap_k, full_bar + 8 * stage, 0, row, op_g, policy);
       }
+      }  // mine
       if (++stage == S) {
         stage = 0;
         ++round;
@@ -392,9 +399,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
         page = page_of();
       }
     }
-    // Let copies still in flight land before the CTA can exit.
+    // Let this producer's copies still in flight land before the CTA can exit.
     for (int64_t j = (i > S ? i - S : 0); j < i; ++j)
-      ptx::mbar_wait_bounded(full_bar + 8 * (j % S), static_cast<uint32_t>((j / S) & 1), limit);
+      if ((static_cast<uint32_t>(j) & 1u) == pid)
+        ptx::mbar_wait_bounded(full_bar + 8 * (j % S), static_cast<uint32_t>((j / S) & 1), limit);
   } else if (warp == kWarpS) {
     // ============================================================ S warp
     // S_n = Q K_n^T into TMEM buffer n % kTcBufs once block n's K has landed and the P V of
@@ -521,20 +529,34 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
       ++wg_phase;
       return __all_sync(0xffffffffu, ok);
     };
+    int is = 0;  // stage of block i (i % S, kept incrementally)
     for (int64_t i = 0; i < total && !failed; ++i) {
       // Another warp's failed wait ends the CTA; checked every 8 blocks (each wait here is
       // bounded, so a stale flag only costs time).
-      if ((i & 7) == 0 && __any_sync(0xffffffffu, aborted())) break;
-      const int sb = static_cast<int>(i % kTcBufs);
-      if (!__all_sync(0xffffffffu, ptx::mbar_wait_bounded(sfull_bar + 8 * sb,
-                                                          static_cast<uint32_t>((i / kTcBufs) & 1), limit))) {
+      const uint32_t i32 = static_cast<uint32_t>(i);  // buffer / phase arithmetic mod 2^32
+      if ((i32 & 7u) == 0 && __any_sync(0xffffffffu, aborted())) break;
+      const int sb = static_cast<int>(i32 % kTcBufs);
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait_bounded(sfull_bar + 8 * sb, (i32 / kTcBufs) & 1u, limit))) {
         abort_all(kErrTimeout);
         failed = true;
         break;
       }
       ptx::tc_fence_after();
-      const TcStageInfo si = info[i % S];
-      const bool first = si.flags & kTcFirst;
+      const int stg = is;
+      if (++is == S) is = 0;
+      const int flags = info[stg].flags;
+      const uint64_t vmask = info[stg].vmask;
+      // What a piece end needs of this block, read while its stage is held (the stage is
+      // refilled once the block's P V completes, which needs this thread's P).
+      int pe_b = 0, pe_seg = 0, pe_nblk = 0;
+      int64_t pe_base = 0;
+      if (flags & kTcLast) {
+        pe_b = info[stg].b;
+        pe_seg = info[stg].seg;
+        pe_nblk = info[stg].nblk;
+        pe_base = info[stg].seg_base;
+      }
+      const bool first = flags & kTcFirst;
       if (first) {
         mref = -INFINITY;
         lsum = 0.f;
@@ -545,7 +567,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
       ptx::tmem_wait_ld();
       // Scores of tokens outside the sequence (or of pages that failed the range check)
       // may be anything, NaN included: they take the raw value that scales to -inf.
-      const uint32_t vm = static_cast<uint32_t>(si.vmask >> (32 * g));
+      const uint32_t vm = static_cast<uint32_t>(vmask >> (32 * g));
       const bool full = vm == 0xffffffffu;
       if (!full) {
         const uint32_t off = pos ? 0xff800000u : 0x7f800000u;  // -inf / +inf
@@ -607,27 +629,27 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
       // pairs overwrite the first 16 of this half's own 32 score columns (token 32 g + 2j,
       // 32 g + 2j + 1 in column 32 g + j), so neither warpgroup touches the other's scores.
       const float nmu = (mref == -INFINITY) ? 0.f : -mref;
+      // Three passes (arguments, exponentials, sums and packing) so the 32 ex2 issue back
+      // to back on the MUFU.
+      float e[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) e[c] = fmaf(__uint_as_float(u[c]), sl2, nmu);
+#pragma unroll
+      for (int c = 0; c < 32; ++c) e[c] = ptx::ex2(e[c]);
+      if (!full) {  // masked scores are exactly 0 (with a zero scale, inf * 0 is NaN)
+#pragma unroll
+        for (int c = 0; c < 32; ++c) e[c] = ((vm >> c) & 1u) ? e[c] : 0.f;
+      }
       uint32_t pk[16];
       float ls0 = 0.f, ls1 = 0.f, ls2 = 0.f, ls3 = 0.f;
 #pragma unroll
       for (int c = 0; c < 32; c += 4) {
-        float a0 = ptx::ex2(fmaf(__uint_as_float(u[c]), sl2, nmu));
-        float a1 = ptx::ex2(fmaf(__uint_as_float(u[c + 1]), sl2, nmu));
-        float a2 = ptx::ex2(fmaf(__uint_as_float(u[c + 2]), sl2, nmu));
-        float a3 = ptx::ex2(fmaf(__uint_as_float(u[c + 3]), sl2, nmu));
-        if (!full) {  // masked scores are exactly 0 (with a zero scale, inf * 0 is NaN)
-          const uint32_t bits = (vm >> c) & 15u;
-          a0 = (bits & 1u) ? a0 : 0.f;
-          a1 = (bits & 2u) ? a1 : 0.f;
-          a2 = (bits & 4u) ? a2 : 0.f;
-          a3 = (bits & 8u) ? a3 : 0.f;
-        }
-        ls0 += a0;
-        ls1 += a1;
-        ls2 += a2;
-        ls3 += a3;
-        pk[c / 2] = ptx::pack_bf16x2(a0, a1);
-        pk[c / 2 + 1] = ptx::pack_bf16x2(a2, a3);
+        ls0 += e[c];
+        ls1 += e[c + 1];
+        ls2 += e[c + 2];
+        ls3 += e[c + 3];
+        pk[c / 2] = ptx::pack_bf16x2(e[c], e[c + 1]);
+        pk[c / 2 + 1] = ptx::pack_bf16x2(e[c + 2], e[c + 3]);
       }
       lsum += (ls0 + ls1) + (ls2 + ls3);
       ptx::tmem_st16(st + 32 * g, pk);
@@ -635,7 +657,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
       ptx::tc_fence_before();
       ptx::mbar_arrive(pfull_bar + 8 * sb);
 
-      if (!(si.flags & kTcLast)) continue;
+      if (!(flags & kTcLast)) continue;
       // ---------------------------------------------------------- end of a piece
       // Combine the two halves: M = max(m0, m1), O = sum_g O_g 2^(m_g - M),
       // L = sum_g l_g 2^(m_g - M).  Warpgroup g finishes output columns [g HD, g HD + HD).
@@ -657,11 +679,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
       const float Mu = (Mx == -INFINITY) ? 0.f : Mx;
       const float w0 = ptx::ex2(m0 - Mu), w1 = ptx::ex2(m1 - Mu);  // 0 for an empty half
       const float ltot = s_xsum[0][r] * w0 + s_xsum[1][r] * w1;
-      const int kvh = si.seg / p.n_ht, ht = si.seg % p.n_ht;
+      const int kvh = pe_seg / p.n_ht, ht = pe_seg % p.n_ht;
       const int nrows = min(hps, p.group - ht * hps);
-      const int64_t row0 = static_cast<int64_t>(si.b) * p.num_heads + kvh * p.group + ht * hps;
-      const bool sole = si.flags & kTcSole;
-      const int64_t slot = w * 2 + ((si.flags & kTcFirstPieceOfCta) ? 0 : 1);
+      const int64_t row0 = static_cast<int64_t>(pe_b) * p.num_heads + kvh * p.group + ht * hps;
+      const bool sole = flags & kTcSole;
+      const int64_t slot = w * 2 + ((flags & kTcFirstPieceOfCta) ? 0 : 1);
       const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
       const float f0 = sole ? w0 * inv : w0, f1 = sole ? w1 * inv : w1;
 #pragma unroll
@@ -702,7 +724,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
         failed = true;
         break;
       }
-      const int64_t segid = static_cast<int64_t>(si.b) * segs + si.seg;
+      const int64_t segid = static_cast<int64_t>(pe_b) * segs + pe_seg;
       if (t == 0) s_prev = atomicAdd(p.counters + segid, 1);
       if (!wg_sync()) {
         abort_all(kErrTimeout);
@@ -710,8 +732,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
         break;
       }
       const int prev = s_prev;
-      const int64_t wf = tc_worker_of(si.seg_base, T, W);
-      const int64_t wl = tc_worker_of(si.seg_base + si.nblk - 1, T, W);
+      const int64_t wf = tc_worker_of(pe_base, T, W);
+      const int64_t wl = tc_worker_of(pe_base + pe_nblk - 1, T, W);
       if (prev != static_cast<int>(wl - wf)) continue;
       __threadfence();
       {
@@ -719,7 +741,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
         // starts inside the segment, so the piece is its first (slot 0); worker wf's piece
         // is its first only if its range starts exactly at the segment start.
         const int np = static_cast<int>(wl - wf + 1);
-        const int64_t slot0 = wf * 2 + (si.seg_base <= tc_wstart(wf, T, W) ? 0 : 1);
+        const int64_t slot0 = wf * 2 + (pe_base <= tc_wstart(wf, T, W) ? 0 : 1);
         auto slot_of = [&](int k) -> int64_t { return k == 0 ? slot0 : (wf + k) * 2; };
         // Lanes across columns (coalesced rows): warp q merges rows q*4 .. q*4+3, then
         // the next 32 rows; 4 rows x 4 pieces of (max, sum) and values per round trip.

@@ -27,8 +27,8 @@
 //       - small groups (G <= 16): each of the 4 consumers takes one 16-token sub-chunk
 //         of every stage for all G heads; at a piece end their partial softmax states
 //         are combined in shared memory.
-//       - large groups (MQA-like, G > 16): each consumer takes 8 or 16 of the query heads
-//         over all 64 tokens of every stage.
+//       - groups of 17..32: each consumer takes 8 of the query heads over all 64
+//         tokens of every stage (larger groups run on the tcgen05 kernel, decode_tc.cu).
 //   * Online softmax in the log2 domain with a lazily moved reference: O and the sum are
 //     rescaled only when a head's running maximum rises by more than 8 (factor 256);
 //     numerator and denominator share the reference, so the result is unchanged.
@@ -966,20 +966,9 @@ cudaError_t launch_d(const DecodeParams& p, const DecodePlan& pl, const CUtensor
   if (!pl.split_heads)
     return pl.n_tiles == 1 ? launch_t<D, 1, false, 4>(p, tk, tv, grid, s, o)
                            : launch_t<D, 2, false, 4>(p, tk, tv, grid, s, o);
-  if (pl.n_tiles == 1) {
-    switch (pl.consumers) {
-      case 3: return launch_t<D, 1, true, 3>(p, tk, tv, grid, s, o);
-      default: return launch_t<D, 1, true, 4>(p, tk, tv, grid, s, o);
-    }
-  }
-  switch (pl.consumers) {
-    case 3: return launch_t<D, 2, true, 3>(p, tk, tv, grid, s, o);
-    case 4: return launch_t<D, 2, true, 4>(p, tk, tv, grid, s, o);
-    case 5: return launch_t<D, 2, true, 5>(p, tk, tv, grid, s, o);
-    case 6: return launch_t<D, 2, true, 6>(p, tk, tv, grid, s, o);
-    case 7: return launch_t<D, 2, true, 7>(p, tk, tv, grid, s, o);
-    default: return launch_t<D, 2, true, 8>(p, tk, tv, grid, s, o);
-  }
+  // Head split (17..32 heads per kv head): one 8-head n-tile per consumer.
+  return pl.consumers == 3 ? launch_t<D, 1, true, 3>(p, tk, tv, grid, s, o)
+                           : launch_t<D, 1, true, 4>(p, tk, tv, grid, s, o);
 }
 
 template <int D, int NT, bool SH, int C>
@@ -992,8 +981,8 @@ void fill(DecodePlan& pl) {
 }  // namespace
 
 // Small groups (G <= 16): token split, 4 consumers, one 8- or 16-head tile per segment.
-// Larger groups: head split; 8 heads per consumer up to G = 32, else 16, and up to 8
-// consumers, so one segment covers up to 128 query heads of its kv head.
+// 17..32: head split, 8 heads per consumer, 3 or 4 consumers.  Larger groups run on the
+// tcgen05 kernel (decode_tc.cu), one 128-row MMA tile of heads per segment.
 DecodePlan plan_decode(int head_dim, int group) {
   DecodePlan pl{};
   if (group > 32) {
@@ -1012,15 +1001,11 @@ DecodePlan plan_decode(int head_dim, int group) {
     pl.n_tiles = group <= 8 ? 1 : 2;
     pl.consumers = 4;
     pl.heads_per_seg = 8 * pl.n_tiles;
-  } else {
+  } else {  // 17..32 heads per kv head: one 8-head n-tile per consumer
     pl.split_heads = 1;
-    pl.n_tiles = group <= 32 ? 1 : 2;
-    const int hg = 8 * pl.n_tiles;
-    int c = (group + hg - 1) / hg;
-    if (pl.n_tiles == 1) c = c <= 3 ? 3 : 4;   // 17..24 -> 3, 25..32 -> 4
-    else c = c < 3 ? 3 : (c > 8 ? 8 : c);
-    pl.consumers = c;
-    pl.heads_per_seg = hg * c;
+    pl.n_tiles = 1;
+    pl.consumers = group <= 24 ? 3 : 4;
+    pl.heads_per_seg = 8 * pl.consumers;
   }
   pl.n_ht = (group + pl.heads_per_seg - 1) / pl.heads_per_seg;
   pl.ctas_per_sm = pl.split_heads ? ctas_per_sm<true>() : ctas_per_sm<false>();
@@ -1028,12 +1013,12 @@ DecodePlan plan_decode(int head_dim, int group) {
   const int nt = pl.n_tiles, c = pl.consumers;
   if (head_dim == 64) {
     if (!sh) { if (nt == 1) fill<64, 1, false, 4>(pl); else fill<64, 2, false, 4>(pl); }
-    else if (nt == 1) { if (c == 3) fill<64, 1, true, 3>(pl); else fill<64, 1, true, 4>(pl); }
-    else fill<64, 2, true, 8>(pl);  // stage count does not depend on C for the head split
+    else if (c == 3) fill<64, 1, true, 3>(pl);
+    else fill<64, 1, true, 4>(pl);
   } else {
     if (!sh) { if (nt == 1) fill<128, 1, false, 4>(pl); else fill<128, 2, false, 4>(pl); }
-    else if (nt == 1) { if (c == 3) fill<128, 1, true, 3>(pl); else fill<128, 1, true, 4>(pl); }
-    else fill<128, 2, true, 8>(pl);
+    else if (c == 3) fill<128, 1, true, 3>(pl);
+    else fill<128, 1, true, 4>(pl);
   }
   return pl;
 }
