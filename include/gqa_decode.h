@@ -190,7 +190,7 @@ const char* gqa_last_error_string(void);
 size_t gqa_kv_cache_bytes(int num_layers, int num_kv_heads, int head_dim, int64_t seq_len);
 
 /*
- * gqa_set_num_workers -- number of split workers (one warp each) used by the next
+ * gqa_set_num_workers -- number of split workers (CTAs) used by the next
  * gqa_paged_decode_attn calls on this process; 0 (default) picks it from the SM count.
  * A fixed count changes how the context is split, never the result beyond fp32
  * rounding order; tests use it to force many or few splits.  Returns
