@@ -44,6 +44,7 @@ constexpr int kTcBufs = 4;      // S/P buffers in TMEM (blocks in flight between
 // 128 head rows), 8 and 11 producers (even and odd blocks), 9 S MMA issuer (and TMEM
 // owner), 10 P V MMA issuer.
 constexpr int kTcSoftThreads = 256;
+constexpr int kStgFloats = 16 * 36;  // piece-end staging per softmax warp
 constexpr int kTcWarps = 12;
 constexpr int kTcThreads = 32 * kTcWarps;
 constexpr int kWarpProducer = 8, kWarpS = 9, kWarpPV = 10, kWarpProducer2 = 11;
@@ -183,6 +184,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
   const uint32_t ofree_bar = pv_bar + 8 * kTcBufs;       // softmax (256) -> P V warp, a piece's O is read
   const uint32_t drain_bar = ofree_bar + 8;       // MMA commit at exit
   const uint32_t wg_bar = drain_bar + 8;          // rendezvous of both softmax warpgroups (256)
+  // Piece-end staging: per softmax warp 16 rows x 36 floats, so a warp writes whole
+  // 128-byte row segments of its 32 rows (16 rows per round) instead of one row per lane.
+  float* const stg_all = reinterpret_cast<float*>(base_ptr + ((wg_bar + 8 - ring + 127u) & ~127u));
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -529,6 +533,97 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
       ++wg_phase;
       return __all_sync(0xffffffffu, ok);
     };
+    // Cross-CTA step of a piece that is not the whole segment (its partial is stored):
+    // count the arrival; the last CTA to finish a piece of the segment merges them all.
+    auto cross_cta = [&](int cb, int cseg, int64_t pe_base, int pe_nblk) -> bool {
+      __threadfence();
+      if (!wg_sync()) return false;
+      const int64_t segid = static_cast<int64_t>(cb) * segs + cseg;
+      if (t == 0) s_prev = atomicAdd(p.counters + segid, 1);
+      if (!wg_sync()) return false;
+      const int prev = s_prev;
+      const int64_t wf = tc_worker_of(pe_base, T, W);
+      const int64_t wl = tc_worker_of(pe_base + pe_nblk - 1, T, W);
+      if (prev != static_cast<int>(wl - wf)) return true;
+      __threadfence();
+      const int kvh = cseg / p.n_ht, ht = cseg % p.n_ht;
+      const int nrows = min(hps, p.group - ht * hps);
+      const int64_t row0 = static_cast<int64_t>(cb) * p.num_heads + kvh * p.group + ht * hps;
+        {
+          // Piece k of the segment belongs to worker wf + k.  For k > 0 that worker's range
+          // starts inside the segment, so the piece is its first (slot 0); worker wf's piece
+          // is its first only if its range starts exactly at the segment start.
+          const int np = static_cast<int>(wl - wf + 1);
+          const int64_t slot0 = wf * 2 + (pe_base <= tc_wstart(wf, T, W) ? 0 : 1);
+          auto slot_of = [&](int k) -> int64_t { return k == 0 ? slot0 : (wf + k) * 2; };
+          // Lanes across columns (coalesced rows): warp q merges rows q*4 .. q*4+3, then
+          // the next 32 rows; 4 rows x 4 pieces of (max, sum) and values per round trip.
+          constexpr int CW = D / 32;  // columns per lane
+          const int q = t >> 5, ln = t & 31;
+          for (int h0 = q * 4; h0 < nrows; h0 += 32) {
+            float M[4], L[4], acc[4][CW];
+  #pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              M[j] = -INFINITY;
+              L[j] = 0.f;
+  #pragma unroll
+              for (int c = 0; c < CW; ++c) acc[j][c] = 0.f;
+            }
+            for (int k0 = 0; k0 < np; k0 += 4) {
+              float2 ml[4][4];
+              float v[4][4][CW];
+  #pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const int64_t sl = slot_of(k0 + k < np ? k0 + k : 0);
+  #pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  const bool act = k0 + k < np && h0 + j < nrows;
+                  const int64_t e = sl * hps + min(h0 + j, nrows - 1);
+                  ml[k][j] = act ? __ldcg(reinterpret_cast<const float2*>(p.part_ml + e * 2))
+                                 : make_float2(-INFINITY, 0.f);
+                  if constexpr (CW == 4) {
+                    const float4 x = act ? __ldcg(reinterpret_cast<const float4*>(p.part_o + e * D) + ln)
+                                         : make_float4(0.f, 0.f, 0.f, 0.f);
+                    v[k][j][0] = x.x; v[k][j][1] = x.y; v[k][j][2] = x.z; v[k][j][3] = x.w;
+                  } else {
+                    const float2 x = act ? __ldcg(reinterpret_cast<const float2*>(p.part_o + e * D) + ln)
+                                         : make_float2(0.f, 0.f);
+                    v[k][j][0] = x.x; v[k][j][1] = x.y;
+                  }
+                }
+              }
+  #pragma unroll
+              for (int k = 0; k < 4; ++k)
+  #pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  const float mn = fmaxf(M[j], ml[k][j].x);
+                  const float mu = (mn == -INFINITY) ? 0.f : mn;
+                  const float a = ptx::ex2(M[j] - mu), bw = ptx::ex2(ml[k][j].x - mu);
+                  L[j] = L[j] * a + ml[k][j].y * bw;
+  #pragma unroll
+                  for (int c = 0; c < CW; ++c) acc[j][c] = acc[j][c] * a + v[k][j][c] * bw;
+                  M[j] = mn;
+                }
+            }
+  #pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              if (h0 + j >= nrows) continue;
+              const float iv = L[j] > 0.f ? 1.f / L[j] : 0.f;
+              uint16_t* dst = p.out + (row0 + h0 + j) * D + ln * CW;
+              if constexpr (CW == 4) {
+                uint2 o;
+                o.x = ptx::pack_bf16x2(acc[j][0] * iv, acc[j][1] * iv);
+                o.y = ptx::pack_bf16x2(acc[j][2] * iv, acc[j][3] * iv);
+                *reinterpret_cast<uint2*>(dst) = o;
+              } else {
+                *reinterpret_cast<uint32_t*>(dst) = ptx::pack_bf16x2(acc[j][0] * iv, acc[j][1] * iv);
+              }
+            }
+          }
+        }
+      if (t == 0) p.counters[segid] = 0;
+      return true;
+    };
     int is = 0;  // stage of block i (i % S, kept incrementally)
     for (int64_t i = 0; i < total && !failed; ++i) {
       // Another warp's failed wait ends the CTA; checked every 8 blocks (each wait here is
@@ -686,30 +781,44 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
       const int64_t slot = w * 2 + ((flags & kTcFirstPieceOfCta) ? 0 : 1);
       const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
       const float f0 = sole ? w0 * inv : w0, f1 = sole ? w1 * inv : w1;
+      float* const rows_buf = stg_all + warp * kStgFloats;
 #pragma unroll
       for (int c0 = 0; c0 < HD; c0 += 32) {
         uint32_t oa[32], ob[32];
         ptx::tmem_ld32(tmem + lane_off + GE::kO0 + g * HD + c0, oa);
         ptx::tmem_ld32(tmem + lane_off + GE::kO1 + g * HD + c0, ob);
         ptx::tmem_wait_ld();
-        float o[32];
+        float* o = reinterpret_cast<float*>(oa);  // combined in place (constant indices only)
 #pragma unroll
         for (int c = 0; c < 32; ++c) o[c] = __uint_as_float(oa[c]) * f0 + __uint_as_float(ob[c]) * f1;
-        if (r < nrows) {
-          if (sole) {  // out is only 8-byte aligned: 4 columns per store
-            uint2* dst = reinterpret_cast<uint2*>(p.out + (row0 + r) * D + g * HD + c0);
+        // 16 rows at a time through shared memory: lane l then writes 4 columns of row
+        // (l / 8) + 4m, so 8 lanes cover one 128-byte row segment.
 #pragma unroll
-            for (int c = 0; c < 32; c += 4) {
-              uint2 v;
-              v.x = ptx::pack_bf16x2(o[c], o[c + 1]);
-              v.y = ptx::pack_bf16x2(o[c + 2], o[c + 3]);
-              dst[c / 4] = v;
-            }
-          } else {
-            float4* dst = reinterpret_cast<float4*>(p.part_o + (slot * hps + r) * D + g * HD + c0);
+        for (int rr = 0; rr < 2; ++rr) {
+          if ((lane >> 4) == rr) {
+            float4* w4 = reinterpret_cast<float4*>(rows_buf + (lane & 15) * 36);
 #pragma unroll
-            for (int c = 0; c < 32; c += 4) dst[c / 4] = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
+            for (int c = 0; c < 8; ++c) w4[c] = make_float4(o[4 * c], o[4 * c + 1], o[4 * c + 2], o[4 * c + 3]);
           }
+          __syncwarp();
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const int lr = (lane >> 3) + 4 * m;
+            const int row = 32 * (warp & 3) + 16 * rr + lr;  // row of the segment tile
+            const float4 x = *reinterpret_cast<const float4*>(rows_buf + lr * 36 + (lane & 7) * 4);
+            const int col = g * HD + c0 + (lane & 7) * 4;
+            if (row < nrows) {
+              if (sole) {  // out is only 8-byte aligned: 4 columns per store
+                uint2 v;
+                v.x = ptx::pack_bf16x2(x.x, x.y);
+                v.y = ptx::pack_bf16x2(x.z, x.w);
+                *reinterpret_cast<uint2*>(p.out + (row0 + row) * D + col) = v;
+              } else {
+                *reinterpret_cast<float4*>(p.part_o + (slot * hps + row) * D + col) = x;
+              }
+            }
+          }
+          __syncwarp();
         }
       }
       if (!sole && g == 0 && r < nrows)
@@ -717,98 +826,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
       ptx::tc_fence_before();
       ptx::mbar_arrive(ofree_bar);  // O may be overwritten by the next piece
       if (sole) continue;
-      // Cross-CTA step: the last CTA to finish its piece of the segment merges them all.
-      __threadfence();
-      if (!wg_sync()) {
+      if (!cross_cta(pe_b, pe_seg, pe_base, pe_nblk)) {
         abort_all(kErrTimeout);
         failed = true;
         break;
       }
-      const int64_t segid = static_cast<int64_t>(pe_b) * segs + pe_seg;
-      if (t == 0) s_prev = atomicAdd(p.counters + segid, 1);
-      if (!wg_sync()) {
-        abort_all(kErrTimeout);
-        failed = true;
-        break;
-      }
-      const int prev = s_prev;
-      const int64_t wf = tc_worker_of(pe_base, T, W);
-      const int64_t wl = tc_worker_of(pe_base + pe_nblk - 1, T, W);
-      if (prev != static_cast<int>(wl - wf)) continue;
-      __threadfence();
-      {
-        // Piece k of the segment belongs to worker wf + k.  For k > 0 that worker's range
-        // starts inside the segment, so the piece is its first (slot 0); worker wf's piece
-        // is its first only if its range starts exactly at the segment start.
-        const int np = static_cast<int>(wl - wf + 1);
-        const int64_t slot0 = wf * 2 + (pe_base <= tc_wstart(wf, T, W) ? 0 : 1);
-        auto slot_of = [&](int k) -> int64_t { return k == 0 ? slot0 : (wf + k) * 2; };
-        // Lanes across columns (coalesced rows): warp q merges rows q*4 .. q*4+3, then
-        // the next 32 rows; 4 rows x 4 pieces of (max, sum) and values per round trip.
-        constexpr int CW = D / 32;  // columns per lane
-        const int q = t >> 5, ln = t & 31;
-        for (int h0 = q * 4; h0 < nrows; h0 += 32) {
-          float M[4], L[4], acc[4][CW];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            M[j] = -INFINITY;
-            L[j] = 0.f;
-#pragma unroll
-            for (int c = 0; c < CW; ++c) acc[j][c] = 0.f;
-          }
-          for (int k0 = 0; k0 < np; k0 += 4) {
-            float2 ml[4][4];
-            float v[4][4][CW];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const int64_t sl = slot_of(k0 + k < np ? k0 + k : 0);
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const bool act = k0 + k < np && h0 + j < nrows;
-                const int64_t e = sl * hps + min(h0 + j, nrows - 1);
-                ml[k][j] = act ? __ldcg(reinterpret_cast<const float2*>(p.part_ml + e * 2))
-                               : make_float2(-INFINITY, 0.f);
-                if constexpr (CW == 4) {
-                  const float4 x = act ? __ldcg(reinterpret_cast<const float4*>(p.part_o + e * D) + ln)
-                                       : make_float4(0.f, 0.f, 0.f, 0.f);
-                  v[k][j][0] = x.x; v[k][j][1] = x.y; v[k][j][2] = x.z; v[k][j][3] = x.w;
-                } else {
-                  const float2 x = act ? __ldcg(reinterpret_cast<const float2*>(p.part_o + e * D) + ln)
-                                       : make_float2(0.f, 0.f);
-                  v[k][j][0] = x.x; v[k][j][1] = x.y;
-                }
-              }
-            }
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const float mn = fmaxf(M[j], ml[k][j].x);
-                const float mu = (mn == -INFINITY) ? 0.f : mn;
-                const float a = ptx::ex2(M[j] - mu), bw = ptx::ex2(ml[k][j].x - mu);
-                L[j] = L[j] * a + ml[k][j].y * bw;
-#pragma unroll
-                for (int c = 0; c < CW; ++c) acc[j][c] = acc[j][c] * a + v[k][j][c] * bw;
-                M[j] = mn;
-              }
-          }
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            if (h0 + j >= nrows) continue;
-            const float iv = L[j] > 0.f ? 1.f / L[j] : 0.f;
-            uint16_t* dst = p.out + (row0 + h0 + j) * D + ln * CW;
-            if constexpr (CW == 4) {
-              uint2 o;
-              o.x = ptx::pack_bf16x2(acc[j][0] * iv, acc[j][1] * iv);
-              o.y = ptx::pack_bf16x2(acc[j][2] * iv, acc[j][3] * iv);
-              *reinterpret_cast<uint2*>(dst) = o;
-            } else {
-              *reinterpret_cast<uint32_t*>(dst) = ptx::pack_bf16x2(acc[j][0] * iv, acc[j][1] * iv);
-            }
-          }
-        }
-      }
-      if (t == 0) p.counters[segid] = 0;
     }
   }
 
@@ -825,7 +847,8 @@ template <int D>
 constexpr size_t tc_smem_bytes() {
   using GE = TcGeo<D>;
   return 1024 + static_cast<size_t>(GE::kStages) * GE::kStage + GE::kQTile +
-         GE::kStages * sizeof(TcStageInfo) + 16 * GE::kStages + 24 * kTcBufs + 64;
+         GE::kStages * sizeof(TcStageInfo) + 16 * GE::kStages + 24 * kTcBufs + 64 + 128 +
+         kTcSoftThreads / 32 * kStgFloats * sizeof(float);
 }
 
 template <int D>
