@@ -129,7 +129,9 @@ gqa_status gqa_paged_decode_attn(const void* q, const void* k_pages, const void*
  * overlaps the append (programmatic dependent launch): its prologue and block-table
  * reads run while the append finishes, and its first K/V copy waits for it.  This is
  * the step tiny-llm's "优化" page describes (append position, then attention over the
- * block table) as one call.
+ * block table) as one call.  Calls never synchronise or read device data on the host, so
+ * after a first call on the device (which sets up the workspace) the step can be captured
+ * in a CUDA graph and replayed with new contents of the same buffers.
  */
 gqa_status gqa_decode_step(const void* q, const void* k_new, const void* v_new, void* k_pages,
                            void* v_pages, const int32_t* block_table, const int32_t* positions,

@@ -259,6 +259,118 @@ def test_consecutive_steps_rewrite_what_the_previous_decode_read(cuda_device):
         assert_close(gpu_f64(outs[step]), oracle_out(dict(h, k=k2, v=v2)), what=f"step {step}")
 
 
+def _append_then_attend_reference(inp, positions, kn, vn):
+    h = host_arrays(inp)
+    k2, v2 = oracle.kv_append(h["k"], h["v"], bf16_bits(kn), bf16_bits(vn), h["bt"], positions.numpy())
+    return k2, v2, oracle_out(dict(h, k=k2, v=v2))
+
+
+@pytest.mark.parametrize("heads", [(16, 4), (96, 1), (200, 1)], ids=["gqa", "mqa", "two_head_tiles"])
+def test_decode_step_positions_outside_attended_range(cuda_device, heads):
+    """A row appended beyond seq_lens[b] is written to the pool but not attended; one at
+    seq_lens[b] - 1 is attended (the one-launch step writes both kinds)."""
+    H, Hk = heads
+    # No slot is reserved for the append here (append=False), so attended slots all hold data.
+    inp = make_custom_inputs([300, 70, 129], H, Hk, 64, 16, seed=33, extra_pages=6)
+    g = torch.Generator().manual_seed(33)
+    kn = torch.randn((3, Hk, 64), generator=g).to(torch.bfloat16)
+    vn = torch.randn((3, Hk, 64), generator=g).to(torch.bfloat16)
+    # 303 and 140 lie past the attended lengths but inside each sequence's last page
+    positions = torch.tensor([303, 69, 140], dtype=torch.int32)
+    d = inp.to(cuda_device)
+    out = gq.decode_step(d.q, kn.to(cuda_device), vn.to(cuda_device), d.k_pages, d.v_pages, d.block_table,
+                         positions.to(cuda_device), d.seq_lens, scale=d.scale)
+    gq.check_device_error()
+    k2, v2, want = _append_then_attend_reference(inp, positions, kn, vn)
+    assert np.array_equal(bf16_bits(d.k_pages), k2)
+    assert np.array_equal(bf16_bits(d.v_pages), v2)
+    assert_close(gpu_f64(out), want, what=str(heads))
+
+
+@pytest.mark.parametrize("workers", [1, 3, 57, 400])
+@pytest.mark.parametrize("heads", [(16, 2), (200, 1)], ids=["gqa", "two_head_tiles"])
+def test_decode_step_under_forced_splits(cuda_device, heads, workers):
+    """The block holding the appended row may sit anywhere in a CTA's range (first, last,
+    alone); with two head tiles two CTAs write the same row before reading it."""
+    H, Hk = heads
+    inp = make_custom_inputs([1100, 513, 64, 1], H, Hk, 128, 16, seed=34 + workers, append=True)
+    d = inp.to(cuda_device)
+    gq.set_num_workers(workers)
+    try:
+        out = gq.decode_step(d.q, d.k_new, d.v_new, d.k_pages, d.v_pages, d.block_table, d.positions,
+                             d.seq_lens, scale=d.scale)
+        gq.check_device_error()
+    finally:
+        gq.set_num_workers(0)
+    k2, v2, want = _append_then_attend_reference(inp, inp.positions, inp.k_new, inp.v_new)
+    assert np.array_equal(bf16_bits(d.k_pages), k2)
+    assert_close(gpu_f64(out), want, what=f"workers={workers}")
+
+
+def test_decode_step_bad_position_skips_row_and_reports(cuda_device):
+    inp = make_custom_inputs([200, 40], 8, 2, 128, 16, seed=35, append=True, max_blocks_per_seq=16)
+    positions = inp.positions.clone()
+    positions[1] = 16 * 16 + 3  # beyond max_blocks_per_seq * page_size
+    d = inp.to(cuda_device)
+    gq.decode_step(d.q, d.k_new, d.v_new, d.k_pages, d.v_pages, d.block_table, positions.to(cuda_device),
+                   d.seq_lens, scale=d.scale)
+    with pytest.raises(gq.GQAError) as ei:
+        gq.check_device_error()
+    assert ei.value.status == -4
+    # only sequence 0's row is appended; every other byte of the pools is unchanged
+    h = host_arrays(inp)
+    k2, v2 = oracle.kv_append(h["k"], h["v"], bf16_bits(inp.k_new[:1]), bf16_bits(inp.v_new[:1]), h["bt"][:1],
+                              positions[:1].numpy())
+    assert np.array_equal(bf16_bits(d.k_pages), k2)
+    assert np.array_equal(bf16_bits(d.v_pages), v2)
+
+
+def test_decode_step_replays_in_a_cuda_graph(cuda_device):
+    """After a first call, the step is captured once and replayed with new buffer contents
+    (new rows, positions and lengths advanced by one each step)."""
+    B, H, Hk, D, ps = 3, 32, 8, 128, 16
+    # lengths leave room in each sequence's last page for three more appended tokens
+    inp = make_custom_inputs([200, 27, 70], H, Hk, D, ps, seed=36, append=True, extra_pages=8,
+                             max_blocks_per_seq=24)
+    d = inp.to(cuda_device)
+    out = torch.empty((B, H, D), dtype=torch.bfloat16, device=cuda_device)
+    kn = d.k_new.clone()
+    vn = d.v_new.clone()
+    pos = d.positions.clone()
+    lens = d.seq_lens.clone()
+    s = torch.cuda.Stream(cuda_device)
+    with torch.cuda.stream(s):
+        gq.decode_step(d.q, kn, vn, d.k_pages, d.v_pages, d.block_table, pos, lens, out=out, scale=d.scale)
+    s.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        gq.decode_step(d.q, kn, vn, d.k_pages, d.v_pages, d.block_table, pos, lens, out=out, scale=d.scale)
+    g = torch.Generator().manual_seed(7)
+    h = host_arrays(inp)
+    h["k"], h["v"] = oracle.kv_append(h["k"], h["v"], bf16_bits(inp.k_new), bf16_bits(inp.v_new), h["bt"],
+                                     inp.positions.numpy())
+    assert_close(gpu_f64(out), oracle_out(h), what="first call")
+    hpos = inp.positions.clone()
+    hlens = inp.seq_lens.clone()
+    for step in range(3):
+        hpos += 1
+        hlens += 1
+        new_k = torch.randn((B, Hk, D), generator=g).to(torch.bfloat16)
+        new_v = torch.randn((B, Hk, D), generator=g).to(torch.bfloat16)
+        kn.copy_(new_k)
+        vn.copy_(new_v)
+        pos.copy_(hpos)
+        lens.copy_(hlens)
+        graph.replay()
+        torch.cuda.synchronize()
+        gq.check_device_error()
+        h["k"], h["v"] = oracle.kv_append(h["k"], h["v"], bf16_bits(new_k), bf16_bits(new_v), h["bt"],
+                                         hpos.numpy())
+        h["sl"] = hlens.numpy()
+        assert_close(gpu_f64(out), oracle_out(h), what=f"replay {step}")
+    del graph
+
+
 # ------------------------------------------------------------------ large groups (tcgen05 path)
 
 TC_CASES = [
