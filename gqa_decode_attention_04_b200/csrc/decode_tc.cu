@@ -26,7 +26,12 @@
 //     domain over its half with its own O accumulator (rescaled in TMEM only when its
 //     reference rises by more than 8), writing P (bf16) over its half of S.  At a piece
 //     end the two (max, sum, O) are combined; the result is normalised and written out,
-//     or stored for the cross-CTA log-sum-exp merge (the last CTA to finish merges).
+//     or, for a segment cut between CTAs, stored as a partial (O, max, sum).
+//   * Split merge (a second kernel, launched with programmatic dependent launch so it is
+//     resident when the decode drains): one block per cut segment and 32 rows merges the
+//     partials by log-sum-exp weights.  Merging inside the decode (the last CTA of a
+//     segment to finish merges it) put the merge's dependent loads behind the other CTAs'
+//     K/V streams at the very end of every CTA's range.
 //   * Safety: every wait is bounded; on a timeout all warps leave their loops, the MMA
 //     warps wait for their issued MMAs, and TMEM is released before exit.
 #include "internal.cuh"
@@ -67,9 +72,8 @@ struct TcGeo {
 };
 
 struct TcStageInfo {
-  int64_t seg_base;
   uint64_t vmask;  // bit t: token t of the block is inside the sequence and its page was loaded
-  int b, seg, blk, nblk, nvalid, flags, piece, pad;
+  int b, seg, blk, nvalid, flags, piece;
 };
 enum : int { kTcFirst = 1, kTcLast = 2, kTcSole = 4, kTcFirstPieceOfCta = 8 };
 
@@ -96,7 +100,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
   __shared__ int s_start_b;
   __shared__ int64_t s_start_base;
   __shared__ uint32_t s_tmem;
-  __shared__ int s_prev;
   __shared__ int s_abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -105,6 +108,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
   const int cap = p.max_blocks * p.page_size;
   const int hps = p.heads_per_seg;
 
+  // The split merge (the next kernel) may launch now; it waits for this grid to complete
+  // before reading anything this grid writes.
+  ptx::pdl_launch_dependents();
   // ---------------------------------------------------------------- prologue (split)
   int64_t mine = 0;
   for (int b = threadIdx.x; b < B; b += blockDim.x) {
@@ -295,7 +301,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
       return (lane < nchunks && cu.blk * kTcBlk + cl * R < cu.len) ? pg : -1;
     };
     start_piece();
-    int64_t seg_base = x0 - cu.blk;
     int piece = 0;
     bool first_piece = true;
     int piece_blk0 = cu.blk;
@@ -348,12 +353,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
           if ((okbits >> c) & 1u) vmask |= chunk_mask << (c * R);
         if (nvalid < kTcBlk) vmask &= (1ull << nvalid) - 1ull;
         TcStageInfo& si = info[stage];
-        si.seg_base = seg_base;
         si.vmask = vmask;
         si.b = cu.b;
         si.seg = cu.seg;
         si.blk = cu.blk;
-        si.nblk = cu.nblk;
         si.nvalid = nvalid;
         si.piece = piece;
         si.flags = (first ? kTcFirst : 0) | (last ? kTcLast : 0) |
@@ -397,7 +400,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
               next_len = (cu.b + 1 < B) ? __ldg(p.seq_lens + cu.b + 1) : 0;
             } while (cu.nblk == 0 && cu.b + 1 < B);
           }
-          seg_base = x0 + i + 1;
           start_piece();
         }
         page = page_of();
@@ -533,97 +535,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
       ++wg_phase;
       return __all_sync(0xffffffffu, ok);
     };
-    // Cross-CTA step of a piece that is not the whole segment (its partial is stored):
-    // count the arrival; the last CTA to finish a piece of the segment merges them all.
-    auto cross_cta = [&](int cb, int cseg, int64_t pe_base, int pe_nblk) -> bool {
-      __threadfence();
-      if (!wg_sync()) return false;
-      const int64_t segid = static_cast<int64_t>(cb) * segs + cseg;
-      if (t == 0) s_prev = atomicAdd(p.counters + segid, 1);
-      if (!wg_sync()) return false;
-      const int prev = s_prev;
-      const int64_t wf = tc_worker_of(pe_base, T, W);
-      const int64_t wl = tc_worker_of(pe_base + pe_nblk - 1, T, W);
-      if (prev != static_cast<int>(wl - wf)) return true;
-      __threadfence();
-      const int kvh = cseg / p.n_ht, ht = cseg % p.n_ht;
-      const int nrows = min(hps, p.group - ht * hps);
-      const int64_t row0 = static_cast<int64_t>(cb) * p.num_heads + kvh * p.group + ht * hps;
-        {
-          // Piece k of the segment belongs to worker wf + k.  For k > 0 that worker's range
-          // starts inside the segment, so the piece is its first (slot 0); worker wf's piece
-          // is its first only if its range starts exactly at the segment start.
-          const int np = static_cast<int>(wl - wf + 1);
-          const int64_t slot0 = wf * 2 + (pe_base <= tc_wstart(wf, T, W) ? 0 : 1);
-          auto slot_of = [&](int k) -> int64_t { return k == 0 ? slot0 : (wf + k) * 2; };
-          // Lanes across columns (coalesced rows): warp q merges rows q*4 .. q*4+3, then
-          // the next 32 rows; 4 rows x 4 pieces of (max, sum) and values per round trip.
-          constexpr int CW = D / 32;  // columns per lane
-          const int q = t >> 5, ln = t & 31;
-          for (int h0 = q * 4; h0 < nrows; h0 += 32) {
-            float M[4], L[4], acc[4][CW];
-  #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              M[j] = -INFINITY;
-              L[j] = 0.f;
-  #pragma unroll
-              for (int c = 0; c < CW; ++c) acc[j][c] = 0.f;
-            }
-            for (int k0 = 0; k0 < np; k0 += 4) {
-              float2 ml[4][4];
-              float v[4][4][CW];
-  #pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                const int64_t sl = slot_of(k0 + k < np ? k0 + k : 0);
-  #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                  const bool act = k0 + k < np && h0 + j < nrows;
-                  const int64_t e = sl * hps + min(h0 + j, nrows - 1);
-                  ml[k][j] = act ? __ldcg(reinterpret_cast<const float2*>(p.part_ml + e * 2))
-                                 : make_float2(-INFINITY, 0.f);
-                  if constexpr (CW == 4) {
-                    const float4 x = act ? __ldcg(reinterpret_cast<const float4*>(p.part_o + e * D) + ln)
-                                         : make_float4(0.f, 0.f, 0.f, 0.f);
-                    v[k][j][0] = x.x; v[k][j][1] = x.y; v[k][j][2] = x.z; v[k][j][3] = x.w;
-                  } else {
-                    const float2 x = act ? __ldcg(reinterpret_cast<const float2*>(p.part_o + e * D) + ln)
-                                         : make_float2(0.f, 0.f);
-                    v[k][j][0] = x.x; v[k][j][1] = x.y;
-                  }
-                }
-              }
-  #pragma unroll
-              for (int k = 0; k < 4; ++k)
-  #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                  const float mn = fmaxf(M[j], ml[k][j].x);
-                  const float mu = (mn == -INFINITY) ? 0.f : mn;
-                  const float a = ptx::ex2(M[j] - mu), bw = ptx::ex2(ml[k][j].x - mu);
-                  L[j] = L[j] * a + ml[k][j].y * bw;
-  #pragma unroll
-                  for (int c = 0; c < CW; ++c) acc[j][c] = acc[j][c] * a + v[k][j][c] * bw;
-                  M[j] = mn;
-                }
-            }
-  #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              if (h0 + j >= nrows) continue;
-              const float iv = L[j] > 0.f ? 1.f / L[j] : 0.f;
-              uint16_t* dst = p.out + (row0 + h0 + j) * D + ln * CW;
-              if constexpr (CW == 4) {
-                uint2 o;
-                o.x = ptx::pack_bf16x2(acc[j][0] * iv, acc[j][1] * iv);
-                o.y = ptx::pack_bf16x2(acc[j][2] * iv, acc[j][3] * iv);
-                *reinterpret_cast<uint2*>(dst) = o;
-              } else {
-                *reinterpret_cast<uint32_t*>(dst) = ptx::pack_bf16x2(acc[j][0] * iv, acc[j][1] * iv);
-              }
-            }
-          }
-        }
-      if (t == 0) p.counters[segid] = 0;
-      return true;
-    };
     int is = 0;  // stage of block i (i % S, kept incrementally)
     for (int64_t i = 0; i < total && !failed; ++i) {
       // Another warp's failed wait ends the CTA; checked every 8 blocks (each wait here is
@@ -643,13 +554,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
       const uint64_t vmask = info[stg].vmask;
       // What a piece end needs of this block, read while its stage is held (the stage is
       // refilled once the block's P V completes, which needs this thread's P).
-      int pe_b = 0, pe_seg = 0, pe_nblk = 0;
-      int64_t pe_base = 0;
+      int pe_b = 0, pe_seg = 0;
       if (flags & kTcLast) {
         pe_b = info[stg].b;
         pe_seg = info[stg].seg;
-        pe_nblk = info[stg].nblk;
-        pe_base = info[stg].seg_base;
       }
       const bool first = flags & kTcFirst;
       if (first) {
@@ -673,21 +581,28 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
       // Row maximum of this half's scaled scores (log2 domain), a tree over raw scores.
       float mx;
       {
-        float tt[16];
+        // 32 -> 11 -> 4 -> 1 with three-input max (min for a negative scale).
+        float tt[11];
         if (pos) {
 #pragma unroll
-          for (int c = 0; c < 16; ++c) tt[c] = fmaxf(__uint_as_float(u[c]), __uint_as_float(u[c + 16]));
-#pragma unroll
-          for (int w2 = 8; w2 > 0; w2 >>= 1)
-#pragma unroll
-            for (int c = 0; c < w2; ++c) tt[c] = fmaxf(tt[c], tt[c + w2]);
+          for (int c = 0; c < 10; ++c)
+            tt[c] = ptx::max3(__uint_as_float(u[3 * c]), __uint_as_float(u[3 * c + 1]), __uint_as_float(u[3 * c + 2]));
+          tt[10] = fmaxf(__uint_as_float(u[30]), __uint_as_float(u[31]));
+          tt[0] = ptx::max3(tt[0], tt[1], tt[2]);
+          tt[3] = ptx::max3(tt[3], tt[4], tt[5]);
+          tt[6] = ptx::max3(tt[6], tt[7], tt[8]);
+          tt[9] = fmaxf(tt[9], tt[10]);
+          tt[0] = fmaxf(ptx::max3(tt[0], tt[3], tt[6]), tt[9]);
         } else {
 #pragma unroll
-          for (int c = 0; c < 16; ++c) tt[c] = fminf(__uint_as_float(u[c]), __uint_as_float(u[c + 16]));
-#pragma unroll
-          for (int w2 = 8; w2 > 0; w2 >>= 1)
-#pragma unroll
-            for (int c = 0; c < w2; ++c) tt[c] = fminf(tt[c], tt[c + w2]);
+          for (int c = 0; c < 10; ++c)
+            tt[c] = ptx::min3(__uint_as_float(u[3 * c]), __uint_as_float(u[3 * c + 1]), __uint_as_float(u[3 * c + 2]));
+          tt[10] = fminf(__uint_as_float(u[30]), __uint_as_float(u[31]));
+          tt[0] = ptx::min3(tt[0], tt[1], tt[2]);
+          tt[3] = ptx::min3(tt[3], tt[4], tt[5]);
+          tt[6] = ptx::min3(tt[6], tt[7], tt[8]);
+          tt[9] = fminf(tt[9], tt[10]);
+          tt[0] = fminf(ptx::min3(tt[0], tt[3], tt[6]), tt[9]);
         }
         mx = tt[0] * sl2;
         if (mx != mx) mx = -INFINITY;  // every token masked and a zero scale
@@ -720,15 +635,21 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
           mref = mx;
         }
       }
-      // P = 2^(score * scale_log2 - reference), one FFMA and one ex2 per score; bf16
+      // P = 2^(score * scale_log2 - reference), one ex2 per score (the arguments and the
+      // row sum in packed fp32 pairs, two scores per instruction); bf16
       // pairs overwrite the first 16 of this half's own 32 score columns (token 32 g + 2j,
       // 32 g + 2j + 1 in column 32 g + j), so neither warpgroup touches the other's scores.
       const float nmu = (mref == -INFINITY) ? 0.f : -mref;
       // Three passes (arguments, exponentials, sums and packing) so the 32 ex2 issue back
       // to back on the MUFU.
       float e[32];
+      {
+        const uint64_t s2 = ptx::f2_pack(sl2, sl2), n2 = ptx::f2_pack(nmu, nmu);
 #pragma unroll
-      for (int c = 0; c < 32; ++c) e[c] = fmaf(__uint_as_float(u[c]), sl2, nmu);
+        for (int c = 0; c < 32; c += 2)
+          ptx::f2_unpack(ptx::f2_fma(ptx::f2_pack(__uint_as_float(u[c]), __uint_as_float(u[c + 1])), s2, n2),
+                         e[c], e[c + 1]);
+      }
 #pragma unroll
       for (int c = 0; c < 32; ++c) e[c] = ptx::ex2(e[c]);
       if (!full) {  // masked scores are exactly 0 (with a zero scale, inf * 0 is NaN)
@@ -736,17 +657,19 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
         for (int c = 0; c < 32; ++c) e[c] = ((vm >> c) & 1u) ? e[c] : 0.f;
       }
       uint32_t pk[16];
-      float ls0 = 0.f, ls1 = 0.f, ls2 = 0.f, ls3 = 0.f;
+      {
+        uint64_t a0 = ptx::f2_pack(e[0], e[1]), a1 = ptx::f2_pack(e[2], e[3]);
 #pragma unroll
-      for (int c = 0; c < 32; c += 4) {
-        ls0 += e[c];
-        ls1 += e[c + 1];
-        ls2 += e[c + 2];
-        ls3 += e[c + 3];
-        pk[c / 2] = ptx::pack_bf16x2(e[c], e[c + 1]);
-        pk[c / 2 + 1] = ptx::pack_bf16x2(e[c + 2], e[c + 3]);
+        for (int c = 4; c < 32; c += 4) {
+          a0 = ptx::f2_add(a0, ptx::f2_pack(e[c], e[c + 1]));
+          a1 = ptx::f2_add(a1, ptx::f2_pack(e[c + 2], e[c + 3]));
+        }
+        float s0, s1;
+        ptx::f2_unpack(ptx::f2_add(a0, a1), s0, s1);
+        lsum += s0 + s1;
       }
-      lsum += (ls0 + ls1) + (ls2 + ls3);
+#pragma unroll
+      for (int c = 0; c < 32; c += 2) pk[c / 2] = ptx::pack_bf16x2(e[c], e[c + 1]);
       ptx::tmem_st16(st + 32 * g, pk);
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
@@ -825,12 +748,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
         *reinterpret_cast<float2*>(p.part_ml + (slot * hps + r) * 2) = make_float2(Mx, ltot);
       ptx::tc_fence_before();
       ptx::mbar_arrive(ofree_bar);  // O may be overwritten by the next piece
-      if (sole) continue;
-      if (!cross_cta(pe_b, pe_seg, pe_base, pe_nblk)) {
-        abort_all(kErrTimeout);
-        failed = true;
-        break;
-      }
     }
   }
 
@@ -839,6 +756,151 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
   __syncthreads();
   ptx::tc_fence_after();
   if (warp == kWarpS) ptx::tmem_dealloc(tmem, kTmemCols);
+}
+
+// ------------------------------------------------------------------ split merge
+// Second kernel of a tcgen05 decode.  Block (w - 1, y) merges the segment that worker w's
+// range starts inside, when w is the first worker starting inside it (every cut segment
+// has exactly one such worker), rows 32 y .. 32 y + 31 of its head tile: out = sum_j
+// O_j 2^(m_j - M) / sum_j l_j 2^(m_j - M) over the segment's pieces j (partials in worker
+// order; M the largest m_j).
+constexpr int kMergeThreads = 256;
+constexpr int kMergeRows = 32;  // rows per block: 4 per warp
+
+template <int D>
+__global__ void __launch_bounds__(kMergeThreads) merge_tc_kernel(const DecodeParams p) {
+  __shared__ int64_t s_part[kMergeThreads / 32];
+  __shared__ int s_b;
+  __shared__ int64_t s_base;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int B = p.num_seqs;
+  const int segs = p.num_kv_heads * p.n_ht;
+  const int cap = p.max_blocks * p.page_size;
+  const int hps = p.heads_per_seg;
+
+  // The work list as the decode split it (seq_lens is not written by the decode).
+  int64_t mine = 0;
+  for (int b = threadIdx.x; b < B; b += blockDim.x)
+    mine += static_cast<int64_t>((tc_eff_len(__ldg(p.seq_lens + b), cap) + kTcBlk - 1) / kTcBlk) * segs;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, off);
+  if (lane == 0) s_part[warp] = mine;
+  if (threadIdx.x == 0) s_b = -1;
+  __syncthreads();
+  int64_t T = 0;
+  for (int i = 0; i < kMergeThreads / 32; ++i) T += s_part[i];
+  const int64_t W = min(static_cast<int64_t>(p.num_workers), T);
+  const int64_t w = static_cast<int64_t>(blockIdx.x) + 1;
+  if (w >= W) return;
+  const int64_t x = tc_wstart(w, T, W);
+  __syncthreads();
+  {
+    int64_t base = 0;
+    for (int t0 = 0; t0 < B && base <= x; t0 += blockDim.x) {
+      const int b = t0 + threadIdx.x;
+      int64_t n = 0;
+      if (b < B) n = static_cast<int64_t>((tc_eff_len(__ldg(p.seq_lens + b), cap) + kTcBlk - 1) / kTcBlk) * segs;
+      int64_t incl = n;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int64_t v = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += v;
+      }
+      if (lane == 31) s_part[warp] = incl;
+      __syncthreads();
+      int64_t pre = 0, tot = 0;
+      for (int i = 0; i < kMergeThreads / 32; ++i) {
+        if (i < warp) pre += s_part[i];
+        tot += s_part[i];
+      }
+      incl += pre;
+      if (n > 0 && x >= base + incl - n && x < base + incl) {
+        s_b = b;
+        s_base = base + incl - n;
+      }
+      base += tot;
+      __syncthreads();
+    }
+  }
+  const int b = s_b;
+  if (b < 0) return;
+  const int nblk = (tc_eff_len(__ldg(p.seq_lens + b), cap) + kTcBlk - 1) / kTcBlk;
+  const int seg = static_cast<int>((x - s_base) / nblk);
+  const int64_t seg_base = s_base + static_cast<int64_t>(seg) * nblk;
+  if (seg_base == x) return;  // worker w starts at a segment start: nothing is cut there
+  const int64_t wf = tc_worker_of(seg_base, T, W);
+  if (wf + 1 != w) return;    // a worker before w also starts inside this segment
+  const int64_t wl = tc_worker_of(seg_base + nblk - 1, T, W);
+  const int np = static_cast<int>(wl - wf + 1);
+  // Piece j belongs to worker wf + j: for j > 0 it is that worker's first piece (slot 0);
+  // worker wf's piece is its first only if its range starts at the segment start.
+  const int64_t slot0 = wf * 2 + (seg_base == tc_wstart(wf, T, W) ? 0 : 1);
+  auto slot_of = [&](int j) -> int64_t { return j == 0 ? slot0 : (wf + j) * 2; };
+  const int kvh = seg / p.n_ht, ht = seg % p.n_ht;
+  const int nrows = min(hps, p.group - ht * hps);
+  const int64_t row0 = static_cast<int64_t>(b) * p.num_heads + kvh * p.group + ht * hps;
+  const int h0 = blockIdx.y * kMergeRows + warp * 4;
+  if (h0 >= nrows) return;
+
+  ptx::pdl_wait_prerequisites();  // the partials are the decode's
+  constexpr int CW = D / 32;  // columns per lane
+  float M[4], L[4], acc[4][CW];
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    M[r] = -INFINITY;
+    L[r] = 0.f;
+#pragma unroll
+    for (int c = 0; c < CW; ++c) acc[r][c] = 0.f;
+  }
+  for (int k0 = 0; k0 < np; k0 += 4) {
+    float2 ml[4][4];
+    float v[4][4][CW];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int64_t sl = slot_of(k0 + k < np ? k0 + k : 0);
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const bool act = k0 + k < np && h0 + r < nrows;
+        const int64_t e = sl * hps + min(h0 + r, nrows - 1);
+        ml[k][r] = act ? __ldcg(reinterpret_cast<const float2*>(p.part_ml + e * 2)) : make_float2(-INFINITY, 0.f);
+        if constexpr (CW == 4) {
+          const float4 t = act ? __ldcg(reinterpret_cast<const float4*>(p.part_o + e * D) + lane)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+          v[k][r][0] = t.x; v[k][r][1] = t.y; v[k][r][2] = t.z; v[k][r][3] = t.w;
+        } else {
+          const float2 t = act ? __ldcg(reinterpret_cast<const float2*>(p.part_o + e * D) + lane)
+                               : make_float2(0.f, 0.f);
+          v[k][r][0] = t.x; v[k][r][1] = t.y;
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const float mn = fmaxf(M[r], ml[k][r].x);
+        const float mu = (mn == -INFINITY) ? 0.f : mn;
+        const float a = ptx::ex2(M[r] - mu), bw = ptx::ex2(ml[k][r].x - mu);
+        L[r] = L[r] * a + ml[k][r].y * bw;
+#pragma unroll
+        for (int c = 0; c < CW; ++c) acc[r][c] = acc[r][c] * a + v[k][r][c] * bw;
+        M[r] = mn;
+      }
+  }
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    if (h0 + r >= nrows) continue;
+    const float iv = L[r] > 0.f ? 1.f / L[r] : 0.f;
+    uint16_t* dst = p.out + (row0 + h0 + r) * D + lane * CW;
+    if constexpr (CW == 4) {
+      uint2 o;
+      o.x = ptx::pack_bf16x2(acc[r][0] * iv, acc[r][1] * iv);
+      o.y = ptx::pack_bf16x2(acc[r][2] * iv, acc[r][3] * iv);
+      *reinterpret_cast<uint2*>(dst) = o;
+    } else {
+      *reinterpret_cast<uint32_t*>(dst) = ptx::pack_bf16x2(acc[r][0] * iv, acc[r][1] * iv);
+    }
+  }
 }
 
 // ------------------------------------------------------------------ host side
@@ -874,7 +936,17 @@ cudaError_t launch_tc_t(const DecodeParams& p, const CUtensorMap& tk, const CUte
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = overlap ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kern, tk, tv, tq, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tk, tv, tq, p);
+  if (e != cudaSuccess || grid < 2) return e;
+  // The split merge: one block column per worker boundary, launched so that it can be
+  // resident while the decode drains (it waits for the decode's completion itself).
+  cudaLaunchConfig_t mc = {};
+  mc.gridDim = dim3(grid - 1, (p.heads_per_seg + kMergeRows - 1) / kMergeRows);
+  mc.blockDim = dim3(kMergeThreads);
+  mc.stream = stream;
+  mc.attrs = attr;
+  mc.numAttrs = 1;
+  return cudaLaunchKernelEx(&mc, merge_tc_kernel<D>, p);
 }
 }  // namespace
 

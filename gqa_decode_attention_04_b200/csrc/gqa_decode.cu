@@ -324,7 +324,7 @@ gqa_status decode_impl(const void* q, const void* k_pages, const void* v_pages,
                                    overlap_previous, &s);
   if (s != GQA_OK) return s;
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
-  g_launches.fetch_add(1);
+  g_launches.fetch_add(plan.tensor_cores && grid > 1 ? 2 : 1);
   return GQA_OK;
 }
 
@@ -525,7 +525,7 @@ gqa_status gqa_paged_decode_attn_noalloc(const void* q, const void* k_pages, con
                        false, &s);
   if (s != GQA_OK) return s;
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
-  g_launches.fetch_add(1);
+  g_launches.fetch_add(plan.tensor_cores && workers > 1 ? 2 : 1);
   return GQA_OK;
 }
 
