@@ -34,6 +34,8 @@
 //     K/V streams at the very end of every CTA's range.
 //   * Safety: every wait is bounded; on a timeout all warps leave their loops, the MMA
 //     warps wait for their issued MMAs, and TMEM is released before exit.
+#include <type_traits>
+
 #include "internal.cuh"
 #include "ptx.cuh"
 
@@ -761,14 +763,15 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
 // ------------------------------------------------------------------ split merge
 // Second kernel of a tcgen05 decode.  Block (w - 1, y) merges the segment that worker w's
 // range starts inside, when w is the first worker starting inside it (every cut segment
-// has exactly one such worker), rows 32 y .. 32 y + 31 of its head tile: out = sum_j
+// has exactly one such worker), rows 16 y .. 16 y + 15 of its head tile: out = sum_j
 // O_j 2^(m_j - M) / sum_j l_j 2^(m_j - M) over the segment's pieces j (partials in worker
 // order; M the largest m_j).
-constexpr int kMergeThreads = 256;
-constexpr int kMergeRows = 32;  // rows per block: 4 per warp
+constexpr int kMergeThreads = 128;
+constexpr int kMergeRowsPerWarp = 4;
+constexpr int kMergeRows = kMergeThreads / 32 * kMergeRowsPerWarp;  // rows per block
 
 template <int D>
-__global__ void __launch_bounds__(kMergeThreads) merge_tc_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kMergeThreads, 6) merge_tc_kernel(const DecodeParams p) {
   __shared__ int64_t s_part[kMergeThreads / 32];
   __shared__ int s_b;
   __shared__ int64_t s_base;
@@ -839,66 +842,78 @@ __global__ void __launch_bounds__(kMergeThreads) merge_tc_kernel(const DecodePar
   const int kvh = seg / p.n_ht, ht = seg % p.n_ht;
   const int nrows = min(hps, p.group - ht * hps);
   const int64_t row0 = static_cast<int64_t>(b) * p.num_heads + kvh * p.group + ht * hps;
-  const int h0 = blockIdx.y * kMergeRows + warp * 4;
+  const int h0 = blockIdx.y * kMergeRows + warp * kMergeRowsPerWarp;
   if (h0 >= nrows) return;
 
   ptx::pdl_wait_prerequisites();  // the partials are the decode's
+  // Per row: M = max_j m_j and L = sum_j l_j 2^(m_j - M) with lanes across pieces (lane j
+  // keeps piece j's (m, l) when there are at most 32), then out = sum_j 2^(m_j - M) O_j / L
+  // with lanes across columns, the O loads of the first pieces issued with the (m, l) loads.
   constexpr int CW = D / 32;  // columns per lane
-  float M[4], L[4], acc[4][CW];
+  using VecT = typename std::conditional<CW == 4, float4, float2>::type;
+  auto o_ptr = [&](int j, int h) -> const VecT* {
+    return reinterpret_cast<const VecT*>(p.part_o + (slot_of(j) * hps + h) * D) + lane;
+  };
+  for (int r = 0; r < kMergeRowsPerWarp; ++r) {
+    const int h = h0 + r;
+    if (h >= nrows) break;
+    float2 mlj = make_float2(-INFINITY, 0.f);  // lane j: piece j's (max, sum)
+    if (lane < np) mlj = __ldcg(reinterpret_cast<const float2*>(p.part_ml + (slot_of(lane) * hps + h) * 2));
+    VecT o4[4];
 #pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    M[r] = -INFINITY;
-    L[r] = 0.f;
+    for (int j = 0; j < 4; ++j) o4[j] = j < np ? __ldcg(o_ptr(j, h)) : VecT{};
+    float M = mlj.x;
+    for (int j = lane + 32; j < np; j += 32)
+      M = fmaxf(M, __ldcg(p.part_ml + (slot_of(j) * hps + h) * 2));
 #pragma unroll
-    for (int c = 0; c < CW; ++c) acc[r][c] = 0.f;
-  }
-  for (int k0 = 0; k0 < np; k0 += 4) {
-    float2 ml[4][4];
-    float v[4][4][CW];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int64_t sl = slot_of(k0 + k < np ? k0 + k : 0);
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const bool act = k0 + k < np && h0 + r < nrows;
-        const int64_t e = sl * hps + min(h0 + r, nrows - 1);
-        ml[k][r] = act ? __ldcg(reinterpret_cast<const float2*>(p.part_ml + e * 2)) : make_float2(-INFINITY, 0.f);
-        if constexpr (CW == 4) {
-          const float4 t = act ? __ldcg(reinterpret_cast<const float4*>(p.part_o + e * D) + lane)
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
-          v[k][r][0] = t.x; v[k][r][1] = t.y; v[k][r][2] = t.z; v[k][r][3] = t.w;
-        } else {
-          const float2 t = act ? __ldcg(reinterpret_cast<const float2*>(p.part_o + e * D) + lane)
-                               : make_float2(0.f, 0.f);
-          v[k][r][0] = t.x; v[k][r][1] = t.y;
-        }
-      }
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    const float Mu = (M == -INFINITY) ? 0.f : M;
+    float Lp = mlj.y * ptx::ex2(mlj.x - Mu);
+    for (int j = lane + 32; j < np; j += 32) {
+      const float2 t = __ldcg(reinterpret_cast<const float2*>(p.part_ml + (slot_of(j) * hps + h) * 2));
+      Lp += t.y * ptx::ex2(t.x - Mu);
     }
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
+    for (int off = 16; off > 0; off >>= 1) Lp += __shfl_xor_sync(0xffffffffu, Lp, off);
+    const float iv = Lp > 0.f ? 1.f / Lp : 0.f;
+    const float wl = ptx::ex2(mlj.x - Mu) * iv;  // lane j: piece j's weight (j < 32)
+    auto weight = [&](int j) -> float {
+      if (j < 32) return __shfl_sync(0xffffffffu, wl, j);
+      return ptx::ex2(__ldcg(p.part_ml + (slot_of(j) * hps + h) * 2) - Mu) * iv;
+    };
+    float acc[CW];
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const float mn = fmaxf(M[r], ml[k][r].x);
-        const float mu = (mn == -INFINITY) ? 0.f : mn;
-        const float a = ptx::ex2(M[r] - mu), bw = ptx::ex2(ml[k][r].x - mu);
-        L[r] = L[r] * a + ml[k][r].y * bw;
-#pragma unroll
-        for (int c = 0; c < CW; ++c) acc[r][c] = acc[r][c] * a + v[k][r][c] * bw;
-        M[r] = mn;
+    for (int c = 0; c < CW; ++c) acc[c] = 0.f;
+    auto add = [&](float wj, const VecT& v) {
+      if constexpr (CW == 4) {
+        acc[0] = fmaf(wj, v.x, acc[0]); acc[1] = fmaf(wj, v.y, acc[1]);
+        acc[2] = fmaf(wj, v.z, acc[2]); acc[3] = fmaf(wj, v.w, acc[3]);
+      } else {
+        acc[0] = fmaf(wj, v.x, acc[0]); acc[1] = fmaf(wj, v.y, acc[1]);
       }
-  }
+    };
 #pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    if (h0 + r >= nrows) continue;
-    const float iv = L[r] > 0.f ? 1.f / L[r] : 0.f;
-    uint16_t* dst = p.out + (row0 + h0 + r) * D + lane * CW;
+    for (int j = 0; j < 4; ++j) {
+      const float wj = weight(j < np ? j : 0);
+      if (j < np) add(wj, o4[j]);
+    }
+    for (int j0 = 4; j0 < np; j0 += 4) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) o4[j] = j0 + j < np ? __ldcg(o_ptr(j0 + j, h)) : VecT{};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float wj = weight(j0 + j < np ? j0 + j : 0);
+        if (j0 + j < np) add(wj, o4[j]);
+      }
+    }
+    uint16_t* dst = p.out + (row0 + h) * D + lane * CW;
     if constexpr (CW == 4) {
       uint2 o;
-      o.x = ptx::pack_bf16x2(acc[r][0] * iv, acc[r][1] * iv);
-      o.y = ptx::pack_bf16x2(acc[r][2] * iv, acc[r][3] * iv);
+      o.x = ptx::pack_bf16x2(acc[0], acc[1]);
+      o.y = ptx::pack_bf16x2(acc[2], acc[3]);
       *reinterpret_cast<uint2*>(dst) = o;
     } else {
-      *reinterpret_cast<uint32_t*>(dst) = ptx::pack_bf16x2(acc[r][0] * iv, acc[r][1] * iv);
+      *reinterpret_cast<uint32_t*>(dst) = ptx::pack_bf16x2(acc[0], acc[1]);
     }
   }
 }
