@@ -7,6 +7,7 @@ is missing or the tensors are not on a CUDA device, the calls raise.
 
     kv_append(k_new, v_new, k_pages, v_pages, block_table, positions)
     paged_decode_attn(q, k_pages, v_pages, block_table, seq_lens, out=None, scale=None)
+    Pager(num_pages, page_size, max_seqs, max_blocks_per_seq)   host page bookkeeping
 """
 from __future__ import annotations
 
@@ -29,6 +30,7 @@ __all__ = [
     "set_num_workers",
     "set_wait_limit_ns",
     "launch_count",
+    "Pager",
     "EXPORTED_SYMBOLS",
 ]
 
@@ -37,9 +39,10 @@ _LIB_NAME = "libgqa_decode.so"
 
 GQA_OK = 0
 STATUS_NAMES = {0: "GQA_OK", -1: "GQA_ERR_INVALID_ARG", -2: "GQA_ERR_UNSUPPORTED",
-                -3: "GQA_ERR_CUDA", -4: "GQA_ERR_DEVICE_BOUNDS", -5: "GQA_ERR_TIMEOUT"}
+                -3: "GQA_ERR_CUDA", -4: "GQA_ERR_DEVICE_BOUNDS", -5: "GQA_ERR_TIMEOUT",
+                -6: "GQA_ERR_OUT_OF_PAGES"}
 
-# Every extern "C" entry point declared in include/gqa_decode.h.
+# Every extern "C" entry point declared in include/*.h.
 EXPORTED_SYMBOLS = (
     "gqa_kv_append",
     "gqa_paged_decode_attn",
@@ -52,6 +55,15 @@ EXPORTED_SYMBOLS = (
     "gqa_set_wait_limit_ns",
     "gqa_launch_count",
     "gqa_abi_version",
+    # include/gqa_pager.h
+    "gqa_pager_create",
+    "gqa_pager_destroy",
+    "gqa_pager_extend",
+    "gqa_pager_step",
+    "gqa_pager_truncate",
+    "gqa_pager_gather",
+    "gqa_pager_free_pages",
+    "gqa_pager_seq_len",
 )
 
 
@@ -104,6 +116,22 @@ def load_library() -> ctypes.CDLL:
     lib.gqa_launch_count.restype = ctypes.c_uint64
     lib.gqa_abi_version.argtypes = []
     lib.gqa_abi_version.restype = i32
+    lib.gqa_pager_create.argtypes = [i32, i32, i32, i32, ctypes.POINTER(vp)]
+    lib.gqa_pager_create.restype = i32
+    lib.gqa_pager_destroy.argtypes = [vp]
+    lib.gqa_pager_destroy.restype = None
+    lib.gqa_pager_extend.argtypes = [vp, i32, i32]
+    lib.gqa_pager_extend.restype = i32
+    lib.gqa_pager_step.argtypes = [vp, vp, i32, vp, vp]
+    lib.gqa_pager_step.restype = i32
+    lib.gqa_pager_truncate.argtypes = [vp, i32, i32]
+    lib.gqa_pager_truncate.restype = i32
+    lib.gqa_pager_gather.argtypes = [vp, vp, i32, vp, vp]
+    lib.gqa_pager_gather.restype = i32
+    lib.gqa_pager_free_pages.argtypes = [vp]
+    lib.gqa_pager_free_pages.restype = i32
+    lib.gqa_pager_seq_len.argtypes = [vp, i32]
+    lib.gqa_pager_seq_len.restype = i32
     _lib = lib
     return lib
 
@@ -272,3 +300,76 @@ def set_wait_limit_ns(limit_ns: int, arm_without_copy: bool = False) -> None:
 
 def launch_count() -> int:
     return int(load_library().gqa_launch_count())
+
+
+def _host_i32(x, name: str) -> torch.Tensor:
+    t = torch.as_tensor(x, dtype=torch.int32)
+    if t.device.type != "cpu":
+        raise ValueError(f"{name} must be on the host")
+    return t.contiguous().reshape(-1)
+
+
+class Pager:
+    """Host page bookkeeping for one preallocated page pool (include/gqa_pager.h).
+
+    Slots own pool pages in token order; `gather` gives the block table and lengths of a
+    batch of slots (host int32 tensors, ready to copy to the device), `step` grows every
+    listed slot by one token and returns the new tokens' positions and the new lengths.
+    Every call is all-or-nothing and raises GQAError (GQA_ERR_OUT_OF_PAGES when the free
+    list is too short).  Host-only and not thread-safe.
+    """
+
+    def __init__(self, num_pages: int, page_size: int, max_seqs: int, max_blocks_per_seq: int):
+        self._lib = load_library()
+        h = ctypes.c_void_p()
+        _check(self._lib.gqa_pager_create(int(num_pages), int(page_size), int(max_seqs),
+                                          int(max_blocks_per_seq), ctypes.byref(h)))
+        self._h = h
+        self.num_pages, self.page_size = int(num_pages), int(page_size)
+        self.max_seqs, self.max_blocks_per_seq = int(max_seqs), int(max_blocks_per_seq)
+
+    def close(self) -> None:
+        if getattr(self, "_h", None) is not None and self._h.value:
+            self._lib.gqa_pager_destroy(self._h)
+        self._h = None
+
+    def __del__(self):
+        self.close()
+
+    def _handle(self):
+        if self._h is None:
+            raise ValueError("pager is closed")
+        return self._h
+
+    def extend(self, seq: int, n_tokens: int) -> None:
+        _check(self._lib.gqa_pager_extend(self._handle(), int(seq), int(n_tokens)))
+
+    def step(self, seqs):
+        s = _host_i32(seqs, "seqs")
+        pos = torch.empty(s.numel(), dtype=torch.int32)
+        lens = torch.empty(s.numel(), dtype=torch.int32)
+        _check(self._lib.gqa_pager_step(self._handle(), s.data_ptr(), s.numel(), pos.data_ptr(), lens.data_ptr()))
+        return pos, lens
+
+    def truncate(self, seq: int, new_len: int) -> None:
+        _check(self._lib.gqa_pager_truncate(self._handle(), int(seq), int(new_len)))
+
+    def release(self, seq: int) -> None:
+        self.truncate(seq, 0)
+
+    def gather(self, seqs):
+        s = _host_i32(seqs, "seqs")
+        bt = torch.empty(s.numel(), self.max_blocks_per_seq, dtype=torch.int32)
+        lens = torch.empty(s.numel(), dtype=torch.int32)
+        _check(self._lib.gqa_pager_gather(self._handle(), s.data_ptr(), s.numel(), bt.data_ptr(), lens.data_ptr()))
+        return bt, lens
+
+    @property
+    def free_pages(self) -> int:
+        return int(self._lib.gqa_pager_free_pages(self._handle()))
+
+    def seq_len(self, seq: int) -> int:
+        n = int(self._lib.gqa_pager_seq_len(self._handle(), int(seq)))
+        if n < 0:
+            raise ValueError(f"slot {seq} out of range")
+        return n

@@ -1,4 +1,5 @@
-"""Build the CUDA library in-tree: csrc/*.cu -> libgqa_decode.so (sm_100a only).
+"""Build the CUDA library in-tree: csrc/*.cu (+ host-only csrc/*.cpp) -> libgqa_decode.so
+(sm_100a only).
 
 Usage:  python -m gqa_decode_attention_04_b200.build [--verbose]
 The shared object is written next to this file so it travels with the source tree.
@@ -31,7 +32,7 @@ def _nvcc() -> str:
 
 
 def sources():
-    return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cpp")))
 
 
 def needs_rebuild() -> bool:
@@ -49,7 +50,7 @@ def build(verbose: bool = False, force: bool = False) -> str:
     os.makedirs(objdir, exist_ok=True)
     objs = []
     for src in sources():
-        obj = os.path.join(objdir, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(objdir, os.path.splitext(os.path.basename(src))[0] + ".o")
         cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if verbose or r.returncode != 0:

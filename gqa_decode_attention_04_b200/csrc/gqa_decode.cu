@@ -34,6 +34,18 @@ gqa_status fail(gqa_status s, const char* fmt, ...) {
   return s;
 }
 
+}  // namespace
+
+gqa_status gqa::set_error(gqa_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err_msg, sizeof(g_err_msg), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+namespace {
+
 gqa_status cuda_fail(cudaError_t e, const char* what) {
   return fail(GQA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
 }

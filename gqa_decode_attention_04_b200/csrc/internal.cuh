@@ -5,7 +5,12 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "gqa_decode.h"
+
 namespace gqa {
+
+// Sets the calling thread's gqa_last_error_string() text and returns s.
+gqa_status set_error(gqa_status s, const char* fmt, ...);
 
 // Bits of the per-device error word.
 enum : uint32_t {

@@ -75,7 +75,8 @@ typedef enum {
   GQA_ERR_UNSUPPORTED = -2,   /* valid but not built: head_dim, page_size, limits  */
   GQA_ERR_CUDA = -3,          /* a CUDA runtime/driver call failed                 */
   GQA_ERR_DEVICE_BOUNDS = -4, /* device-side index out of range (work skipped)     */
-  GQA_ERR_TIMEOUT = -5        /* a kernel's bounded wait ran out (work skipped)    */
+  GQA_ERR_TIMEOUT = -5,       /* a kernel's bounded wait ran out (work skipped)    */
+  GQA_ERR_OUT_OF_PAGES = -6   /* gqa_pager.h: the free list is too short           */
 } gqa_status;
 
 /*

@@ -1,6 +1,7 @@
 """CPU tests of the C-ABI library: it loads, exports every declared entry point, and
 rejects bad arguments on the host before touching a GPU."""
 import ctypes
+import glob
 import json
 import os
 import re
@@ -10,7 +11,7 @@ import pytest
 import gqa_decode_attention_04_b200 as gq
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "gqa_decode.h")
+HEADERS = sorted(glob.glob(os.path.join(ROOT, "include", "*.h")))
 
 
 @pytest.fixture(scope="module")
@@ -22,7 +23,7 @@ def lib():
 
 
 def _declared_functions():
-    text = open(HEADER).read()
+    text = "".join(open(h).read() for h in HEADERS)
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(gqa_[a-z0-9_]+)\s*\(", text)))
 
