@@ -12,6 +12,9 @@ from .paged_attention import (  # noqa: F401
     paged_decode_attention,
     paged_decode_attention_rows,
     kv_append,
+    multi_query_window,
+    paged_multi_query_attention,
+    kv_append_multi,
     partial_softmax_piece,
     merge_partial_pieces,
     kv_cache_bytes,

@@ -29,6 +29,11 @@ Readings where the pages are silent (each is restated in the design notes):
   * seq_len == 0 yields an all-zero output row.
   * the split-KV combine (FlashDecoding) is not spelled out on the pages; the
     oracle states the plain log-sum-exp merge of softmax pieces.
+  * several query tokens per sequence (the MQA plugin's entry point carries a
+    query length, seq_q, beside seq_kv): they are the sequence's q_len newest
+    tokens, and each attends to itself and every token before it, as the
+    same tokens would one step at a time (speculative verification, chunked
+    prefill over the cache).
 
 Every function is pinned by tests in tests/test_oracle.py against closed forms,
 a library routine (torch scaled_dot_product_attention in float64), brute-force
@@ -50,6 +55,9 @@ __all__ = [
     "paged_decode_attention",
     "paged_decode_attention_rows",
     "kv_append",
+    "multi_query_window",
+    "paged_multi_query_attention",
+    "kv_append_multi",
     "partial_softmax_piece",
     "merge_partial_pieces",
     "kv_cache_bytes",
@@ -172,6 +180,54 @@ def kv_append(k_pages_bits, v_pages_bits, k_new_bits, v_new_bits, block_table,
         slot = pos % ps
         k[page, :, slot, :] = k_new_bits[b]
         v[page, :, slot, :] = v_new_bits[b]
+    return k, v
+
+
+def multi_query_window(seq_len: int, q_len: int, i: int) -> int:
+    """Tokens that query token i of q_len sees when the sequence holds seq_len tokens
+    (the q_len newest included): positions 0 .. seq_len - q_len + i, none if that is
+    negative."""
+    return max(0, min(seq_len, seq_len - q_len + 1 + i))
+
+
+def paged_multi_query_attention(q_bits, k_pages_bits, v_pages_bits, block_table,
+                                seq_lens, scale: float) -> np.ndarray:
+    """Attention of q_len query tokens per sequence over the paged cache: [B, Q, H, D].
+
+    q_bits [B, Q, H, D] uint16.  Query token i of sequence b is the token at
+    position seq_lens[b] - Q + i; it attends to the first multi_query_window(...)
+    tokens of its sequence.  With Q = 1 this is paged_decode_attention.
+    """
+    B, Q, H, D = q_bits.shape
+    Hk, ps = k_pages_bits.shape[1], k_pages_bits.shape[2]
+    out = np.zeros((B, Q, H, D), dtype=np.float64)
+    q = bf16_bits_to_f64(q_bits)
+    for b in range(B):
+        L = int(seq_lens[b])
+        for kvh in range(Hk):
+            K = gather_sequence_kv(k_pages_bits, block_table[b], kvh, L, ps)
+            V = gather_sequence_kv(v_pages_bits, block_table[b], kvh, L, ps)
+            for i in range(Q):
+                n = multi_query_window(L, Q, i)
+                for h in range(H):
+                    if kv_head_of(h, H, Hk) == kvh:
+                        out[b, i, h] = attend_one_query(q[b, i, h], K[:n], V[:n], scale)
+    return out
+
+
+def kv_append_multi(k_pages_bits, v_pages_bits, k_new_bits, v_new_bits, block_table,
+                    positions) -> Tuple[np.ndarray, np.ndarray]:
+    """q_len new rows per sequence: k_new [B, Q, Hk, D]; row i of sequence b goes to
+    token position positions[b] + i (same page/slot rule as kv_append)."""
+    k = np.array(k_pages_bits, copy=True)
+    v = np.array(v_pages_bits, copy=True)
+    ps = k.shape[2]
+    for b in range(k_new_bits.shape[0]):
+        for i in range(k_new_bits.shape[1]):
+            pos = int(positions[b]) + i
+            page = int(block_table[b][pos // ps])
+            k[page, :, pos % ps, :] = k_new_bits[b, i]
+            v[page, :, pos % ps, :] = v_new_bits[b, i]
     return k, v
 
 

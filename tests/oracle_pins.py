@@ -359,6 +359,81 @@ def check_lse_merge():
     assert abs(lse - math.log(np.sum(np.exp(s)))) < 1e-11
 
 
+def _random_multi(rng, seq_lens, Q, H, Hk, D, ps):
+    """A paged cache as _random_paged plus a [B, Q, H, D] block of query tokens."""
+    _, kp, vp, bt, Kc, Vc = _random_paged(rng, seq_lens, H, Hk, D, ps)
+    return _rand_bits(rng, (len(seq_lens), Q, H, D)), kp, vp, bt, Kc, Vc
+
+
+def check_multi_query_against_sdpa_causal():
+    """Several query tokens per sequence against torch scaled_dot_product_attention
+    (CPU, float64) with an explicit boolean mask: query token i (the token at position
+    L - Q + i) may read key j iff j <= L - Q + i."""
+    rng = np.random.default_rng(21)
+    for sl, Q, H, Hk, D, ps in (([9, 40, 17], 4, 8, 2, 16, 16), ([33, 5], 3, 6, 1, 8, 4),
+                                ([64, 7], 7, 4, 4, 32, 16)):
+        q, kp, vp, bt, Kc, Vc = _random_multi(rng, sl, Q, H, Hk, D, ps)
+        scale = 0.3
+        got = PA.paged_multi_query_attention(q, kp, vp, bt, np.array(sl), scale)
+        G = H // Hk
+        for b, L in enumerate(sl):
+            qt = torch.from_numpy(PA.bf16_bits_to_f64(q[b])).permute(1, 0, 2)[None]   # [1, H, Q, D]
+            Kt = torch.from_numpy(PA.bf16_bits_to_f64(Kc[b])).repeat_interleave(G, dim=0)[None]
+            Vt = torch.from_numpy(PA.bf16_bits_to_f64(Vc[b])).repeat_interleave(G, dim=0)[None]
+            allowed = torch.arange(L)[None, :] <= (L - Q + torch.arange(Q))[:, None]
+            ok = allowed.any(dim=1)
+            o = torch.nn.functional.scaled_dot_product_attention(qt, Kt, Vt, attn_mask=allowed, scale=scale)
+            want = o[0].permute(1, 0, 2).numpy()                                    # [Q, H, D]
+            assert np.allclose(got[b][ok.numpy()], want[ok.numpy()], rtol=0, atol=1e-12), (sl, Q, b)
+            assert np.all(got[b][~ok.numpy()] == 0.0)                                # empty windows
+
+
+def check_multi_query_single_token_and_newest():
+    """q_len = 1 is the decode; the newest query token sees the whole sequence, the
+    oldest sees all but the q_len - 1 tokens after it."""
+    rng = np.random.default_rng(22)
+    sl, H, Hk, D, ps = [30, 3, 17], 4, 2, 16, 8
+    q, kp, vp, bt, Kc, Vc = _random_multi(rng, sl, 1, H, Hk, D, ps)
+    one = PA.paged_multi_query_attention(q, kp, vp, bt, np.array(sl), 0.5)[:, 0]
+    assert np.array_equal(one, PA.paged_decode_attention(q[:, 0], kp, vp, bt, np.array(sl), 0.5))
+    Q = 3
+    q, kp, vp, bt, Kc, Vc = _random_multi(rng, sl, Q, H, Hk, D, ps)
+    got = PA.paged_multi_query_attention(q, kp, vp, bt, np.array(sl), 0.5)
+    assert np.array_equal(got[:, Q - 1], PA.paged_decode_attention(q[:, Q - 1], kp, vp, bt, np.array(sl), 0.5))
+    shorter = np.maximum(np.array(sl) - (Q - 1), 0)
+    assert np.array_equal(got[:, 0], PA.paged_decode_attention(q[:, 0], kp, vp, bt, shorter, 0.5))
+    assert PA.multi_query_window(3, 3, 0) == 1 and PA.multi_query_window(2, 4, 0) == 0
+    assert PA.multi_query_window(2, 4, 3) == 2 and PA.multi_query_window(0, 1, 0) == 0
+
+
+def check_kv_append_multi():
+    """Row i of sequence b lands at position positions[b] + i bit for bit (gathered
+    back through the block table); every other byte is unchanged; q_len = 1 is kv_append."""
+    rng = np.random.default_rng(23)
+    sl = [20, 6, 33]
+    Hk, D, ps, Q = 2, 8, 4, 3
+    _, kp, vp, bt, Kc, Vc = _random_paged(rng, sl, 4, Hk, D, ps, extra_pages=2)
+    pos = np.array([17, 3, 30])
+    kn = _rand_bits(rng, (3, Q, Hk, D))
+    vn = _rand_bits(rng, (3, Q, Hk, D))
+    k2, v2 = PA.kv_append_multi(kp, vp, kn, vn, bt, pos)
+    changed = np.zeros(kp.shape[:3], dtype=bool)
+    for b in range(3):
+        for kvh in range(Hk):
+            gk = PA.gather_sequence_kv(k2, bt[b], kvh, pos[b] + Q, ps)
+            gv = PA.gather_sequence_kv(v2, bt[b], kvh, pos[b] + Q, ps)
+            for i in range(Q):
+                assert np.array_equal(gk[pos[b] + i], PA.bf16_bits_to_f64(kn[b, i, kvh]))
+                assert np.array_equal(gv[pos[b] + i], PA.bf16_bits_to_f64(vn[b, i, kvh]))
+        for i in range(Q):
+            t = pos[b] + i
+            changed[bt[b, t // ps], :, t % ps] = True
+    assert np.array_equal(k2[~changed], kp[~changed]) and np.array_equal(v2[~changed], vp[~changed])
+    k1, v1 = PA.kv_append_multi(kp, vp, kn[:, :1], vn[:, :1], bt, pos)
+    k0, v0 = PA.kv_append(kp, vp, kn[:, 0], vn[:, 0], bt, pos)
+    assert np.array_equal(k1, k0) and np.array_equal(v1, v0)
+
+
 ALL_CHECKS = [
     check_bf16_decode,
     check_closed_form_three_tokens,
@@ -377,4 +452,7 @@ ALL_CHECKS = [
     check_kv_append,
     check_kv_cache_bytes,
     check_lse_merge,
+    check_multi_query_against_sdpa_causal,
+    check_multi_query_single_token_and_newest,
+    check_kv_append_multi,
 ]

@@ -84,6 +84,33 @@ def _cache_bytes_single(num_layers, num_kv_heads, head_dim, seq_len, batch=1, by
     return num_layers * num_kv_heads * head_dim * seq_len * batch * bytes_per_elem  # K only
 
 
+def _window_excludes_self(seq_len, q_len, i):
+    return max(0, min(seq_len, seq_len - q_len + i))   # a query token misses itself
+
+
+def _window_sees_drafts(seq_len, q_len, i):
+    return seq_len                                  # no causal limit among new tokens
+
+
+def _append_multi_reversed(kp, vp, kn, vn, bt, positions):
+    return PA.kv_append(kp, vp, kn[:, -1], vn[:, -1], bt, positions) if kn.shape[1] == 1 else \
+        _append_multi_rows_reversed(kp, vp, kn, vn, bt, positions)
+
+
+def _append_multi_rows_reversed(kp, vp, kn, vn, bt, positions):
+    k = np.array(kp, copy=True)
+    v = np.array(vp, copy=True)
+    ps = k.shape[2]
+    Q = kn.shape[1]
+    for b in range(kn.shape[0]):
+        for i in range(Q):
+            pos = int(positions[b]) + i
+            pg = int(bt[b][pos // ps])
+            k[pg, :, pos % ps, :] = kn[b, Q - 1 - i]   # rows in reverse order
+            v[pg, :, pos % ps, :] = vn[b, Q - 1 - i]
+    return k, v
+
+
 MUTANTS = [
     ("kv_head_of", _kv_head_modulo),
     ("gather_sequence_kv", _gather_swapped),
@@ -95,6 +122,9 @@ MUTANTS = [
     ("merge_partial_pieces", _merge_no_weights),
     ("kv_append", _append_wrong_slot),
     ("kv_cache_bytes", _cache_bytes_single),
+    ("multi_query_window", _window_excludes_self),
+    ("multi_query_window", _window_sees_drafts),
+    ("kv_append_multi", _append_multi_reversed),
 ]
 
 
