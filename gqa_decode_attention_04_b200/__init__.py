@@ -25,6 +25,9 @@ __all__ = [
     "paged_decode_attn",
     "decode_step",
     "paged_decode_attn_noalloc",
+    "kv_append_multi",
+    "paged_multi_query_attn",
+    "multi_query_step",
     "check_device_error",
     "kv_cache_bytes",
     "set_num_workers",
@@ -48,6 +51,9 @@ EXPORTED_SYMBOLS = (
     "gqa_paged_decode_attn",
     "gqa_decode_step",
     "gqa_paged_decode_attn_noalloc",
+    "gqa_kv_append_multi",
+    "gqa_paged_multi_query_attn",
+    "gqa_multi_query_step",
     "gqa_check_device_error",
     "gqa_last_error_string",
     "gqa_kv_cache_bytes",
@@ -102,6 +108,14 @@ def load_library() -> ctypes.CDLL:
     lib.gqa_decode_step.restype = i32
     lib.gqa_paged_decode_attn_noalloc.argtypes = lib.gqa_paged_decode_attn.argtypes
     lib.gqa_paged_decode_attn_noalloc.restype = i32
+    lib.gqa_kv_append_multi.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp]
+    lib.gqa_kv_append_multi.restype = i32
+    lib.gqa_paged_multi_query_attn.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32,
+                                               i32, i32, vp]
+    lib.gqa_paged_multi_query_attn.restype = i32
+    lib.gqa_multi_query_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                         f32, i32, i32, vp]
+    lib.gqa_multi_query_step.restype = i32
     lib.gqa_check_device_error.argtypes = [vp]
     lib.gqa_check_device_error.restype = i32
     lib.gqa_last_error_string.argtypes = []
@@ -247,6 +261,102 @@ def decode_step(q, k_new, v_new, k_pages, v_pages, block_table, positions, seq_l
                                    v_pages.data_ptr(), block_table.data_ptr(), positions.data_ptr(),
                                    seq_lens.data_ptr(), out.data_ptr(), B, H, Hk, D, ps, float(scale),
                                    block_table.shape[1], P, _stream_ptr(stream)))
+    return out
+
+
+def _multi_shapes(q, k_pages, v_pages, block_table, seq_lens):
+    B, Q, H, D = q.shape
+    P, Hk, ps, D2 = k_pages.shape
+    if D2 != D or tuple(v_pages.shape) != (P, Hk, ps, D):
+        raise ValueError("page pools must be [num_pages, num_kv_heads, page_size, head_dim]")
+    if block_table.dim() != 2 or block_table.shape[0] != B or tuple(seq_lens.shape) != (B,):
+        raise ValueError("block_table must be [num_seqs, max_blocks], seq_lens [num_seqs]")
+    return B, Q, H, D, P, Hk, ps
+
+
+def _multi_out(out, shape, dev):
+    if out is None:
+        return torch.empty(shape, dtype=torch.bfloat16, device=dev)
+    _need(out, "out", torch.bfloat16, dev)
+    if tuple(out.shape) != tuple(shape):
+        raise ValueError(f"out must be {list(shape)}")
+    return out
+
+
+def kv_append_multi(k_new, v_new, k_pages, v_pages, block_table, positions, stream=None) -> None:
+    """Write k_new/v_new [B, Q, Hk, D]: row i of sequence b to position positions[b] + i."""
+    dev = k_pages.device
+    for t, n, dt in ((k_new, "k_new", torch.bfloat16), (v_new, "v_new", torch.bfloat16),
+                     (k_pages, "k_pages", torch.bfloat16), (v_pages, "v_pages", torch.bfloat16),
+                     (block_table, "block_table", torch.int32), (positions, "positions", torch.int32)):
+        _need(t, n, dt, dev)
+    P, Hk, ps, D = k_pages.shape
+    if tuple(v_pages.shape) != (P, Hk, ps, D):
+        raise ValueError("v_pages shape differs from k_pages")
+    if k_new.dim() != 4:
+        raise ValueError("k_new / v_new must be [num_seqs, q_len, num_kv_heads, head_dim]")
+    B, Q = k_new.shape[0], k_new.shape[1]
+    if tuple(k_new.shape) != (B, Q, Hk, D) or tuple(v_new.shape) != (B, Q, Hk, D):
+        raise ValueError("k_new / v_new must be [num_seqs, q_len, num_kv_heads, head_dim]")
+    if block_table.dim() != 2 or block_table.shape[0] != B or tuple(positions.shape) != (B,):
+        raise ValueError("block_table must be [num_seqs, max_blocks], positions [num_seqs]")
+    lib = load_library()
+    with torch.cuda.device(dev):
+        _check(lib.gqa_kv_append_multi(k_new.data_ptr(), v_new.data_ptr(), k_pages.data_ptr(),
+                                       v_pages.data_ptr(), block_table.data_ptr(), positions.data_ptr(),
+                                       B, Q, Hk, D, ps, block_table.shape[1], P, _stream_ptr(stream)))
+
+
+def paged_multi_query_attn(q, k_pages, v_pages, block_table, seq_lens, out: Optional[torch.Tensor] = None,
+                           scale: Optional[float] = None, stream=None) -> torch.Tensor:
+    """q [B, Q, H, D]: query token i of sequence b (position seq_lens[b] - Q + i) attends to
+    positions 0 .. seq_lens[b] - Q + i; out [B, Q, H, D] bf16."""
+    dev = q.device
+    for t, n, dt in ((q, "q", torch.bfloat16), (k_pages, "k_pages", torch.bfloat16),
+                     (v_pages, "v_pages", torch.bfloat16), (block_table, "block_table", torch.int32),
+                     (seq_lens, "seq_lens", torch.int32)):
+        _need(t, n, dt, dev)
+    if q.dim() != 4:
+        raise ValueError("q must be [num_seqs, q_len, num_heads, head_dim]")
+    B, Q, H, D, P, Hk, ps = _multi_shapes(q, k_pages, v_pages, block_table, seq_lens)
+    out = _multi_out(out, (B, Q, H, D), dev)
+    if scale is None:
+        scale = 1.0 / (D ** 0.5)
+    lib = load_library()
+    with torch.cuda.device(dev):
+        _check(lib.gqa_paged_multi_query_attn(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(),
+                                              block_table.data_ptr(), seq_lens.data_ptr(), out.data_ptr(),
+                                              B, Q, H, Hk, D, ps, float(scale), block_table.shape[1], P,
+                                              _stream_ptr(stream)))
+    return out
+
+
+def multi_query_step(q, k_new, v_new, k_pages, v_pages, block_table, positions, seq_lens,
+                     out: Optional[torch.Tensor] = None, scale: Optional[float] = None,
+                     stream=None) -> torch.Tensor:
+    """kv_append_multi of k_new/v_new [B, Q, Hk, D] at positions, then paged_multi_query_attn."""
+    dev = q.device
+    for t, n, dt in ((q, "q", torch.bfloat16), (k_new, "k_new", torch.bfloat16),
+                     (v_new, "v_new", torch.bfloat16), (k_pages, "k_pages", torch.bfloat16),
+                     (v_pages, "v_pages", torch.bfloat16), (block_table, "block_table", torch.int32),
+                     (positions, "positions", torch.int32), (seq_lens, "seq_lens", torch.int32)):
+        _need(t, n, dt, dev)
+    if q.dim() != 4:
+        raise ValueError("q must be [num_seqs, q_len, num_heads, head_dim]")
+    B, Q, H, D, P, Hk, ps = _multi_shapes(q, k_pages, v_pages, block_table, seq_lens)
+    if tuple(k_new.shape) != (B, Q, Hk, D) or tuple(v_new.shape) != (B, Q, Hk, D):
+        raise ValueError("k_new / v_new must be [num_seqs, q_len, num_kv_heads, head_dim]")
+    if tuple(positions.shape) != (B,):
+        raise ValueError("positions must be [num_seqs]")
+    out = _multi_out(out, (B, Q, H, D), dev)
+    if scale is None:
+        scale = 1.0 / (D ** 0.5)
+    lib = load_library()
+    with torch.cuda.device(dev):
+        _check(lib.gqa_multi_query_step(q.data_ptr(), k_new.data_ptr(), v_new.data_ptr(), k_pages.data_ptr(),
+                                        v_pages.data_ptr(), block_table.data_ptr(), positions.data_ptr(),
+                                        seq_lens.data_ptr(), out.data_ptr(), B, Q, H, Hk, D, ps, float(scale),
+                                        block_table.shape[1], P, _stream_ptr(stream)))
     return out
 
 

@@ -65,7 +65,7 @@ struct StageInfo {
   int nvalid;        // valid tokens of this block (1..64)
   int submask;       // bit s: sub-chunk s was loaded
   int flags;
-  int pad;
+  int rem;           // tokens of the sequence from this block's first one on (unclamped)
 };
 enum : int { kFirstOfPiece = 1, kLastOfPiece = 2, kSole = 4, kFirstPieceOfCta = 8 };
 
@@ -111,12 +111,16 @@ __device__ __forceinline__ int piece_slot(int64_t w, int64_t seg_base, int64_t T
 
 // One 16-token sub-chunk for NT n-tiles of 8 heads: S^T = K Q^T, online softmax down the
 // token axis, O^T += V^T P^T.  kb/vb: shared addresses of the sub-chunk's swizzled K/V.
-template <int D, int NT>
+// MQ (several query tokens per sequence): column (head) e of n-tile nt sees only the
+// first rem - cdrop[nt][e] tokens from this sub-chunk's first one (rem: tokens of the
+// sequence from there on; cdrop: newer query tokens than the column's own).
+template <int D, int NT, bool MQ>
 __device__ __forceinline__ void attend_subchunk(uint32_t kb, uint32_t vb, int nvalid,
                                                 const uint32_t (&kofs)[4], const uint32_t (&vofs)[4],
                                                 const uint32_t (&qf)[D / 16][NT][2],
                                                 float (&o)[D / 16][NT][4], float (&mref)[NT][2],
-                                                float (&lsum)[NT][2], float sl2, int g, int q) {
+                                                float (&lsum)[NT][2], float sl2, int g, int q,
+                                                int rem, int max_drop, const int (&cdrop)[NT][2]) {
   using G_ = Geo<D>;
   constexpr int KS = D / 16;
   constexpr int MT = D / 16;
@@ -138,7 +142,18 @@ __device__ __forceinline__ void attend_subchunk(uint32_t kb, uint32_t vb, int nv
   for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
     for (int e = 0; e < 4; ++e) sc[nt][e] = (s[0][nt][e] + s[1][nt][e]) * sl2;
-  if (nvalid < kChunk) {
+  if constexpr (MQ) {
+    if (rem - max_drop < kChunk) {  // a column's window may end inside this sub-chunk
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int lim = rem - cdrop[nt][e];
+          if (g >= lim) sc[nt][e] = -INFINITY;
+          if (g + 8 >= lim) sc[nt][e + 2] = -INFINITY;
+        }
+    }
+  } else if (nvalid < kChunk) {
     const bool v0 = g < nvalid, v1 = g + 8 < nvalid;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
@@ -230,8 +245,10 @@ template <bool SPLIT_HEADS>
 constexpr int ctas_per_sm() { return SPLIT_HEADS ? GQA_CTAS_HEAD_SPLIT : GQA_CTAS_TOKEN_SPLIT; }
 
 // D: head_dim.  NT: 8-head n-tiles per consumer.  SPLIT_HEADS: consumers split the
-// query heads (else the 64 tokens of a stage).  C: consumer warps.  S: stages.
-template <int D, int NT, bool SPLIT_HEADS, int C, int S>
+// query heads (else the 64 tokens of a stage).  C: consumer warps.  S: stages.  MQ:
+// several query tokens per sequence (p.q_len): a kv head's rows are its group of heads
+// for each query token in turn (row r: token r / group, head r % group), one segment.
+template <int D, int NT, bool SPLIT_HEADS, int C, int S, bool MQ>
 __global__ void __launch_bounds__((C + (SPLIT_HEADS ? 1 : 2)) * 32, ctas_per_sm<SPLIT_HEADS>())
 decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
                  const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
@@ -253,6 +270,17 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
   const int B = p.num_seqs;
   const int segs = p.num_kv_heads * p.n_ht;
   const int cap = p.max_blocks * p.page_size;
+  // Rows per kv head, and the memory row (of q and out) of row r of kv head kvh.
+  const int grp = MQ ? p.group * p.q_len : p.group;
+  auto seq_row = [&](int b, int kvh, int r) -> int64_t {
+    if constexpr (MQ) {
+      const int i = r / p.group;
+      return (static_cast<int64_t>(b) * p.q_len + i) * p.num_heads + kvh * p.group + (r - i * p.group);
+    } else {
+      return static_cast<int64_t>(b) * p.num_heads + kvh * p.group + r;
+    }
+  };
+  const int rows_per_seq = MQ ? p.num_heads * p.q_len : p.num_heads;
 
   // ---------------------------------------------------------------- prologue
   // Pass 1: block counts per sequence, their total T (and zero rows of empty sequences).
@@ -263,8 +291,8 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int Le = eff_len(L, cap);
     if ((L < 0 || L > cap) && blockIdx.x == 0) atomicOr(p.err, kErrBounds);
     if (Le == 0 && (b % gridDim.x) == blockIdx.x) {
-      uint32_t* o = reinterpret_cast<uint32_t*>(p.out + static_cast<int64_t>(b) * p.num_heads * D);
-      for (int i = 0; i < p.num_heads * D / 2; ++i) o[i] = 0u;
+      uint32_t* o = reinterpret_cast<uint32_t*>(p.out + static_cast<int64_t>(b) * rows_per_seq * D);
+      for (int i = 0; i < rows_per_seq * D / 2; ++i) o[i] = 0u;
     }
     const int64_t n = static_cast<int64_t>((Le + kBlock - 1) / kBlock) * segs;
     if (b == static_cast<int>(threadIdx.x)) n_first = n;
@@ -427,15 +455,21 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
     // Bytes of a piece's query rows (contiguous in q): the token split stages them.
     auto q_rows_bytes = [&](const Cursor& c) -> uint32_t {
       const int ht = c.seg % p.n_ht;
-      return static_cast<uint32_t>(min(NH, p.group - ht * NH)) * D * 2u;
+      return static_cast<uint32_t>(min(NH, grp - ht * NH)) * D * 2u;
     };
     // Pull a piece's query rows into L2 ahead of the consumers that load them.
     auto prefetch_q = [&](const Cursor& c) {
       const int kvh = c.seg / p.n_ht, ht = c.seg % p.n_ht;
-      const int nrows = min(p.heads_per_seg, p.group - ht * p.heads_per_seg);
-      const uint8_t* q0 = reinterpret_cast<const uint8_t*>(
-          p.q + (static_cast<int64_t>(c.b) * p.num_heads + kvh * p.group + ht * p.heads_per_seg) * D);
-      for (int off = lane * 128; off < nrows * D * 2; off += 32 * 128) ptx::prefetch_l2(q0 + off);
+      const int nrows = min(p.heads_per_seg, grp - ht * p.heads_per_seg);
+      if constexpr (MQ) {  // rows of one query token at a time are contiguous
+        for (int r = lane; r < nrows; r += 32) {
+          const uint8_t* qr = reinterpret_cast<const uint8_t*>(p.q + seq_row(c.b, kvh, ht * p.heads_per_seg + r) * D);
+          for (int off = 0; off < D * 2; off += 128) ptx::prefetch_l2(qr + off);
+        }
+      } else {
+        const uint8_t* q0 = reinterpret_cast<const uint8_t*>(p.q + seq_row(c.b, kvh, ht * p.heads_per_seg) * D);
+        for (int off = lane * 128; off < nrows * D * 2; off += 32 * 128) ptx::prefetch_l2(q0 + off);
+      }
     };
     int page = page_of(cu);
     if (SPLIT_HEADS) prefetch_q(cu);
@@ -472,6 +506,7 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
         si.nblk = cu.nblk;
         si.nvalid = nvalid;
         si.submask = static_cast<int>(submask);
+        si.rem = cu.len - cu.blk * kBlock;
         si.flags = (first ? kFirstOfPiece : 0) | (last ? kLastOfPiece : 0) |
                    ((last && piece_blk0 == 0 && cu.blk + 1 == cu.nblk) ? kSole : 0) |
                    (first_piece ? kFirstPieceOfCta : 0);
@@ -482,10 +517,21 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
       }
       if (i == 0) ptx::pdl_wait_prerequisites();  // K/V may still be written by the previous kernel
       __syncwarp();
-      if (!SPLIT_HEADS && first && lane == kSubChunks && !p.arm_without_copy) {
-        const int kvh = cu.seg / p.n_ht, ht = cu.seg % p.n_ht;
-        const uint16_t* src = p.q + (static_cast<int64_t>(cu.b) * p.num_heads + kvh * p.group + ht * NH) * D;
-        ptx::bulk_load(ptx::smem_u32(qbuf + stage * kQBytes), src, q_rows_bytes(cu), full_bar + 8 * stage);
+      if constexpr (!SPLIT_HEADS) {
+        if (first && !p.arm_without_copy) {
+          const int kvh = cu.seg / p.n_ht, ht = cu.seg % p.n_ht;
+          if constexpr (MQ) {
+            // One copy per query token (its group's rows are contiguous in q); a
+            // segment is the whole kv head (ht == 0) when there are several tokens.
+            for (int i = lane - kSubChunks; i >= 0 && i < p.q_len; i += 32 - kSubChunks)
+              ptx::bulk_load(ptx::smem_u32(qbuf + stage * kQBytes) + i * p.group * D * 2,
+                             p.q + seq_row(cu.b, kvh, i * p.group) * D,
+                             static_cast<uint32_t>(p.group) * D * 2u, full_bar + 8 * stage);
+          } else if (lane == kSubChunks) {
+            ptx::bulk_load(ptx::smem_u32(qbuf + stage * kQBytes), p.q + seq_row(cu.b, kvh, ht * NH) * D,
+                           q_rows_bytes(cu), full_bar + 8 * stage);
+          }
+        }
       }
       if (ok && !p.arm_without_copy) {
         const int kvh = cu.seg / p.n_ht;
@@ -535,8 +581,7 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const float* ml = cml + stage * C * NH * 2;  // [C][NH][2]
         const uint8_t* st = base_ptr + stage * G_::kStageBytes;
         const int kvh = si.seg / p.n_ht, ht = si.seg % p.n_ht;
-        const int nrows = min(hps, p.group - ht * hps);
-        const int64_t row0 = static_cast<int64_t>(si.b) * p.num_heads + kvh * p.group + ht * hps;
+        const int nrows = min(hps, grp - ht * hps);
         const bool sole = si.flags & kSole;
         const int64_t slot = w * 2 + ((si.flags & kFirstPieceOfCta) ? 0 : 1);
         for (int h = 0; h < nrows; ++h) {
@@ -564,7 +609,7 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
           }
           if (sole) {
             const float inv = L > 0.f ? 1.f / L : 0.f;
-            uint16_t* dst = p.out + (row0 + h) * D + d0;
+            uint16_t* dst = p.out + seq_row(si.b, kvh, ht * hps + h) * D + d0;
             if constexpr (CPL == 4) {
               uint2 v;
               v.x = ptx::pack_bf16x2(acc[0] * inv, acc[1] * inv);
@@ -639,7 +684,7 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
               for (int k = 0; k < 8; ++k) {
                 if (h0 + k < nrows) {
                   const float inv = L[k] > 0.f ? 1.f / L[k] : 0.f;
-                  uint16_t* dst = p.out + (row0 + h0 + k) * D + d0;
+                  uint16_t* dst = p.out + seq_row(si.b, kvh, ht * hps + h0 + k) * D + d0;
                   if constexpr (CPL == 4) {
                     uint2 u;
                     u.x = ptx::pack_bf16x2(acc[k][0] * inv, acc[k][1] * inv);
@@ -686,23 +731,29 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
   int nrows_seg = 0;  // valid heads of the segment
   int nrows_c = 0;    // valid heads of this consumer's tile
   int hoff_c = 0;     // first segment-relative head of this consumer's tile
+  int cdrop[NT][2];   // MQ: query tokens newer than each column's own
+  const int max_drop = MQ ? p.q_len - 1 : 0;
   const float sl2 = p.scale_log2;
 
   auto load_q = [&](int b, int seg, int stage) {
     const int kvh = seg / p.n_ht;
     const int ht = seg % p.n_ht;
-    nrows_seg = min(p.heads_per_seg, p.group - ht * p.heads_per_seg);
+    nrows_seg = min(p.heads_per_seg, grp - ht * p.heads_per_seg);
     hoff_c = SPLIT_HEADS ? j * NH : 0;
     nrows_c = max(0, min(NH, nrows_seg - hoff_c));
-    const int head0 = kvh * p.group + ht * p.heads_per_seg + hoff_c;
+    const int r0 = ht * p.heads_per_seg + hoff_c;  // first row of this consumer's tile
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e)
+        cdrop[nt][e] = MQ ? max_drop - (r0 + nt * 8 + 2 * q + e) / p.group : 0;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const int h = nt * 8 + g;
       const bool v = h < nrows_c;
       // token split: from the rows staged with the piece's first block; else from HBM/L2
       const uint32_t* qrow =
-          SPLIT_HEADS ? reinterpret_cast<const uint32_t*>(
-                            p.q + (static_cast<int64_t>(b) * p.num_heads + head0 + (v ? h : 0)) * D)
+          SPLIT_HEADS ? reinterpret_cast<const uint32_t*>(p.q + seq_row(b, kvh, r0 + (v ? h : 0)) * D)
                       : reinterpret_cast<const uint32_t*>(qbuf + stage * kQBytes) + (v ? h : 0) * (D / 2);
 #pragma unroll
       for (int ks = 0; ks < MT; ++ks) {
@@ -737,7 +788,6 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int hps = p.heads_per_seg;
     const int kvh = si.seg / p.n_ht;
     const int ht = si.seg % p.n_ht;
-    const int64_t row0 = static_cast<int64_t>(si.b) * p.num_heads + kvh * p.group + ht * hps;
     // Outputs in batches of 8 per thread; for each piece the 8 (max, sum) pairs and 8
     // partial values are loaded together, so a piece costs one L2 round trip per batch.
     const int total_out = nrows_seg * D;
@@ -780,7 +830,7 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
 #pragma unroll
       for (int k = 0; k < 8; ++k)
         if (act[k])
-          reinterpret_cast<__nv_bfloat16*>(p.out)[row0 * D + off_o[k]] =
+          reinterpret_cast<__nv_bfloat16*>(p.out)[seq_row(si.b, kvh, ht * hps + off_o[k] / D) * D + off_o[k] % D] =
               __float2bfloat16_rn(L[k] > 0.f ? acc[k] / L[k] : 0.f);
     }
     if (tid == 0) p.counters[segid] = 0;
@@ -803,16 +853,18 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
         for (int sc = 0; sc < kSubChunks; ++sc) {
           if ((si.submask >> sc) & 1) {
             const uint32_t kb = kst + sc * G_::kSubBytes;
-            attend_subchunk<D, NT>(kb, kb + G_::kTileBytes, min(kChunk, si.nvalid - sc * kChunk),
-                                   kofs, vofs, qf, o, mref, lsum, sl2, g, q);
+            attend_subchunk<D, NT, MQ>(kb, kb + G_::kTileBytes, min(kChunk, si.nvalid - sc * kChunk),
+                                       kofs, vofs, qf, o, mref, lsum, sl2, g, q, si.rem - sc * kChunk,
+                                       max_drop, cdrop);
           }
         }
       }
     } else {
       if ((si.submask >> j) & 1) {
         const uint32_t kb = kst + j * G_::kSubBytes;
-        attend_subchunk<D, NT>(kb, kb + G_::kTileBytes, min(kChunk, si.nvalid - j * kChunk),
-                               kofs, vofs, qf, o, mref, lsum, sl2, g, q);
+        attend_subchunk<D, NT, MQ>(kb, kb + G_::kTileBytes, min(kChunk, si.nvalid - j * kChunk),
+                                   kofs, vofs, qf, o, mref, lsum, sl2, g, q, si.rem - j * kChunk, max_drop,
+                                   cdrop);
       }
     }
     const bool piece_end = si.flags & kLastOfPiece;
@@ -839,7 +891,6 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int hps = p.heads_per_seg;
     const int kvh = si.seg / p.n_ht;
     const int ht = si.seg % p.n_ht;
-    const int64_t row0 = static_cast<int64_t>(si.b) * p.num_heads + kvh * p.group + ht * hps;
     const int slot = static_cast<int>(w * 2 + ((si.flags & kFirstPieceOfCta) ? 0 : 1));
 
     if constexpr (SPLIT_HEADS) {
@@ -853,7 +904,7 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
             const int hs = hoff_c + h;         // within the segment
             if (sole) {
               const float inv = lt[nt][e] > 0.f ? 1.f / lt[nt][e] : 0.f;
-              __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + (row0 + hs) * D;
+              __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + seq_row(si.b, kvh, ht * hps + hs) * D;
 #pragma unroll
               for (int mt = 0; mt < MT; ++mt) {
                 dst[mt * 16 + g] = __float2bfloat16_rn(o[mt][nt][e] * inv);
@@ -928,11 +979,11 @@ struct Cfg {
                                   kStages * (sizeof(StageInfo) + 24);
 };
 
-template <int D, int NT, bool SH, int C>
+template <int D, int NT, bool SH, int C, bool MQ>
 cudaError_t launch_t(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int grid,
                      cudaStream_t stream, bool overlap) {
   using CF = Cfg<D, NT, SH, C>;
-  auto kern = decode_ws_kernel<D, NT, SH, C, CF::kStages>;
+  auto kern = decode_ws_kernel<D, NT, SH, C, CF::kStages, MQ>;
   static thread_local int configured_device = -1;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -960,15 +1011,15 @@ cudaError_t launch_t(const DecodeParams& p, const CUtensorMap& tk, const CUtenso
   return cudaLaunchKernelEx(&cfg, kern, tk, tv, p);
 }
 
-template <int D>
+template <int D, bool MQ>
 cudaError_t launch_d(const DecodeParams& p, const DecodePlan& pl, const CUtensorMap& tk,
                      const CUtensorMap& tv, int grid, cudaStream_t s, bool o) {
   if (!pl.split_heads)
-    return pl.n_tiles == 1 ? launch_t<D, 1, false, 4>(p, tk, tv, grid, s, o)
-                           : launch_t<D, 2, false, 4>(p, tk, tv, grid, s, o);
+    return pl.n_tiles == 1 ? launch_t<D, 1, false, 4, MQ>(p, tk, tv, grid, s, o)
+                           : launch_t<D, 2, false, 4, MQ>(p, tk, tv, grid, s, o);
   // Head split (17..32 heads per kv head): one 8-head n-tile per consumer.
-  return pl.consumers == 3 ? launch_t<D, 1, true, 3>(p, tk, tv, grid, s, o)
-                           : launch_t<D, 1, true, 4>(p, tk, tv, grid, s, o);
+  return pl.consumers == 3 ? launch_t<D, 1, true, 3, MQ>(p, tk, tv, grid, s, o)
+                           : launch_t<D, 1, true, 4, MQ>(p, tk, tv, grid, s, o);
 }
 
 template <int D, int NT, bool SH, int C>
@@ -1025,8 +1076,11 @@ DecodePlan plan_decode(int head_dim, int group) {
 
 cudaError_t launch_decode(const DecodeParams& p, const DecodePlan& pl, const CUtensorMap& tk,
                           const CUtensorMap& tv, int grid, cudaStream_t stream, bool overlap) {
-  if (p.head_dim == 64) return launch_d<64>(p, pl, tk, tv, grid, stream, overlap);
-  return launch_d<128>(p, pl, tk, tv, grid, stream, overlap);
+  if (p.q_len > 1)
+    return p.head_dim == 64 ? launch_d<64, true>(p, pl, tk, tv, grid, stream, overlap)
+                            : launch_d<128, true>(p, pl, tk, tv, grid, stream, overlap);
+  if (p.head_dim == 64) return launch_d<64, false>(p, pl, tk, tv, grid, stream, overlap);
+  return launch_d<128, false>(p, pl, tk, tv, grid, stream, overlap);
 }
 
 }  // namespace gqa

@@ -256,9 +256,10 @@ gqa_status decode_impl(const void* q, const void* k_pages, const void* v_pages,
                        const int32_t* block_table, const int32_t* seq_lens, void* out,
                        int num_seqs, int num_heads, int num_kv_heads, int head_dim, int page_size,
                        float scale, int max_blocks_per_seq, int num_pages, void* stream,
-                       bool overlap_previous) {
+                       bool overlap_previous, int q_len = 1) {
   if (num_seqs < 0) return fail(GQA_ERR_INVALID_ARG, "num_seqs < 0");
   if (num_seqs > 65536) return fail(GQA_ERR_UNSUPPORTED, "num_seqs > 65536");
+  if (q_len < 1) return fail(GQA_ERR_INVALID_ARG, "q_len %d < 1", q_len);
   if (num_heads < 1 || num_kv_heads < 1 || head_dim < 1 || page_size < 1 ||
       max_blocks_per_seq < 1 || num_pages < 1)
     return fail(GQA_ERR_INVALID_ARG, "sizes must be positive");
@@ -275,6 +276,11 @@ gqa_status decode_impl(const void* q, const void* k_pages, const void* v_pages,
     return fail(GQA_ERR_UNSUPPORTED, "num_pages * num_kv_heads * page_size exceeds 2^31");
   if (static_cast<int64_t>(max_blocks_per_seq) * page_size >= (int64_t{1} << 31))
     return fail(GQA_ERR_UNSUPPORTED, "max_blocks_per_seq * page_size exceeds 2^31");
+  // Several query tokens: each kv head's rows are its group for every token, read with
+  // one pass over its K/V (the mma.sync kernel, up to 32 rows per kv head).
+  if (q_len > 1 && static_cast<int64_t>(num_heads / num_kv_heads) * q_len > 32)
+    return fail(GQA_ERR_UNSUPPORTED, "q_len %d x %d query heads per kv head exceeds 32", q_len,
+                num_heads / num_kv_heads);
   if (num_seqs == 0) return GQA_OK;
   if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !out)
     return fail(GQA_ERR_INVALID_ARG, "null pointer argument");
@@ -290,7 +296,7 @@ gqa_status decode_impl(const void* q, const void* k_pages, const void* v_pages,
   cudaStream_t strm = static_cast<cudaStream_t>(stream);
 
   const int group = num_heads / num_kv_heads;
-  const gqa::DecodePlan plan = gqa::plan_decode(head_dim, group);
+  const gqa::DecodePlan plan = gqa::plan_decode(head_dim, group * q_len);
   // Upper bound on the block count (seq_lens are device data).
   const int64_t blocks_per_seq =
       (static_cast<int64_t>(max_blocks_per_seq) * page_size + gqa::kBlock - 1) / gqa::kBlock;
@@ -332,11 +338,57 @@ gqa_status decode_impl(const void* q, const void* k_pages, const void* v_pages,
   p.num_workers = static_cast<int>(workers);
   p.wait_limit_ns = static_cast<uint64_t>(g_wait_limit_ns.load());
   p.arm_without_copy = g_arm_without_copy.load();
+  p.q_len = q_len;
   cudaError_t e = launch_with_maps(p, plan, q, k_pages, v_pages, rows, dev, grid, strm,
                                    overlap_previous, &s);
   if (s != GQA_OK) return s;
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   g_launches.fetch_add(plan.tensor_cores && grid > 1 ? 2 : 1);
+  return GQA_OK;
+}
+
+}  // namespace
+
+namespace {
+
+gqa_status append_impl(const void* k_new, const void* v_new, void* k_pages, void* v_pages,
+                       const int32_t* block_table, const int32_t* positions, int num_seqs, int q_len,
+                       int num_kv_heads, int head_dim, int page_size, int max_blocks_per_seq,
+                       int num_pages, void* stream) {
+  if (q_len < 1) return fail(GQA_ERR_INVALID_ARG, "q_len %d < 1", q_len);
+  if (num_seqs < 0) return fail(GQA_ERR_INVALID_ARG, "num_seqs < 0");
+  if (num_kv_heads < 1 || head_dim < 1 || page_size < 1 || max_blocks_per_seq < 1 || num_pages < 1)
+    return fail(GQA_ERR_INVALID_ARG, "sizes must be positive");
+  if (head_dim % 8 != 0) return fail(GQA_ERR_UNSUPPORTED, "head_dim must be a multiple of 8");
+  if (static_cast<int64_t>(max_blocks_per_seq) * page_size > INT32_MAX)
+    return fail(GQA_ERR_UNSUPPORTED, "max_blocks_per_seq * page_size exceeds 2^31");
+  if (num_seqs == 0) return GQA_OK;
+  if (!k_new || !v_new || !k_pages || !v_pages || !block_table || !positions)
+    return fail(GQA_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_pages, 16) || !aligned(v_pages, 16))
+    return fail(GQA_ERR_INVALID_ARG, "bf16 tensors must be 16-byte aligned");
+  DeviceState* st;
+  int dev;
+  gqa_status s = get_state(&st, &dev);
+  if (s != GQA_OK) return s;
+  gqa::AppendParams p;
+  p.k_new = static_cast<const uint4*>(k_new);
+  p.v_new = static_cast<const uint4*>(v_new);
+  p.k_pages = static_cast<uint4*>(k_pages);
+  p.v_pages = static_cast<uint4*>(v_pages);
+  p.block_table = block_table;
+  p.positions = positions;
+  p.err = st->err;
+  p.num_seqs = num_seqs;
+  p.num_kv_heads = num_kv_heads;
+  p.vec_per_row = head_dim / 8;
+  p.page_size = page_size;
+  p.max_blocks = max_blocks_per_seq;
+  p.num_pages = num_pages;
+  p.q_len = q_len;
+  cudaError_t e = gqa::launch_kv_append(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "kv_append launch");
+  g_launches.fetch_add(1);
   return GQA_OK;
 }
 
@@ -373,39 +425,16 @@ gqa_status gqa_kv_append(const void* k_new, const void* v_new, void* k_pages, vo
                          const int32_t* block_table, const int32_t* positions, int num_seqs,
                          int num_kv_heads, int head_dim, int page_size, int max_blocks_per_seq,
                          int num_pages, void* stream) {
-  if (num_seqs < 0) return fail(GQA_ERR_INVALID_ARG, "num_seqs < 0");
-  if (num_kv_heads < 1 || head_dim < 1 || page_size < 1 || max_blocks_per_seq < 1 || num_pages < 1)
-    return fail(GQA_ERR_INVALID_ARG, "sizes must be positive");
-  if (head_dim % 8 != 0) return fail(GQA_ERR_UNSUPPORTED, "head_dim must be a multiple of 8");
-  if (static_cast<int64_t>(max_blocks_per_seq) * page_size > INT32_MAX)
-    return fail(GQA_ERR_UNSUPPORTED, "max_blocks_per_seq * page_size exceeds 2^31");
-  if (num_seqs == 0) return GQA_OK;
-  if (!k_new || !v_new || !k_pages || !v_pages || !block_table || !positions)
-    return fail(GQA_ERR_INVALID_ARG, "null pointer argument");
-  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_pages, 16) || !aligned(v_pages, 16))
-    return fail(GQA_ERR_INVALID_ARG, "bf16 tensors must be 16-byte aligned");
-  DeviceState* st;
-  int dev;
-  gqa_status s = get_state(&st, &dev);
-  if (s != GQA_OK) return s;
-  gqa::AppendParams p;
-  p.k_new = static_cast<const uint4*>(k_new);
-  p.v_new = static_cast<const uint4*>(v_new);
-  p.k_pages = static_cast<uint4*>(k_pages);
-  p.v_pages = static_cast<uint4*>(v_pages);
-  p.block_table = block_table;
-  p.positions = positions;
-  p.err = st->err;
-  p.num_seqs = num_seqs;
-  p.num_kv_heads = num_kv_heads;
-  p.vec_per_row = head_dim / 8;
-  p.page_size = page_size;
-  p.max_blocks = max_blocks_per_seq;
-  p.num_pages = num_pages;
-  cudaError_t e = gqa::launch_kv_append(p, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "kv_append launch");
-  g_launches.fetch_add(1);
-  return GQA_OK;
+  return append_impl(k_new, v_new, k_pages, v_pages, block_table, positions, num_seqs, 1, num_kv_heads,
+                     head_dim, page_size, max_blocks_per_seq, num_pages, stream);
+}
+
+gqa_status gqa_kv_append_multi(const void* k_new, const void* v_new, void* k_pages, void* v_pages,
+                               const int32_t* block_table, const int32_t* positions, int num_seqs,
+                               int q_len, int num_kv_heads, int head_dim, int page_size,
+                               int max_blocks_per_seq, int num_pages, void* stream) {
+  return append_impl(k_new, v_new, k_pages, v_pages, block_table, positions, num_seqs, q_len,
+                     num_kv_heads, head_dim, page_size, max_blocks_per_seq, num_pages, stream);
 }
 
 gqa_status gqa_paged_decode_attn(const void* q, const void* k_pages, const void* v_pages,
@@ -432,6 +461,34 @@ gqa_status gqa_decode_step(const void* q, const void* k_new, const void* v_new, 
   return decode_impl(q, k_pages, v_pages, block_table, seq_lens, out, num_seqs, num_heads,
                      num_kv_heads, head_dim, page_size, scale, max_blocks_per_seq, num_pages,
                      stream, true);
+}
+
+gqa_status gqa_paged_multi_query_attn(const void* q, const void* k_pages, const void* v_pages,
+                                      const int32_t* block_table, const int32_t* seq_lens, void* out,
+                                      int num_seqs, int q_len, int num_heads, int num_kv_heads,
+                                      int head_dim, int page_size, float scale, int max_blocks_per_seq,
+                                      int num_pages, void* stream) {
+  return decode_impl(q, k_pages, v_pages, block_table, seq_lens, out, num_seqs, num_heads,
+                     num_kv_heads, head_dim, page_size, scale, max_blocks_per_seq, num_pages,
+                     stream, false, q_len);
+}
+
+gqa_status gqa_multi_query_step(const void* q, const void* k_new, const void* v_new, void* k_pages,
+                                void* v_pages, const int32_t* block_table, const int32_t* positions,
+                                const int32_t* seq_lens, void* out, int num_seqs, int q_len,
+                                int num_heads, int num_kv_heads, int head_dim, int page_size,
+                                float scale, int max_blocks_per_seq, int num_pages, void* stream) {
+  if (q_len < 1) return fail(GQA_ERR_INVALID_ARG, "q_len %d < 1", q_len);
+  if (num_kv_heads >= 1 && num_heads % num_kv_heads == 0 &&
+      static_cast<int64_t>(num_heads / num_kv_heads) * q_len > 32 && q_len > 1)
+    return fail(GQA_ERR_UNSUPPORTED, "q_len %d x %d query heads per kv head exceeds 32", q_len,
+                num_heads / num_kv_heads);
+  gqa_status s = append_impl(k_new, v_new, k_pages, v_pages, block_table, positions, num_seqs, q_len,
+                             num_kv_heads, head_dim, page_size, max_blocks_per_seq, num_pages, stream);
+  if (s != GQA_OK) return s;
+  return decode_impl(q, k_pages, v_pages, block_table, seq_lens, out, num_seqs, num_heads,
+                     num_kv_heads, head_dim, page_size, scale, max_blocks_per_seq, num_pages,
+                     stream, true, q_len);
 }
 
 gqa_status gqa_paged_decode_attn_noalloc(const void* q, const void* k_pages, const void* v_pages,
@@ -533,6 +590,7 @@ gqa_status gqa_paged_decode_attn_noalloc(const void* q, const void* k_pages, con
   p.num_workers = static_cast<int>(workers);
   p.wait_limit_ns = static_cast<uint64_t>(g_wait_limit_ns.load());
   p.arm_without_copy = g_arm_without_copy.load();
+  p.q_len = 1;
   e = launch_with_maps(p, plan, q, k_pages, v_pages, rows, dev, static_cast<int>(workers), strm,
                        false, &s);
   if (s != GQA_OK) return s;

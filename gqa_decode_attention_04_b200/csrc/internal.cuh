@@ -52,6 +52,7 @@ struct DecodeParams {
   int num_workers;            // CTAs the work list is split over
   uint64_t wait_limit_ns;
   int arm_without_copy;
+  int q_len;                  // query tokens per sequence (q, out: [B, q_len, H, D]); 1 = decode
 };
 
 struct AppendParams {
@@ -63,6 +64,7 @@ struct AppendParams {
   const int32_t* positions;
   uint32_t* err;
   int num_seqs, num_kv_heads, vec_per_row, page_size, max_blocks, num_pages;
+  int q_len;                  // rows per sequence: k_new [B, q_len, Hk, D] to positions[b] + i
 };
 
 // Launchers (return the cudaError_t of the launch).

@@ -143,6 +143,41 @@ gqa_status gqa_decode_step(const void* q, const void* k_new, const void* v_new, 
                            int max_blocks_per_seq, int num_pages, void* stream);
 
 /*
+ * Several query tokens per sequence (speculative verification, chunked prefill over the
+ * cache).  The MQA plugin's entry point on the TensorRT MQA page carries a query length
+ * (seq_q) beside the KV length; here the q_len query tokens of sequence b are its q_len
+ * newest tokens, at positions seq_lens[b] - q_len .. seq_lens[b] - 1, and query token i
+ * attends to positions 0 .. seq_lens[b] - q_len + i: itself and everything before it,
+ * as one decode step per token would.  A token whose window is empty (seq_lens[b] <
+ * q_len - i) gets zeros.  q_len = 1 is gqa_paged_decode_attn.
+ *
+ * gqa_kv_append_multi -- q_len new rows per sequence: k_new, v_new [num_seqs, q_len,
+ *   num_kv_heads, head_dim]; row i of sequence b goes to position positions[b] + i (all
+ *   of them inside max_blocks_per_seq * page_size, else that sequence's rows are skipped
+ *   and reported as GQA_ERR_DEVICE_BOUNDS).  Otherwise as gqa_kv_append.
+ * gqa_paged_multi_query_attn -- q, out [num_seqs, q_len, num_heads, head_dim] bf16; the
+ *   other arguments, layouts, requirements and errors as gqa_paged_decode_attn.  Each kv
+ *   head's K/V are read once for all q_len x (num_heads / num_kv_heads) query rows; that
+ *   product must be <= 32 when q_len > 1 (GQA_ERR_UNSUPPORTED otherwise).
+ * gqa_multi_query_step -- gqa_kv_append_multi, then gqa_paged_multi_query_attn, as
+ *   gqa_decode_step does for one token (the attention launch overlaps the append).
+ */
+gqa_status gqa_kv_append_multi(const void* k_new, const void* v_new, void* k_pages, void* v_pages,
+                               const int32_t* block_table, const int32_t* positions, int num_seqs,
+                               int q_len, int num_kv_heads, int head_dim, int page_size,
+                               int max_blocks_per_seq, int num_pages, void* stream);
+gqa_status gqa_paged_multi_query_attn(const void* q, const void* k_pages, const void* v_pages,
+                                      const int32_t* block_table, const int32_t* seq_lens, void* out,
+                                      int num_seqs, int q_len, int num_heads, int num_kv_heads,
+                                      int head_dim, int page_size, float scale, int max_blocks_per_seq,
+                                      int num_pages, void* stream);
+gqa_status gqa_multi_query_step(const void* q, const void* k_new, const void* v_new, void* k_pages,
+                                void* v_pages, const int32_t* block_table, const int32_t* positions,
+                                const int32_t* seq_lens, void* out, int num_seqs, int q_len,
+                                int num_heads, int num_kv_heads, int head_dim, int page_size,
+                                float scale, int max_blocks_per_seq, int num_pages, void* stream);
+
+/*
  * gqa_paged_decode_attn_noalloc -- the same decode attention as gqa_paged_decode_attn
  * (same arguments, layouts and result), for callers that cannot allocate device memory:
  * an engine that has already reserved nearly all of the GPU for its own caching

@@ -101,3 +101,27 @@ def test_binding_refuses_cpu_tensors():
     sl = torch.ones(1, dtype=torch.int32)
     with pytest.raises(ValueError, match="CUDA"):
         gq.paged_decode_attn(q, kp, kp, bt, sl)
+
+
+def _multi(lib, B=2, Q=2, H=4, Hk=1, D=64, ps=16, MB=4, P=8, ptr=1 << 20):
+    p = ctypes.c_void_p(ptr)
+    return lib.gqa_paged_multi_query_attn(p, p, p, p, p, p, B, Q, H, Hk, D, ps, ctypes.c_float(0.125),
+                                          MB, P, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(Q=0), -1),                # no query token
+    (dict(Q=9, H=4, Hk=1), -2),     # 9 x 4 rows per kv head > 32
+    (dict(Q=3, H=24, Hk=2), -2),    # 3 x 12 > 32
+    (dict(B=0, Q=8, H=4, Hk=1), 0), # 32 rows: accepted, nothing to do
+])
+def test_multi_query_host_validation(lib, kw, status):
+    assert _multi(lib, **kw) == status
+    if status != 0:
+        assert len(lib.gqa_last_error_string()) > 0
+
+
+def test_kv_append_multi_host_validation(lib):
+    p = ctypes.c_void_p(1 << 20)
+    assert lib.gqa_kv_append_multi(p, p, p, p, p, p, 2, 0, 1, 64, 16, 4, 8, None) == -1
+    assert lib.gqa_kv_append_multi(p, p, p, p, p, p, 0, 3, 1, 64, 16, 4, 8, None) == 0

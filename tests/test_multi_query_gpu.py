@@ -1,0 +1,142 @@
+"""Several query tokens per sequence on the GPU (gqa_paged_multi_query_attn,
+gqa_kv_append_multi, gqa_multi_query_step) against the oracle: query token i of sequence
+b attends to positions 0 .. seq_lens[b] - q_len + i.  Cases cover every kernel shape the
+q_len x group rows select (8-, 16-row token split; 24-, 32-row head split), both head
+dims, page sizes 16..64, windows that end inside a sub-chunk, a block or a page, empty
+windows (seq_len < q_len), forced split counts (pieces merged across CTAs) and poisoned
+unused slots."""
+import numpy as np
+import pytest
+import torch
+
+import gqa_decode_attention_04_b200 as gq
+import oracle
+from parity import assert_close, gpu_f64
+from workloads import bf16_bits, make_custom_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def _case(lens, Q, H, Hk, D, ps, seed):
+    inp = make_custom_inputs(lens, H, Hk, D, ps, seed=seed, extra_pages=2)
+    gen = torch.Generator().manual_seed(seed + 99)
+    q = torch.randn(len(lens), Q, H, D, generator=gen).to(torch.bfloat16)
+    return inp, q
+
+
+def _oracle(inp, q):
+    return oracle.paged_multi_query_attention(bf16_bits(q), bf16_bits(inp.k_pages), bf16_bits(inp.v_pages),
+                                              inp.block_table.numpy(), inp.seq_lens.numpy(), inp.scale)
+
+
+CASES = [
+    # lens, q_len, H, Hk, D, ps           rows per kv head
+    ([5, 37, 64, 130, 1, 16], 4, 8, 2, 128, 16),    # 16: token split, two n-tiles
+    ([200, 17, 3, 66], 2, 4, 1, 64, 16),            # 8: token split, one n-tile, D = 64
+    ([300, 65, 48, 7], 8, 4, 1, 128, 32),           # 32: head split, 4 consumers
+    ([150, 90, 2], 3, 24, 4, 128, 16),              # 18: head split, 3 consumers
+    ([1000, 20], 2, 16, 1, 128, 64),                # 32, page size 64
+    ([77, 300, 4], 5, 4, 4, 128, 16),               # MHA: 5 rows
+    ([129, 63, 64, 65], 7, 4, 1, 64, 16),           # windows ending around block edges
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: f"L{len(c[0])}_Q{c[1]}_H{c[2]}_Hk{c[3]}_D{c[4]}_ps{c[5]}")
+def test_multi_query_parity(cuda_device, case):
+    lens, Q, H, Hk, D, ps = case
+    inp, q = _case(lens, Q, H, Hk, D, ps, seed=len(lens) * 31 + Q)
+    d = inp.to(cuda_device)
+    out = gq.paged_multi_query_attn(q.to(cuda_device), d.k_pages, d.v_pages, d.block_table, d.seq_lens,
+                                    scale=inp.scale)
+    gq.check_device_error()
+    assert_close(gpu_f64(out), _oracle(inp, q), what=str(case))
+
+
+@pytest.mark.parametrize("workers", [1, 3, 57, 400])
+def test_multi_query_forced_splits(cuda_device, workers):
+    lens, Q, H, Hk, D, ps = [900, 333, 64, 2], 4, 8, 2, 128, 16
+    inp, q = _case(lens, Q, H, Hk, D, ps, seed=5)
+    d = inp.to(cuda_device)
+    try:
+        gq.set_num_workers(workers)
+        out = gq.paged_multi_query_attn(q.to(cuda_device), d.k_pages, d.v_pages, d.block_table, d.seq_lens,
+                                        scale=inp.scale)
+        gq.check_device_error()
+    finally:
+        gq.set_num_workers(0)
+    assert_close(gpu_f64(out), _oracle(inp, q), what=f"workers={workers}")
+
+
+def test_single_query_token_equals_the_decode(cuda_device):
+    inp, q = _case([40, 700, 3], 1, 8, 2, 128, 16, seed=9)
+    d = inp.to(cuda_device)
+    a = gq.paged_multi_query_attn(q.to(cuda_device), d.k_pages, d.v_pages, d.block_table, d.seq_lens,
+                                  scale=inp.scale)
+    b = gq.paged_decode_attn(q[:, 0].contiguous().to(cuda_device), d.k_pages, d.v_pages, d.block_table,
+                             d.seq_lens, scale=inp.scale)
+    gq.check_device_error()
+    assert torch.equal(a[:, 0], b)
+
+
+def test_newest_token_equals_a_decode_over_the_whole_sequence(cuda_device):
+    """The last query token sees every token: the same numbers as a one-token decode
+    within the tolerance, and the first sees q_len - 1 fewer."""
+    Q = 4
+    inp, q = _case([90, 513, 16], Q, 8, 2, 128, 16, seed=12)
+    d = inp.to(cuda_device)
+    out = gq.paged_multi_query_attn(q.to(cuda_device), d.k_pages, d.v_pages, d.block_table, d.seq_lens,
+                                    scale=inp.scale)
+    last = gq.paged_decode_attn(q[:, Q - 1].contiguous().to(cuda_device), d.k_pages, d.v_pages,
+                                d.block_table, d.seq_lens, scale=inp.scale)
+    first = gq.paged_decode_attn(q[:, 0].contiguous().to(cuda_device), d.k_pages, d.v_pages, d.block_table,
+                                 (d.seq_lens - (Q - 1)).contiguous(), scale=inp.scale)
+    gq.check_device_error()
+    assert_close(gpu_f64(out[:, Q - 1]), gpu_f64(last), max_abs=1e-2, mean_abs=1e-3, what="newest")
+    assert_close(gpu_f64(out[:, 0]), gpu_f64(first), max_abs=1e-2, mean_abs=1e-3, what="oldest")
+
+
+def test_kv_append_multi_is_bit_exact(cuda_device):
+    Q = 3
+    inp = make_custom_inputs([20, 6, 33], 4, 2, 128, 16, seed=14, extra_pages=3)
+    gen = torch.Generator().manual_seed(15)
+    kn = torch.randn(3, Q, 2, 128, generator=gen).to(torch.bfloat16)
+    vn = torch.randn(3, Q, 2, 128, generator=gen).to(torch.bfloat16)
+    pos = (inp.seq_lens - Q).to(torch.int32)
+    d = inp.to(cuda_device)
+    gq.kv_append_multi(kn.to(cuda_device), vn.to(cuda_device), d.k_pages, d.v_pages, d.block_table,
+                       pos.to(cuda_device))
+    gq.check_device_error()
+    k2, v2 = oracle.kv_append_multi(bf16_bits(inp.k_pages), bf16_bits(inp.v_pages), bf16_bits(kn),
+                                    bf16_bits(vn), inp.block_table.numpy(), pos.numpy())
+    assert np.array_equal(bf16_bits(d.k_pages), k2) and np.array_equal(bf16_bits(d.v_pages), v2)
+
+
+@pytest.mark.parametrize("Q,H,Hk", [(4, 8, 2), (8, 4, 1), (2, 32, 2)])
+def test_multi_query_step_equals_append_then_attend(cuda_device, Q, H, Hk):
+    lens = [70, 300, 5, 129]
+    inp = make_custom_inputs(lens, H, Hk, 128, 16, seed=17 + Q, extra_pages=2)
+    gen = torch.Generator().manual_seed(18 + Q)
+    B = len(lens)
+    q = torch.randn(B, Q, H, 128, generator=gen).to(torch.bfloat16)
+    kn = torch.randn(B, Q, Hk, 128, generator=gen).to(torch.bfloat16)
+    vn = torch.randn(B, Q, Hk, 128, generator=gen).to(torch.bfloat16)
+    pos = (inp.seq_lens - Q).clamp(min=0).to(torch.int32)
+    d = inp.to(cuda_device)
+    out = gq.multi_query_step(q.to(cuda_device), kn.to(cuda_device), vn.to(cuda_device), d.k_pages,
+                              d.v_pages, d.block_table, pos.to(cuda_device), d.seq_lens, scale=inp.scale)
+    gq.check_device_error()
+    k2, v2 = oracle.kv_append_multi(bf16_bits(inp.k_pages), bf16_bits(inp.v_pages), bf16_bits(kn),
+                                    bf16_bits(vn), inp.block_table.numpy(), pos.numpy())
+    assert np.array_equal(bf16_bits(d.k_pages), k2) and np.array_equal(bf16_bits(d.v_pages), v2)
+    want = oracle.paged_multi_query_attention(bf16_bits(q), k2, v2, inp.block_table.numpy(),
+                                              inp.seq_lens.numpy(), inp.scale)
+    assert_close(gpu_f64(out), want, what=f"Q={Q} H={H} Hk={Hk}")
+
+
+def test_too_many_rows_is_refused_and_launches_nothing(cuda_device):
+    inp, q = _case([40], 9, 4, 1, 128, 16, seed=3)
+    d = inp.to(cuda_device)
+    n0 = gq.launch_count()
+    with pytest.raises(gq.GQAError) as e:
+        gq.paged_multi_query_attn(q.to(cuda_device), d.k_pages, d.v_pages, d.block_table, d.seq_lens)
+    assert e.value.status == -2 and gq.launch_count() == n0
