@@ -48,8 +48,8 @@ KERNEL_SOURCES = {
 
 def decode_kernel_for(inp) -> str:
     """The decode kernel the library picks for this head grouping: the tcgen05 kernel
-    for more than 32 query heads per kv head, the mma.sync kernel otherwise."""
-    return "decode_tc_kernel" if inp.num_heads // inp.num_kv_heads > 32 else "decode_ws_kernel"
+    for more than 16 query heads per kv head, the mma.sync kernel otherwise."""
+    return "decode_tc_kernel" if inp.num_heads // inp.num_kv_heads > 16 else "decode_ws_kernel"
 
 
 # ------------------------------------------------------------------ helpers

@@ -27,8 +27,9 @@
 //       - small groups (G <= 16): each of the 4 consumers takes one 16-token sub-chunk
 //         of every stage for all G heads; at a piece end their partial softmax states
 //         are combined in shared memory.
-//       - groups of 17..32: each consumer takes 8 of the query heads over all 64
-//         tokens of every stage (larger groups run on the tcgen05 kernel, decode_tc.cu).
+//       - 17..32 rows (several query tokens' heads of one kv head): each consumer takes
+//         8 of the rows over all 64 tokens of every stage.  Single-token groups of more
+//         than 16 heads run on the tcgen05 kernel (decode_tc.cu).
 //   * Online softmax in the log2 domain with a lazily moved reference: O and the sum are
 //     rescaled only when a head's running maximum rises by more than 8 (factor 256);
 //     numerator and denominator share the reference, so the result is unchanged.
@@ -1032,11 +1033,14 @@ void fill(DecodePlan& pl) {
 }  // namespace
 
 // Small groups (G <= 16): token split, 4 consumers, one 8- or 16-head tile per segment.
-// 17..32: head split, 8 heads per consumer, 3 or 4 consumers.  Larger groups run on the
-// tcgen05 kernel (decode_tc.cu), one 128-row MMA tile of heads per segment.
-DecodePlan plan_decode(int head_dim, int group) {
+// Larger groups run on the tcgen05 kernel (decode_tc.cu), one 128-row MMA tile of heads
+// per segment: from 17 heads on its per-block cost (fixed by the 128-row tile) is below
+// the mma.sync kernel's, whose work grows with the heads (measured: 24 and 32 heads per
+// kv head, 29-49 us against 46-73 us).  Rows of several query tokens per sequence
+// (mq_rows) stay on the mma.sync kernel, whose head split covers 17..32 rows.
+DecodePlan plan_decode(int head_dim, int group, bool mq_rows) {
   DecodePlan pl{};
-  if (group > 32) {
+  if (group > 16 && !mq_rows) {
     // Dense enough for the 5th-generation tensor cores: one 128-row MMA tile of heads.
     pl.tensor_cores = 1;
     pl.split_heads = 1;

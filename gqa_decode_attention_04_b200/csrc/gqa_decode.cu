@@ -296,7 +296,7 @@ gqa_status decode_impl(const void* q, const void* k_pages, const void* v_pages,
   cudaStream_t strm = static_cast<cudaStream_t>(stream);
 
   const int group = num_heads / num_kv_heads;
-  const gqa::DecodePlan plan = gqa::plan_decode(head_dim, group * q_len);
+  const gqa::DecodePlan plan = gqa::plan_decode(head_dim, group * q_len, q_len > 1);
   // Upper bound on the block count (seq_lens are device data).
   const int64_t blocks_per_seq =
       (static_cast<int64_t>(max_blocks_per_seq) * page_size + gqa::kBlock - 1) / gqa::kBlock;

@@ -83,7 +83,8 @@ struct DecodePlan {
   size_t smem_bytes;
 };
 
-DecodePlan plan_decode(int head_dim, int group);
+// group: query rows per kv head; mq_rows: they are several query tokens' heads.
+DecodePlan plan_decode(int head_dim, int group, bool mq_rows = false);
 // overlap_previous: launch with programmatic stream serialization, so the prologue
 // overlaps the preceding kernel of the stream (which must write nothing the decode reads
 // except the K/V pools); the producer waits for that kernel before its first K/V copy.

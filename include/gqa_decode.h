@@ -108,7 +108,7 @@ gqa_status gqa_kv_append(const void* k_new, const void* v_new, void* k_pages, vo
  * Each kv head's K/V are read from HBM once for all of its query heads.  Long
  * contexts are split across the GPU (FlashDecoding, named on the tiny-llm page);
  * partial results are merged with their log-sum-exp: inside the same launch for
- * groups of up to 32 query heads per kv head, by a second kernel on the same stream
+ * groups of up to 16 query heads per kv head, by a second kernel on the same stream
  * (launched to overlap the first one's end) for larger groups.
  *
  *   scale           multiplier of q.k (usually 1/sqrt(head_dim)), finite.

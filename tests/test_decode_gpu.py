@@ -388,6 +388,9 @@ TC_CASES = [
     ([900, 130], 64, 1, 128, 80),             # page 80
     ([1100, 96], 40, 1, 64, 96),              # page 96 (32-row copies), head_dim 64
     ([800, 193], 72, 1, 128, 192),            # page 192: 64-row copies, three blocks per page
+    ([600, 33, 2], 17, 1, 128, 16),           # G = 17: smallest group on tcgen05
+    ([450, 129], 48, 2, 64, 32),              # G = 24, head_dim 64
+    ([1000, 64, 7], 128, 4, 128, 16),         # G = 32, four kv heads
 ]
 
 
