@@ -76,6 +76,7 @@ struct TcGeo {
 struct TcStageInfo {
   uint64_t vmask;  // bit t: token t of the block is inside the sequence and its page was loaded
   int b, seg, blk, nvalid, flags, piece;
+  int rem, pad;    // rem: tokens of the sequence from this block's first one on (unclamped)
 };
 enum : int { kTcFirst = 1, kTcLast = 2, kTcSole = 4, kTcFirstPieceOfCta = 8 };
 
@@ -89,7 +90,10 @@ struct TcCursor {
 
 }  // namespace
 
-template <int D>
+// MQ: several query tokens per sequence (p.q_len): a kv head's rows are its group of
+// heads for each query token in turn (row r: token r / group, head r % group), all in one
+// segment (at most 128 rows); row r sees the sequence up to its own token.
+template <int D, bool MQ>
 __global__ void __launch_bounds__(kTcThreads, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                  const __grid_constant__ CUtensorMap tmap_q, const DecodeParams p) {
@@ -109,6 +113,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
   const int segs = p.num_kv_heads * p.n_ht;
   const int cap = p.max_blocks * p.page_size;
   const int hps = p.heads_per_seg;
+  const int rows_per_seq = MQ ? p.num_heads * p.q_len : p.num_heads;
 
   // The split merge (the next kernel) may launch now; it waits for this grid to complete
   // before reading anything this grid writes.
@@ -120,8 +125,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
     const int Le = tc_eff_len(L, cap);
     if ((L < 0 || L > cap) && blockIdx.x == 0) atomicOr(p.err, kErrBounds);
     if (Le == 0 && (b % gridDim.x) == blockIdx.x) {
-      uint32_t* o = reinterpret_cast<uint32_t*>(p.out + static_cast<int64_t>(b) * p.num_heads * D);
-      for (int i = 0; i < p.num_heads * D / 2; ++i) o[i] = 0u;
+      uint32_t* o = reinterpret_cast<uint32_t*>(p.out + static_cast<int64_t>(b) * rows_per_seq * D);
+      for (int i = 0; i < rows_per_seq * D / 2; ++i) o[i] = 0u;
     }
     mine += static_cast<int64_t>((Le + kTcBlk - 1) / kTcBlk) * segs;
   }
@@ -335,9 +340,20 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
           break;
         }
         if (lane == 0) {
-          ptx::mbar_arrive_expect_tx(qfull_bar, p.arm_without_copy ? 1u : GE::kQTile);
-          if (!p.arm_without_copy)  // one box: 128 rows x every column group
-            ptx::tma_load_3d(qbuf, &tmap_q, qfull_bar, 0, q_row0, 0, 0);
+          if constexpr (MQ) {
+            // One box per column group: the kv head's rows (token, head) of this sequence
+            // (the 5-D map: columns, head, token, column group, sequence x kv head).
+            const uint32_t qbytes = static_cast<uint32_t>(p.group) * p.q_len * D * 2u;
+            ptx::mbar_arrive_expect_tx(qfull_bar, p.arm_without_copy ? 1u : qbytes);
+            if (!p.arm_without_copy)
+              for (int cgi = 0; cgi < GE::kGroups; ++cgi)
+                ptx::tma_load_5d(qbuf + cgi * GE::kQGroup, &tmap_q, qfull_bar, 0, 0, 0, cgi,
+                                 (cu.b * p.q_len) * p.num_kv_heads + kvh);
+          } else {
+            ptx::mbar_arrive_expect_tx(qfull_bar, p.arm_without_copy ? 1u : GE::kQTile);
+            if (!p.arm_without_copy)  // one box: 128 rows x every column group
+              ptx::tma_load_3d(qbuf, &tmap_q, qfull_bar, 0, q_row0, 0, 0);
+          }
         }
       }
       const int nvalid = min(kTcBlk, cu.len - cu.blk * kTcBlk);
@@ -360,6 +376,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
         si.seg = cu.seg;
         si.blk = cu.blk;
         si.nvalid = nvalid;
+        si.rem = cu.len - cu.blk * kTcBlk;
         si.piece = piece;
         si.flags = (first ? kTcFirst : 0) | (last ? kTcLast : 0) |
                    ((last && piece_blk0 == 0 && cu.blk + 1 == cu.nblk) ? kTcSole : 0) |
@@ -518,6 +535,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
     const bool pos = sl2 >= 0.f;  // a negative scale turns the row maximum into a minimum
     constexpr int HD = D / 2;     // output columns each warpgroup finishes at a piece end
     float mref = -INFINITY, lsum = 0.f;
+    // MQ: query tokens newer than this row's own (rows past the group's are padding).
+    const int cdrop = MQ ? (r < p.group * p.q_len ? p.q_len - 1 - r / p.group : 0) : 0;
     int wg_phase = 0;
     bool failed = false;
     // Every wait outcome is made warp-uniform: the TMEM loads and stores that follow are
@@ -572,7 +591,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
       ptx::tmem_wait_ld();
       // Scores of tokens outside the sequence (or of pages that failed the range check)
       // may be anything, NaN included: they take the raw value that scales to -inf.
-      const uint32_t vm = static_cast<uint32_t>(vmask >> (32 * g));
+      uint32_t vm = static_cast<uint32_t>(vmask >> (32 * g));
+      if constexpr (MQ) {  // this row's window ends q_len - 1 - (its token) tokens early
+        const int lim = info[stg].rem - cdrop - 32 * g;
+        if (lim < 32) vm &= lim <= 0 ? 0u : ((1u << lim) - 1u);
+      }
       const bool full = vm == 0xffffffffu;
       if (!full) {
         const uint32_t off = pos ? 0xff800000u : 0x7f800000u;  // -inf / +inf
@@ -700,7 +723,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
       const float w0 = ptx::ex2(m0 - Mu), w1 = ptx::ex2(m1 - Mu);  // 0 for an empty half
       const float ltot = s_xsum[0][r] * w0 + s_xsum[1][r] * w1;
       const int kvh = pe_seg / p.n_ht, ht = pe_seg % p.n_ht;
-      const int nrows = min(hps, p.group - ht * hps);
+      const int nrows = min(hps, (MQ ? p.group * p.q_len : p.group) - ht * hps);
       const int64_t row0 = static_cast<int64_t>(pe_b) * p.num_heads + kvh * p.group + ht * hps;
       const bool sole = flags & kTcSole;
       const int64_t slot = w * 2 + ((flags & kTcFirstPieceOfCta) ? 0 : 1);
@@ -737,7 +760,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
                 uint2 v;
                 v.x = ptx::pack_bf16x2(x.x, x.y);
                 v.y = ptx::pack_bf16x2(x.z, x.w);
-                *reinterpret_cast<uint2*>(p.out + (row0 + row) * D + col) = v;
+                const int64_t orow =
+                    MQ ? (static_cast<int64_t>(pe_b) * p.q_len + row / p.group) * p.num_heads + kvh * p.group +
+                             row % p.group
+                       : row0 + row;
+                *reinterpret_cast<uint2*>(p.out + orow * D + col) = v;
               } else {
                 *reinterpret_cast<float4*>(p.part_o + (slot * hps + row) * D + col) = x;
               }
@@ -840,8 +867,15 @@ __global__ void __launch_bounds__(kMergeThreads, 6) merge_tc_kernel(const Decode
   const int64_t slot0 = wf * 2 + (seg_base == tc_wstart(wf, T, W) ? 0 : 1);
   auto slot_of = [&](int j) -> int64_t { return j == 0 ? slot0 : (wf + j) * 2; };
   const int kvh = seg / p.n_ht, ht = seg % p.n_ht;
-  const int nrows = min(hps, p.group - ht * hps);
+  const int nrows = min(hps, p.group * p.q_len - ht * hps);
   const int64_t row0 = static_cast<int64_t>(b) * p.num_heads + kvh * p.group + ht * hps;
+  // Memory row of segment row h (several query tokens: row h is token h / group's head
+  // h % group; one segment per kv head then).
+  auto out_row = [&](int h) -> int64_t {
+    return p.q_len > 1
+               ? (static_cast<int64_t>(b) * p.q_len + h / p.group) * p.num_heads + kvh * p.group + h % p.group
+               : row0 + h;
+  };
   const int h0 = blockIdx.y * kMergeRows + warp * kMergeRowsPerWarp;
   if (h0 >= nrows) return;
 
@@ -906,7 +940,7 @@ __global__ void __launch_bounds__(kMergeThreads, 6) merge_tc_kernel(const Decode
         if (j0 + j < np) add(wj, o4[j]);
       }
     }
-    uint16_t* dst = p.out + (row0 + h) * D + lane * CW;
+    uint16_t* dst = p.out + out_row(h) * D + lane * CW;
     if constexpr (CW == 4) {
       uint2 o;
       o.x = ptx::pack_bf16x2(acc[0], acc[1]);
@@ -928,10 +962,10 @@ constexpr size_t tc_smem_bytes() {
          kTcSoftThreads / 32 * kStgFloats * sizeof(float);
 }
 
-template <int D>
+template <int D, bool MQ>
 cudaError_t launch_tc_t(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
                         const CUtensorMap& tq, int grid, cudaStream_t stream, bool overlap) {
-  auto kern = decode_tc_kernel<D>;
+  auto kern = decode_tc_kernel<D, MQ>;
   constexpr size_t smem = tc_smem_bytes<D>();
   static thread_local int configured_device = -1;
   int dev = 0;
@@ -971,8 +1005,11 @@ size_t decode_tc_smem_bytes(int head_dim) {
 
 cudaError_t launch_decode_tc(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
                              const CUtensorMap& tq, int grid, cudaStream_t stream, bool overlap) {
-  if (p.head_dim == 64) return launch_tc_t<64>(p, tk, tv, tq, grid, stream, overlap);
-  return launch_tc_t<128>(p, tk, tv, tq, grid, stream, overlap);
+  if (p.q_len > 1)
+    return p.head_dim == 64 ? launch_tc_t<64, true>(p, tk, tv, tq, grid, stream, overlap)
+                            : launch_tc_t<128, true>(p, tk, tv, tq, grid, stream, overlap);
+  if (p.head_dim == 64) return launch_tc_t<64, false>(p, tk, tv, tq, grid, stream, overlap);
+  return launch_tc_t<128, false>(p, tk, tv, tq, grid, stream, overlap);
 }
 
 }  // namespace gqa

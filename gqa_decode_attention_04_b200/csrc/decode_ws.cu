@@ -1015,12 +1015,9 @@ cudaError_t launch_t(const DecodeParams& p, const CUtensorMap& tk, const CUtenso
 template <int D, bool MQ>
 cudaError_t launch_d(const DecodeParams& p, const DecodePlan& pl, const CUtensorMap& tk,
                      const CUtensorMap& tv, int grid, cudaStream_t s, bool o) {
-  if (!pl.split_heads)
-    return pl.n_tiles == 1 ? launch_t<D, 1, false, 4, MQ>(p, tk, tv, grid, s, o)
-                           : launch_t<D, 2, false, 4, MQ>(p, tk, tv, grid, s, o);
-  // Head split (17..32 heads per kv head): one 8-head n-tile per consumer.
-  return pl.consumers == 3 ? launch_t<D, 1, true, 3, MQ>(p, tk, tv, grid, s, o)
-                           : launch_t<D, 1, true, 4, MQ>(p, tk, tv, grid, s, o);
+  if (pl.split_heads) return cudaErrorInvalidValue;  // rows above 16 run on the tcgen05 kernel
+  return pl.n_tiles == 1 ? launch_t<D, 1, false, 4, MQ>(p, tk, tv, grid, s, o)
+                         : launch_t<D, 2, false, 4, MQ>(p, tk, tv, grid, s, o);
 }
 
 template <int D, int NT, bool SH, int C>
@@ -1037,10 +1034,11 @@ void fill(DecodePlan& pl) {
 // per segment: from 17 heads on its per-block cost (fixed by the 128-row tile) is below
 // the mma.sync kernel's, whose work grows with the heads (measured: 24 and 32 heads per
 // kv head, 29-49 us against 46-73 us).  Rows of several query tokens per sequence
-// (mq_rows) stay on the mma.sync kernel, whose head split covers 17..32 rows.
+// (mq_rows) follow the same rule; on the tcgen05 kernel they form one segment (<= 128).
 DecodePlan plan_decode(int head_dim, int group, bool mq_rows) {
   DecodePlan pl{};
-  if (group > 16 && !mq_rows) {
+  (void)mq_rows;
+  if (group > 16) {
     // Dense enough for the 5th-generation tensor cores: one 128-row MMA tile of heads.
     pl.tensor_cores = 1;
     pl.split_heads = 1;
@@ -1051,29 +1049,16 @@ DecodePlan plan_decode(int head_dim, int group, bool mq_rows) {
     pl.smem_bytes = decode_tc_smem_bytes(head_dim);
     return pl;
   }
-  if (group <= 16) {
-    pl.split_heads = 0;
-    pl.n_tiles = group <= 8 ? 1 : 2;
-    pl.consumers = 4;
-    pl.heads_per_seg = 8 * pl.n_tiles;
-  } else {  // 17..32 heads per kv head: one 8-head n-tile per consumer
-    pl.split_heads = 1;
-    pl.n_tiles = 1;
-    pl.consumers = group <= 24 ? 3 : 4;
-    pl.heads_per_seg = 8 * pl.consumers;
-  }
-  pl.n_ht = (group + pl.heads_per_seg - 1) / pl.heads_per_seg;
-  pl.ctas_per_sm = pl.split_heads ? ctas_per_sm<true>() : ctas_per_sm<false>();
-  const bool sh = pl.split_heads;
-  const int nt = pl.n_tiles, c = pl.consumers;
+  pl.split_heads = 0;
+  pl.n_tiles = group <= 8 ? 1 : 2;
+  pl.consumers = 4;
+  pl.heads_per_seg = 8 * pl.n_tiles;
+  pl.n_ht = 1;
+  pl.ctas_per_sm = ctas_per_sm<false>();
   if (head_dim == 64) {
-    if (!sh) { if (nt == 1) fill<64, 1, false, 4>(pl); else fill<64, 2, false, 4>(pl); }
-    else if (c == 3) fill<64, 1, true, 3>(pl);
-    else fill<64, 1, true, 4>(pl);
+    if (pl.n_tiles == 1) fill<64, 1, false, 4>(pl); else fill<64, 2, false, 4>(pl);
   } else {
-    if (!sh) { if (nt == 1) fill<128, 1, false, 4>(pl); else fill<128, 2, false, 4>(pl); }
-    else if (c == 3) fill<128, 1, true, 3>(pl);
-    else fill<128, 1, true, 4>(pl);
+    if (pl.n_tiles == 1) fill<128, 1, false, 4>(pl); else fill<128, 2, false, 4>(pl);
   }
   return pl;
 }

@@ -189,6 +189,27 @@ gqa_status make_map(CUtensorMap* m, const void* base, int64_t rows, int d, int d
   return GQA_OK;
 }
 
+// Query rows of several tokens per sequence for the tcgen05 kernel, as a 5-D view of
+// q [B, Q, Hk * G, D]: (64 columns, head in group, token, column group, b * Q * Hk + kvh).
+// The last coordinate's stride is G * D elements: (b * Q * Hk + kvh) * G * D is the first
+// element of kv head kvh's group for token 0 of sequence b.  One box = the G x Q rows of a
+// (sequence, kv head) and one column group, landing as rows (token, head) of the tile.
+gqa_status make_qmap_multi(CUtensorMap* m, const void* base, int B, int Q, int Hk, int G, int d) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return fail(GQA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  cuuint64_t dims[5] = {64, static_cast<cuuint64_t>(G), static_cast<cuuint64_t>(Q), static_cast<cuuint64_t>(d / 64),
+                        static_cast<cuuint64_t>(static_cast<int64_t>(B - 1) * Q * Hk + Hk)};
+  cuuint64_t strides[4] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(Hk) * G * d * 2, 128,
+                           static_cast<cuuint64_t>(G) * d * 2};
+  cuuint32_t box[5] = {64, static_cast<cuuint32_t>(G), static_cast<cuuint32_t>(Q), 1, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(GQA_ERR_CUDA, "cuTensorMapEncodeTiled (5-D query map) failed (%d)", (int)r);
+  return GQA_OK;
+}
+
 // Tensor maps of one decode launch and the launch itself (both kernels).
 cudaError_t launch_with_maps(const gqa::DecodeParams& p, const gqa::DecodePlan& plan,
                              const void* q, const void* k_pages, const void* v_pages, int64_t rows,
@@ -201,7 +222,9 @@ cudaError_t launch_with_maps(const gqa::DecodeParams& p, const gqa::DecodePlan& 
     *st = make_map(&tk, k_pages, rows, hd, dev, br, bg);
     if (*st == GQA_OK) *st = make_map(&tv, v_pages, rows, hd, dev, br, bg);
     if (*st == GQA_OK)
-      *st = make_map(&tq, q, static_cast<int64_t>(p.num_seqs) * p.num_heads, hd, dev, 128, hd / 64);
+      *st = p.q_len > 1
+                ? make_qmap_multi(&tq, q, p.num_seqs, p.q_len, p.num_kv_heads, p.group, hd)
+                : make_map(&tq, q, static_cast<int64_t>(p.num_seqs) * p.num_heads, hd, dev, 128, hd / 64);
     if (*st != GQA_OK) return cudaSuccess;
     return gqa::launch_decode_tc(p, tk, tv, tq, grid, strm, overlap);
   }
@@ -277,9 +300,9 @@ gqa_status decode_impl(const void* q, const void* k_pages, const void* v_pages,
   if (static_cast<int64_t>(max_blocks_per_seq) * page_size >= (int64_t{1} << 31))
     return fail(GQA_ERR_UNSUPPORTED, "max_blocks_per_seq * page_size exceeds 2^31");
   // Several query tokens: each kv head's rows are its group for every token, read with
-  // one pass over its K/V (the mma.sync kernel, up to 32 rows per kv head).
-  if (q_len > 1 && static_cast<int64_t>(num_heads / num_kv_heads) * q_len > 32)
-    return fail(GQA_ERR_UNSUPPORTED, "q_len %d x %d query heads per kv head exceeds 32", q_len,
+  // one pass over its K/V (one segment of at most 128 rows).
+  if (q_len > 1 && static_cast<int64_t>(num_heads / num_kv_heads) * q_len > 128)
+    return fail(GQA_ERR_UNSUPPORTED, "q_len %d x %d query heads per kv head exceeds 128", q_len,
                 num_heads / num_kv_heads);
   if (num_seqs == 0) return GQA_OK;
   if (!q || !k_pages || !v_pages || !block_table || !seq_lens || !out)
@@ -480,8 +503,8 @@ gqa_status gqa_multi_query_step(const void* q, const void* k_new, const void* v_
                                 float scale, int max_blocks_per_seq, int num_pages, void* stream) {
   if (q_len < 1) return fail(GQA_ERR_INVALID_ARG, "q_len %d < 1", q_len);
   if (num_kv_heads >= 1 && num_heads % num_kv_heads == 0 &&
-      static_cast<int64_t>(num_heads / num_kv_heads) * q_len > 32 && q_len > 1)
-    return fail(GQA_ERR_UNSUPPORTED, "q_len %d x %d query heads per kv head exceeds 32", q_len,
+      static_cast<int64_t>(num_heads / num_kv_heads) * q_len > 128 && q_len > 1)
+    return fail(GQA_ERR_UNSUPPORTED, "q_len %d x %d query heads per kv head exceeds 128", q_len,
                 num_heads / num_kv_heads);
   gqa_status s = append_impl(k_new, v_new, k_pages, v_pages, block_table, positions, num_seqs, q_len,
                              num_kv_heads, head_dim, page_size, max_blocks_per_seq, num_pages, stream);

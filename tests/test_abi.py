@@ -111,9 +111,9 @@ def _multi(lib, B=2, Q=2, H=4, Hk=1, D=64, ps=16, MB=4, P=8, ptr=1 << 20):
 
 @pytest.mark.parametrize("kw,status", [
     (dict(Q=0), -1),                # no query token
-    (dict(Q=9, H=4, Hk=1), -2),     # 9 x 4 rows per kv head > 32
-    (dict(Q=3, H=24, Hk=2), -2),    # 3 x 12 > 32
-    (dict(B=0, Q=8, H=4, Hk=1), 0), # 32 rows: accepted, nothing to do
+    (dict(Q=33, H=4, Hk=1), -2),    # 33 x 4 rows per kv head > 128
+    (dict(Q=3, H=96, Hk=2), -2),    # 3 x 48 > 128
+    (dict(B=0, Q=32, H=4, Hk=1), 0),  # 128 rows: accepted, nothing to do
 ])
 def test_multi_query_host_validation(lib, kw, status):
     assert _multi(lib, **kw) == status

@@ -1,7 +1,7 @@
 """Several query tokens per sequence on the GPU (gqa_paged_multi_query_attn,
 gqa_kv_append_multi, gqa_multi_query_step) against the oracle: query token i of sequence
 b attends to positions 0 .. seq_lens[b] - q_len + i.  Cases cover every kernel shape the
-q_len x group rows select (8-, 16-row token split; 24-, 32-row head split), both head
+q_len x group rows select (mma.sync for up to 16 rows, tcgen05 for 17..128), both head
 dims, page sizes 16..64, windows that end inside a sub-chunk, a block or a page, empty
 windows (seq_len < q_len), forced split counts (pieces merged across CTAs) and poisoned
 unused slots."""
@@ -30,14 +30,17 @@ def _oracle(inp, q):
 
 
 CASES = [
-    # lens, q_len, H, Hk, D, ps           rows per kv head
-    ([5, 37, 64, 130, 1, 16], 4, 8, 2, 128, 16),    # 16: token split, two n-tiles
-    ([200, 17, 3, 66], 2, 4, 1, 64, 16),            # 8: token split, one n-tile, D = 64
-    ([300, 65, 48, 7], 8, 4, 1, 128, 32),           # 32: head split, 4 consumers
-    ([150, 90, 2], 3, 24, 4, 128, 16),              # 18: head split, 3 consumers
+    # lens, q_len, H, Hk, D, ps           rows per kv head (kernel)
+    ([5, 37, 64, 130, 1, 16], 4, 8, 2, 128, 16),    # 16: mma.sync, two n-tiles
+    ([200, 17, 3, 66], 2, 4, 1, 64, 16),            # 8: mma.sync, one n-tile, D = 64
+    ([77, 300, 4], 5, 4, 4, 128, 16),               # MHA: 5 rows, mma.sync
+    ([300, 65, 48, 7], 8, 4, 1, 128, 32),           # 32: tcgen05
+    ([150, 90, 2], 3, 24, 4, 128, 16),              # 18: tcgen05
     ([1000, 20], 2, 16, 1, 128, 64),                # 32, page size 64
-    ([77, 300, 4], 5, 4, 4, 128, 16),               # MHA: 5 rows
-    ([129, 63, 64, 65], 7, 4, 1, 64, 16),           # windows ending around block edges
+    ([129, 63, 64, 65], 7, 4, 1, 64, 16),           # 28, D = 64: windows around block edges
+    ([700, 130, 9], 16, 8, 1, 128, 16),             # 128 rows: a full tcgen05 tile
+    ([513, 64, 3], 4, 96, 4, 128, 64),              # 96 rows (4 tokens x 24 heads)
+    ([260, 31], 6, 16, 2, 64, 32),                  # 48 rows, D = 64
 ]
 
 
@@ -52,9 +55,10 @@ def test_multi_query_parity(cuda_device, case):
     assert_close(gpu_f64(out), _oracle(inp, q), what=str(case))
 
 
+@pytest.mark.parametrize("rows", [16, 64])
 @pytest.mark.parametrize("workers", [1, 3, 57, 400])
-def test_multi_query_forced_splits(cuda_device, workers):
-    lens, Q, H, Hk, D, ps = [900, 333, 64, 2], 4, 8, 2, 128, 16
+def test_multi_query_forced_splits(cuda_device, workers, rows):
+    lens, Q, H, Hk, D, ps = [900, 333, 64, 2], rows // 4, 8, 2, 128, 16
     inp, q = _case(lens, Q, H, Hk, D, ps, seed=5)
     d = inp.to(cuda_device)
     try:
@@ -111,7 +115,7 @@ def test_kv_append_multi_is_bit_exact(cuda_device):
     assert np.array_equal(bf16_bits(d.k_pages), k2) and np.array_equal(bf16_bits(d.v_pages), v2)
 
 
-@pytest.mark.parametrize("Q,H,Hk", [(4, 8, 2), (8, 4, 1), (2, 32, 2)])
+@pytest.mark.parametrize("Q,H,Hk", [(4, 8, 2), (8, 4, 1), (2, 32, 2), (16, 8, 1)])
 def test_multi_query_step_equals_append_then_attend(cuda_device, Q, H, Hk):
     lens = [70, 300, 5, 129]
     inp = make_custom_inputs(lens, H, Hk, 128, 16, seed=17 + Q, extra_pages=2)
@@ -134,7 +138,7 @@ def test_multi_query_step_equals_append_then_attend(cuda_device, Q, H, Hk):
 
 
 def test_too_many_rows_is_refused_and_launches_nothing(cuda_device):
-    inp, q = _case([40], 9, 4, 1, 128, 16, seed=3)
+    inp, q = _case([40], 33, 4, 1, 128, 16, seed=3)
     d = inp.to(cuda_device)
     n0 = gq.launch_count()
     with pytest.raises(gq.GQAError) as e:
