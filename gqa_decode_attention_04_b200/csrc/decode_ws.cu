@@ -24,19 +24,17 @@
 //     S^T = K Q^T, softmax down the token axis, P^T moved to B-fragment layout with
 //     movmatrix, O^T += V^T P^T with V^T read by ldmatrix.trans.  Every K/V row in shared
 //     memory serves all query heads of its kv head, so HBM is read once per kv head.
-//       - small groups (G <= 16): each of the 4 consumers takes one 16-token sub-chunk
-//         of every stage for all G heads; at a piece end their partial softmax states
-//         are combined in shared memory.
-//       - 17..32 rows (several query tokens' heads of one kv head): each consumer takes
-//         8 of the rows over all 64 tokens of every stage.  Single-token groups of more
-//         than 16 heads run on the tcgen05 kernel (decode_tc.cu).
+//     Each of the 4 consumers takes one 16-token sub-chunk of every stage for all rows of
+//     the segment (up to 16: a group of heads, or several query tokens' groups); at a
+//     piece end their partial softmax states are combined in shared memory by an
+//     epilogue warp.  More rows per kv head run on the tcgen05 kernel (decode_tc.cu).
 //   * Online softmax in the log2 domain with a lazily moved reference: O and the sum are
 //     rescaled only when a head's running maximum rises by more than 8 (factor 256);
 //     numerator and denominator share the reference, so the result is unchanged.
 //   * Cross-CTA merge.  A segment spanning several CTAs leaves one piece per CTA
 //     (unnormalised O, reference max, sum); the last CTA to finish its piece (arrival
-//     counter) merges all pieces with their log-sum-exp weights using all consumer
-//     threads, writes out, and resets the counter to zero.
+//     counter) merges all pieces with their log-sum-exp weights in its epilogue warp,
+//     writes out, and resets the counter to zero.
 //   * Safety.  Page ids and lengths are range-checked on the device (bad work is skipped
 //     and an error bit set); every mbarrier wait is bounded in time.
 #include "internal.cuh"
@@ -229,41 +227,34 @@ __device__ __forceinline__ void attend_subchunk(uint32_t kb, uint32_t vb, int nv
 
 }  // namespace
 
-// Launch shape: CTAs per SM for the token split (several producer warps per SM keep
-// more TMA copies in flight) and for the head split, and the per-SM shared-memory
-// budget shared by their rings and merge areas (overridable at compile time for
-// tuning sweeps).
+// Launch shape: CTAs per SM (several producer warps per SM keep more TMA copies in
+// flight) and the per-SM shared-memory budget shared by their rings and merge areas
+// (overridable at compile time for tuning sweeps).
 #ifndef GQA_CTAS_TOKEN_SPLIT
 #define GQA_CTAS_TOKEN_SPLIT 2
-#endif
-#ifndef GQA_CTAS_HEAD_SPLIT
-#define GQA_CTAS_HEAD_SPLIT 1
 #endif
 #ifndef GQA_SMEM_PER_SM_KB
 #define GQA_SMEM_PER_SM_KB 212
 #endif
-template <bool SPLIT_HEADS>
-constexpr int ctas_per_sm() { return SPLIT_HEADS ? GQA_CTAS_HEAD_SPLIT : GQA_CTAS_TOKEN_SPLIT; }
+constexpr int kWsCtasPerSm = GQA_CTAS_TOKEN_SPLIT;
 
-// D: head_dim.  NT: 8-head n-tiles per consumer.  SPLIT_HEADS: consumers split the
-// query heads (else the 64 tokens of a stage).  C: consumer warps.  S: stages.  MQ:
+// D: head_dim.  NT: 8-head n-tiles per consumer (each consumer takes one 16-token
+// sub-chunk of every stage for all rows).  C: consumer warps.  S: stages.  MQ:
 // several query tokens per sequence (p.q_len): a kv head's rows are its group of heads
 // for each query token in turn (row r: token r / group, head r % group), one segment.
-template <int D, int NT, bool SPLIT_HEADS, int C, int S, bool MQ>
-__global__ void __launch_bounds__((C + (SPLIT_HEADS ? 1 : 2)) * 32, ctas_per_sm<SPLIT_HEADS>())
+template <int D, int NT, int C, int S, bool MQ>
+__global__ void __launch_bounds__((C + 2) * 32, kWsCtasPerSm)
 decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
                  const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
   using G_ = Geo<D>;
   constexpr int MT = D / 16;
   constexpr int NH = 8 * NT;             // heads one consumer covers
-  constexpr int NCT = C * 32;            // consumer threads
-  static_assert(SPLIT_HEADS || C == kSubChunks, "token split needs one consumer per sub-chunk");
+  static_assert(C == kSubChunks, "one consumer per sub-chunk");
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ int64_t s_wtot[kMaxWarps];
   __shared__ int s_start_b;
   __shared__ int64_t s_start_base;
-  __shared__ int s_prev;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -372,11 +363,11 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
   // Token split: at a piece end each consumer leaves its partial O^T in the part of the
   // stage only it read (its sub-chunk's K tile, and V tile for a second n-tile) and its
   // (max, sum) pairs in cml[stage]; the epilogue warp combines them and releases the stage.
-  static_assert(SPLIT_HEADS || 8 * D * 4 == G_::kSubBytes, "an 8-head partial fills one sub-chunk tile");
-  constexpr int kCml = SPLIT_HEADS ? 0 : S * C * NH * 2;  // floats
+  static_assert(8 * D * 4 == G_::kSubBytes, "an 8-head partial fills one sub-chunk tile");
+  constexpr int kCml = S * C * NH * 2;  // floats
   float* cml = reinterpret_cast<float*>(base_ptr + S * G_::kStageBytes);
   // Token split: the query rows of a piece arrive with its first block (bulk copy).
-  constexpr int kQBytes = SPLIT_HEADS ? 0 : NH * D * 2;
+  constexpr int kQBytes = NH * D * 2;
   uint8_t* qbuf = reinterpret_cast<uint8_t*>(cml + kCml);
   StageInfo* info = reinterpret_cast<StageInfo*>(qbuf + S * kQBytes);
   const uint32_t full_bar = ptx::smem_u32(info + S);
@@ -393,7 +384,7 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
     for (int s = 0; s < S; ++s) {
       ptx::mbar_init(full_bar + 8 * s, 1);
       ptx::mbar_init(empty_bar + 8 * s, C);
-      if (!SPLIT_HEADS) ptx::mbar_init(comb_bar + 8 * s, C);
+      ptx::mbar_init(comb_bar + 8 * s, C);
     }
     ptx::fence_mbarrier_init();
   }
@@ -458,22 +449,7 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
       const int ht = c.seg % p.n_ht;
       return static_cast<uint32_t>(min(NH, grp - ht * NH)) * D * 2u;
     };
-    // Pull a piece's query rows into L2 ahead of the consumers that load them.
-    auto prefetch_q = [&](const Cursor& c) {
-      const int kvh = c.seg / p.n_ht, ht = c.seg % p.n_ht;
-      const int nrows = min(p.heads_per_seg, grp - ht * p.heads_per_seg);
-      if constexpr (MQ) {  // rows of one query token at a time are contiguous
-        for (int r = lane; r < nrows; r += 32) {
-          const uint8_t* qr = reinterpret_cast<const uint8_t*>(p.q + seq_row(c.b, kvh, ht * p.heads_per_seg + r) * D);
-          for (int off = 0; off < D * 2; off += 128) ptx::prefetch_l2(qr + off);
-        }
-      } else {
-        const uint8_t* q0 = reinterpret_cast<const uint8_t*>(p.q + seq_row(c.b, kvh, ht * p.heads_per_seg) * D);
-        for (int off = lane * 128; off < nrows * D * 2; off += 32 * 128) ptx::prefetch_l2(q0 + off);
-      }
-    };
     int page = page_of(cu);
-    if (SPLIT_HEADS) prefetch_q(cu);
     int piece_blk0 = cu.blk;
     bool first_piece = true;
     int64_t seg_base = x0 - cu.blk;
@@ -512,13 +488,13 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
                    ((last && piece_blk0 == 0 && cu.blk + 1 == cu.nblk) ? kSole : 0) |
                    (first_piece ? kFirstPieceOfCta : 0);
         uint32_t bytes = static_cast<uint32_t>(__popc(submask)) * 2u * G_::kSubBytes;
-        if (!SPLIT_HEADS && first && !p.arm_without_copy) bytes += q_rows_bytes(cu);
+        if (first && !p.arm_without_copy) bytes += q_rows_bytes(cu);
         if (bytes) ptx::mbar_arrive_expect_tx(full_bar + 8 * stage, bytes);
         else ptx::mbar_arrive(full_bar + 8 * stage);
       }
       if (i == 0) ptx::pdl_wait_prerequisites();  // K/V may still be written by the previous kernel
       __syncwarp();
-      if constexpr (!SPLIT_HEADS) {
+      {
         if (first && !p.arm_without_copy) {
           const int kvh = cu.seg / p.n_ht, ht = cu.seg % p.n_ht;
           if constexpr (MQ) {
@@ -548,17 +524,14 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
       if (last) first_piece = false;
       if (i + 1 < total) {
         walk_next(cu, next_len, p, segs, cap);
-        if (cu.blk == 0) {
-          seg_base = x0 + i + 1;
-          if (SPLIT_HEADS) prefetch_q(cu);
-        }
+        if (cu.blk == 0) seg_base = x0 + i + 1;
         page = page_of(cu);
       }
     }
     return;
   }
 
-  if (!SPLIT_HEADS && warp == C + 1) {
+  if (warp == C + 1) {
     // ============================================================ epilogue warp
     // Walks the same block list.  At each piece end it waits for the C consumers' states
     // in the stage, combines them, writes out (or this CTA's piece of the segment),
@@ -710,7 +683,6 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
   const int j = warp;
   const int g = lane >> 2;
   const int q = lane & 3;
-  const int tid = threadIdx.x;  // 0 .. NCT-1
   uint32_t kofs[4], vofs[4];
   {
     // K as the A operand: matrices (t0-7, d), (t8-15, d), (t0-7, d+8), (t8-15, d+8).
@@ -731,7 +703,6 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
   float mref[NT][2], lsum[NT][2];
   int nrows_seg = 0;  // valid heads of the segment
   int nrows_c = 0;    // valid heads of this consumer's tile
-  int hoff_c = 0;     // first segment-relative head of this consumer's tile
   int cdrop[NT][2];   // MQ: query tokens newer than each column's own
   const int max_drop = MQ ? p.q_len - 1 : 0;
   const float sl2 = p.scale_log2;
@@ -740,9 +711,8 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int kvh = seg / p.n_ht;
     const int ht = seg % p.n_ht;
     nrows_seg = min(p.heads_per_seg, grp - ht * p.heads_per_seg);
-    hoff_c = SPLIT_HEADS ? j * NH : 0;
-    nrows_c = max(0, min(NH, nrows_seg - hoff_c));
-    const int r0 = ht * p.heads_per_seg + hoff_c;  // first row of this consumer's tile
+    nrows_c = min(NH, nrows_seg);
+    const int r0 = ht * p.heads_per_seg;  // first row of the segment
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -752,14 +722,12 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
     for (int nt = 0; nt < NT; ++nt) {
       const int h = nt * 8 + g;
       const bool v = h < nrows_c;
-      // token split: from the rows staged with the piece's first block; else from HBM/L2
-      const uint32_t* qrow =
-          SPLIT_HEADS ? reinterpret_cast<const uint32_t*>(p.q + seq_row(b, kvh, r0 + (v ? h : 0)) * D)
-                      : reinterpret_cast<const uint32_t*>(qbuf + stage * kQBytes) + (v ? h : 0) * (D / 2);
+      // from the rows staged with the piece's first block
+      const uint32_t* qrow = reinterpret_cast<const uint32_t*>(qbuf + stage * kQBytes) + (v ? h : 0) * (D / 2);
 #pragma unroll
       for (int ks = 0; ks < MT; ++ks) {
-        qf[ks][nt][0] = v ? (SPLIT_HEADS ? __ldg(qrow + ks * 8 + q) : qrow[ks * 8 + q]) : 0u;
-        qf[ks][nt][1] = v ? (SPLIT_HEADS ? __ldg(qrow + ks * 8 + 4 + q) : qrow[ks * 8 + 4 + q]) : 0u;
+        qf[ks][nt][0] = v ? qrow[ks * 8 + q] : 0u;
+        qf[ks][nt][1] = v ? qrow[ks * 8 + 4 + q] : 0u;
       }
     }
 #pragma unroll
@@ -773,69 +741,6 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
     }
   };
 
-  // Cross-CTA step of a piece that is not the whole segment: all consumer threads have
-  // stored this CTA's piece; the last CTA to arrive merges every piece into out.
-  auto cross_cta = [&](const StageInfo& si) {
-    __threadfence();
-    ptx::named_barrier_sync(1, NCT);
-    const int64_t segid = static_cast<int64_t>(si.b) * segs + si.seg;
-    if (tid == 0) s_prev = atomicAdd(p.counters + segid, 1);
-    ptx::named_barrier_sync(1, NCT);
-    const int prev = s_prev;
-    const int64_t wf = worker_of(si.seg_base, T, W);
-    const int64_t wl = worker_of(si.seg_base + si.nblk - 1, T, W);
-    if (prev != static_cast<int>(wl - wf)) return;
-    __threadfence();
-    const int hps = p.heads_per_seg;
-    const int kvh = si.seg / p.n_ht;
-    const int ht = si.seg % p.n_ht;
-    // Outputs in batches of 8 per thread; for each piece the 8 (max, sum) pairs and 8
-    // partial values are loaded together, so a piece costs one L2 round trip per batch.
-    const int total_out = nrows_seg * D;
-    for (int base = 0; base < total_out; base += 8 * NCT) {
-      float M[8], L[8], acc[8];
-      int off_o[8], off_ml[8];
-      bool act[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const int idx = base + tid + k * NCT;
-        act[k] = idx < total_out;
-        const int h = act[k] ? idx / D : 0;
-        off_o[k] = act[k] ? h * D + (idx - h * D) : 0;
-        off_ml[k] = h * 2;
-        M[k] = -INFINITY;
-        L[k] = 0.f;
-        acc[k] = 0.f;
-      }
-      for (int64_t ww = wf; ww <= wl; ++ww) {
-        const int64_t sl = piece_slot(ww, si.seg_base, T, W);
-        const float* po = p.part_o + sl * hps * D;
-        const float* pm = p.part_ml + sl * hps * 2;
-        float2 ml[8];
-        float ov[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          ml[k] = act[k] ? __ldcg(reinterpret_cast<const float2*>(pm + off_ml[k])) : make_float2(-INFINITY, 0.f);
-          ov[k] = act[k] ? __ldcg(po + off_o[k]) : 0.f;
-        }
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const float mn = fmaxf(M[k], ml[k].x);
-          const float mu = (mn == -INFINITY) ? 0.f : mn;
-          const float a = ptx::ex2(M[k] - mu), bw = ptx::ex2(ml[k].x - mu);
-          L[k] = L[k] * a + ml[k].y * bw;
-          acc[k] = acc[k] * a + ov[k] * bw;
-          M[k] = mn;
-        }
-      }
-#pragma unroll
-      for (int k = 0; k < 8; ++k)
-        if (act[k])
-          reinterpret_cast<__nv_bfloat16*>(p.out)[seq_row(si.b, kvh, ht * hps + off_o[k] / D) * D + off_o[k] % D] =
-              __float2bfloat16_rn(L[k] > 0.f ? acc[k] / L[k] : 0.f);
-    }
-    if (tid == 0) p.counters[segid] = 0;
-  };
 
   for (int64_t i = 0; i < total; ++i) {
     const int stage = static_cast<int>(i % S);
@@ -848,31 +753,17 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
     if (si.flags & kFirstOfPiece) load_q(si.b, si.seg, stage);
 
     const uint32_t kst = ring + stage * G_::kStageBytes;
-    if constexpr (SPLIT_HEADS) {
-      if (nrows_c > 0) {
-#pragma unroll 1
-        for (int sc = 0; sc < kSubChunks; ++sc) {
-          if ((si.submask >> sc) & 1) {
-            const uint32_t kb = kst + sc * G_::kSubBytes;
-            attend_subchunk<D, NT, MQ>(kb, kb + G_::kTileBytes, min(kChunk, si.nvalid - sc * kChunk),
-                                       kofs, vofs, qf, o, mref, lsum, sl2, g, q, si.rem - sc * kChunk,
-                                       max_drop, cdrop);
-          }
-        }
-      }
-    } else {
-      if ((si.submask >> j) & 1) {
-        const uint32_t kb = kst + j * G_::kSubBytes;
-        attend_subchunk<D, NT, MQ>(kb, kb + G_::kTileBytes, min(kChunk, si.nvalid - j * kChunk),
-                                   kofs, vofs, qf, o, mref, lsum, sl2, g, q, si.rem - j * kChunk, max_drop,
-                                   cdrop);
-      }
+    if ((si.submask >> j) & 1) {
+      const uint32_t kb = kst + j * G_::kSubBytes;
+      attend_subchunk<D, NT, MQ>(kb, kb + G_::kTileBytes, min(kChunk, si.nvalid - j * kChunk),
+                                 kofs, vofs, qf, o, mref, lsum, sl2, g, q, si.rem - j * kChunk, max_drop,
+                                 cdrop);
     }
     const bool piece_end = si.flags & kLastOfPiece;
     __syncwarp();
-    // A token-split piece end keeps the stage: the epilogue warp releases it after the
-    // combine (it arrives for all C consumers).
-    if (lane == 0 && (SPLIT_HEADS || !piece_end)) ptx::mbar_arrive(empty_bar + 8 * stage);
+    // A piece end keeps the stage: the epilogue warp releases it after the combine (it
+    // arrives for all C consumers).
+    if (lane == 0 && !piece_end) ptx::mbar_arrive(empty_bar + 8 * stage);
 
     if (!piece_end) continue;
 
@@ -894,39 +785,8 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int ht = si.seg % p.n_ht;
     const int slot = static_cast<int>(w * 2 + ((si.flags & kFirstPieceOfCta) ? 0 : 1));
 
-    if constexpr (SPLIT_HEADS) {
-      // Each consumer owns its heads over every token: write them directly.
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int h = nt * 8 + 2 * q + e;  // within this consumer's tile
-          if (h < nrows_c) {
-            const int hs = hoff_c + h;         // within the segment
-            if (sole) {
-              const float inv = lt[nt][e] > 0.f ? 1.f / lt[nt][e] : 0.f;
-              __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.out) + seq_row(si.b, kvh, ht * hps + hs) * D;
-#pragma unroll
-              for (int mt = 0; mt < MT; ++mt) {
-                dst[mt * 16 + g] = __float2bfloat16_rn(o[mt][nt][e] * inv);
-                dst[mt * 16 + g + 8] = __float2bfloat16_rn(o[mt][nt][e + 2] * inv);
-              }
-            } else {
-              float* po = p.part_o + (static_cast<int64_t>(slot) * hps + hs) * D;
-#pragma unroll
-              for (int mt = 0; mt < MT; ++mt) {
-                po[mt * 16 + g] = o[mt][nt][e];
-                po[mt * 16 + g + 8] = o[mt][nt][e + 2];
-              }
-              if (g == 0)
-                *reinterpret_cast<float2*>(p.part_ml + (static_cast<int64_t>(slot) * hps + hs) * 2) =
-                    make_float2(mref[nt][e], lt[nt][e]);
-            }
-          }
-        }
-      if (!sole) cross_cta(si);
-    } else {
-      // Token split: hand the piece to the epilogue warp.  This consumer's partial O^T
+    {
+      // Hand the piece to the epilogue warp.  This consumer's partial O^T
       // (relative to its own reference max) goes into the tiles of its sub-chunk, which
       // only it read; its (max, sum) pairs into cml[stage][j].
       float* mlj = cml + (stage * C + j) * NH * 2;
@@ -965,14 +825,13 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
 namespace {
 
 
-template <int D, int NT, bool SPLIT_HEADS, int C>
+template <int D, int NT, int C>
 struct Cfg {
   static constexpr int kNH = 8 * NT;
-  // token split: per-stage (max, sum) hand-off area, sized for up to 8 stages
-  static constexpr size_t kMerge = SPLIT_HEADS ? 0 : static_cast<size_t>(8 * C * kNH * 2) * sizeof(float);
-  static constexpr size_t kBudget =
-      static_cast<size_t>(GQA_SMEM_PER_SM_KB) * 1024 / ctas_per_sm<SPLIT_HEADS>();
-  static constexpr size_t kQBytes = SPLIT_HEADS ? 0 : static_cast<size_t>(kNH) * D * 2;
+  // per-stage (max, sum) hand-off area, sized for up to 8 stages
+  static constexpr size_t kMerge = static_cast<size_t>(8 * C * kNH * 2) * sizeof(float);
+  static constexpr size_t kBudget = static_cast<size_t>(GQA_SMEM_PER_SM_KB) * 1024 / kWsCtasPerSm;
+  static constexpr size_t kQBytes = static_cast<size_t>(kNH) * D * 2;
   static constexpr int kStagesRaw =
       static_cast<int>((kBudget - kMerge) / (Geo<D>::kStageBytes + kQBytes));
   static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
@@ -980,11 +839,11 @@ struct Cfg {
                                   kStages * (sizeof(StageInfo) + 24);
 };
 
-template <int D, int NT, bool SH, int C, bool MQ>
+template <int D, int NT, int C, bool MQ>
 cudaError_t launch_t(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int grid,
                      cudaStream_t stream, bool overlap) {
-  using CF = Cfg<D, NT, SH, C>;
-  auto kern = decode_ws_kernel<D, NT, SH, C, CF::kStages, MQ>;
+  using CF = Cfg<D, NT, C>;
+  auto kern = decode_ws_kernel<D, NT, C, CF::kStages, MQ>;
   static thread_local int configured_device = -1;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -994,7 +853,7 @@ cudaError_t launch_t(const DecodeParams& p, const CUtensorMap& tk, const CUtenso
     if (e != cudaSuccess) return e;
     configured_device = dev;
   }
-  const int threads = (C + (SH ? 1 : 2)) * 32;  // consumers, producer, (epilogue)
+  const int threads = (C + 2) * 32;  // consumers, producer, epilogue
   if (!overlap) {
     kern<<<grid, threads, CF::kSmem, stream>>>(tk, tv, p);
     return cudaGetLastError();
@@ -1015,14 +874,12 @@ cudaError_t launch_t(const DecodeParams& p, const CUtensorMap& tk, const CUtenso
 template <int D, bool MQ>
 cudaError_t launch_d(const DecodeParams& p, const DecodePlan& pl, const CUtensorMap& tk,
                      const CUtensorMap& tv, int grid, cudaStream_t s, bool o) {
-  if (pl.split_heads) return cudaErrorInvalidValue;  // rows above 16 run on the tcgen05 kernel
-  return pl.n_tiles == 1 ? launch_t<D, 1, false, 4, MQ>(p, tk, tv, grid, s, o)
-                         : launch_t<D, 2, false, 4, MQ>(p, tk, tv, grid, s, o);
+  return pl.n_tiles == 1 ? launch_t<D, 1, 4, MQ>(p, tk, tv, grid, s, o) : launch_t<D, 2, 4, MQ>(p, tk, tv, grid, s, o);
 }
 
-template <int D, int NT, bool SH, int C>
+template <int D, int NT, int C>
 void fill(DecodePlan& pl) {
-  using CF = Cfg<D, NT, SH, C>;
+  using CF = Cfg<D, NT, C>;
   pl.stages = CF::kStages;
   pl.smem_bytes = CF::kSmem;
 }
@@ -1041,7 +898,6 @@ DecodePlan plan_decode(int head_dim, int group, bool mq_rows) {
   if (group > 16) {
     // Dense enough for the 5th-generation tensor cores: one 128-row MMA tile of heads.
     pl.tensor_cores = 1;
-    pl.split_heads = 1;
     pl.heads_per_seg = group < 128 ? group : 128;
     pl.n_ht = (group + pl.heads_per_seg - 1) / pl.heads_per_seg;
     pl.ctas_per_sm = 1;
@@ -1049,16 +905,15 @@ DecodePlan plan_decode(int head_dim, int group, bool mq_rows) {
     pl.smem_bytes = decode_tc_smem_bytes(head_dim);
     return pl;
   }
-  pl.split_heads = 0;
   pl.n_tiles = group <= 8 ? 1 : 2;
   pl.consumers = 4;
   pl.heads_per_seg = 8 * pl.n_tiles;
   pl.n_ht = 1;
-  pl.ctas_per_sm = ctas_per_sm<false>();
+  pl.ctas_per_sm = kWsCtasPerSm;
   if (head_dim == 64) {
-    if (pl.n_tiles == 1) fill<64, 1, false, 4>(pl); else fill<64, 2, false, 4>(pl);
+    if (pl.n_tiles == 1) fill<64, 1, 4>(pl); else fill<64, 2, 4>(pl);
   } else {
-    if (pl.n_tiles == 1) fill<128, 1, false, 4>(pl); else fill<128, 2, false, 4>(pl);
+    if (pl.n_tiles == 1) fill<128, 1, 4>(pl); else fill<128, 2, 4>(pl);
   }
   return pl;
 }

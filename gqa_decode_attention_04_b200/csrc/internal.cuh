@@ -73,7 +73,6 @@ cudaError_t launch_kv_append(const AppendParams& p, cudaStream_t stream);
 // How a (head_dim, group) problem is mapped onto the decode kernel.
 struct DecodePlan {
   int tensor_cores;   // 1: tcgen05 kernel (large groups), 0: mma.sync warp-specialized kernel
-  int split_heads;    // 0: consumers split the 64-token stage by tokens; 1: by query heads
   int n_tiles;        // 8-head MMA n-tiles per consumer
   int consumers;      // consumer (MMA) warps per CTA; one producer warp is added
   int heads_per_seg;  // query heads a segment covers
