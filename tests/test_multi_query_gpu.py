@@ -144,3 +144,65 @@ def test_too_many_rows_is_refused_and_launches_nothing(cuda_device):
     with pytest.raises(gq.GQAError) as e:
         gq.paged_multi_query_attn(q.to(cuda_device), d.k_pages, d.v_pages, d.block_table, d.seq_lens)
     assert e.value.status == -2 and gq.launch_count() == n0
+
+
+@pytest.mark.parametrize("Q,H,Hk", [(4, 8, 2), (8, 32, 8)])
+def test_multi_query_step_replays_in_a_cuda_graph(cuda_device, Q, H, Hk):
+    """After a first call the multi-token step is captured once and replayed with new
+    buffer contents: new draft rows, positions and lengths advanced by q_len each time
+    (rows per kv head: 16 on the mma.sync kernel, 32 on the tcgen05 kernel)."""
+    D, ps = 128, 16
+    lens0 = [200, 27, 70]
+    B = len(lens0)
+    inp = make_custom_inputs(lens0, H, Hk, D, ps, seed=40 + Q, extra_pages=12, max_blocks_per_seq=24)
+    d = inp.to(cuda_device)
+    gen = torch.Generator().manual_seed(41 + Q)
+    q = torch.randn(B, Q, H, D, generator=gen).to(torch.bfloat16).to(cuda_device)
+    kn = torch.empty(B, Q, Hk, D, dtype=torch.bfloat16, device=cuda_device)
+    vn = torch.empty_like(kn)
+    pos = torch.empty(B, dtype=torch.int32, device=cuda_device)
+    lens = torch.empty(B, dtype=torch.int32, device=cuda_device)
+    out = torch.empty(B, Q, H, D, dtype=torch.bfloat16, device=cuda_device)
+    # each sequence's block-table row gets the pages its four steps of q_len tokens need
+    steps = 4
+    bt = torch.full((B, 24), -1, dtype=torch.int32)
+    used = set(int(x) for x in inp.block_table.flatten().tolist() if x >= 0)
+    free = [p for p in range(inp.num_pages) if p not in used]
+    for b in range(B):
+        row = [int(x) for x in inp.block_table[b].tolist() if x >= 0]
+        need = -(-(lens0[b] + steps * Q) // ps) - len(row)
+        assert need <= len(free)
+        row += free[:need]
+        free = free[need:]
+        bt[b, :len(row)] = torch.tensor(row, dtype=torch.int32)
+    bt_d = bt.to(cuda_device)
+    h_k, h_v = bf16_bits(inp.k_pages), bf16_bits(inp.v_pages)
+    cur = torch.tensor(lens0, dtype=torch.int32)
+    s = torch.cuda.Stream(cuda_device)
+    graph = None
+    for step in range(steps):
+        new_k = torch.randn(B, Q, Hk, D, generator=gen).to(torch.bfloat16)
+        new_v = torch.randn(B, Q, Hk, D, generator=gen).to(torch.bfloat16)
+        hpos = cur.clone()
+        cur = cur + Q
+        kn.copy_(new_k)
+        vn.copy_(new_v)
+        pos.copy_(hpos)
+        lens.copy_(cur)
+        if step == 0:  # first call, then capture
+            with torch.cuda.stream(s):
+                gq.multi_query_step(q, kn, vn, d.k_pages, d.v_pages, bt_d, pos, lens, out=out, scale=d.scale)
+            s.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=s):
+                gq.multi_query_step(q, kn, vn, d.k_pages, d.v_pages, bt_d, pos, lens, out=out, scale=d.scale)
+            # capture records the launch only; the first call's effect is what the state holds
+        else:
+            graph.replay()
+        torch.cuda.synchronize()
+        gq.check_device_error()
+        h_k, h_v = oracle.kv_append_multi(h_k, h_v, bf16_bits(new_k), bf16_bits(new_v), bt.numpy(), hpos.numpy())
+        want = oracle.paged_multi_query_attention(bf16_bits(q), h_k, h_v, bt.numpy(), cur.numpy(), d.scale)
+        assert np.array_equal(bf16_bits(d.k_pages), h_k), f"step {step}"
+        assert_close(gpu_f64(out), want, what=f"step {step}")
+    del graph
