@@ -158,7 +158,7 @@ gqa_status gqa_decode_step(const void* q, const void* k_new, const void* v_new, 
  * gqa_paged_multi_query_attn -- q, out [num_seqs, q_len, num_heads, head_dim] bf16; the
  *   other arguments, layouts, requirements and errors as gqa_paged_decode_attn.  Each kv
  *   head's K/V are read once for all q_len x (num_heads / num_kv_heads) query rows; that
- *   product must be <= 32 when q_len > 1 (GQA_ERR_UNSUPPORTED otherwise).
+ *   product must be <= 128 when q_len > 1 (GQA_ERR_UNSUPPORTED otherwise).
  * gqa_multi_query_step -- gqa_kv_append_multi, then gqa_paged_multi_query_attn, as
  *   gqa_decode_step does for one token (the attention launch overlaps the append).
  */

@@ -35,7 +35,7 @@ CASES = [
     # (seq_lens, H, Hk, D, ps): long enough that segments span several CTAs, so the
     # split counters and partials in the shared array are exercised.
     ([3000, 17, 900, 1], 32, 8, 128, 16),   # token split (G = 4)
-    ([700, 2500], 96, 1, 128, 64),          # head split (MQA, G = 96)
+    ([700, 2500], 96, 1, 128, 64),          # tcgen05 kernel and split merge (MQA, G = 96)
     ([40, 33], 4, 1, 64, 16),               # head_dim 64, tiny
 ]
 
