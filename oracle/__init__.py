@@ -19,3 +19,11 @@ from .paged_attention import (  # noqa: F401
     merge_partial_pieces,
     kv_cache_bytes,
 )
+from .fp8_cache import (  # noqa: F401
+    E4M3_MAX,
+    e4m3_bits_to_f64,
+    f64_to_e4m3_bits,
+    quantize_pages,
+    dequantize_pages,
+    paged_decode_attention_fp8,
+)

@@ -23,6 +23,7 @@ import os
 import numpy as np
 import torch
 
+import oracle.fp8_cache as F8
 import oracle.paged_attention as PA
 
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "closed_forms.json")
@@ -434,6 +435,80 @@ def check_kv_append_multi():
     assert np.array_equal(k1, k0) and np.array_equal(v1, v0)
 
 
+# ------------------------------------------------------------- FP8 (e4m3) K/V cache
+
+def check_e4m3_decode_matches_torch():
+    """All 256 e4m3 codes decode to torch.float8_e4m3fn's values (a library routine);
+    S.1111.111 is NaN, the largest value 448, the smallest subnormal 2^-9."""
+    codes = np.arange(256, dtype=np.uint8)
+    ours = F8.e4m3_bits_to_f64(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(np.isnan(ours), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(ours[ok], ref[ok])
+    assert np.nanmax(ours) == 448.0 and ours[1] == 2.0 ** -9 and np.isnan(ours[0x7F]) and np.isnan(ours[0xFF])
+
+
+def check_e4m3_encode_rounding_and_saturation():
+    """Nearest code with ties to the even mantissa, every finite code round-trips, values
+    up to the overflow midpoint match torch's cast, larger ones saturate to 448."""
+    codes = np.arange(256, dtype=np.uint8)
+    vals = F8.e4m3_bits_to_f64(codes)
+    fin = codes[~np.isnan(vals)]
+    assert np.array_equal(F8.f64_to_e4m3_bits(F8.e4m3_bits_to_f64(fin)), fin)
+    pos = np.sort(np.unique(vals[(vals > 0) & ~np.isnan(vals)]))
+    for a, b in zip(pos[:-1], pos[1:]):
+        mid = (a + b) / 2
+        ca, cb = F8.f64_to_e4m3_bits([a, b])
+        want = ca if (ca & 1) == 0 else cb      # the even mantissa wins a tie
+        assert F8.f64_to_e4m3_bits([mid])[0] == want, (a, b)
+        assert F8.f64_to_e4m3_bits([-mid])[0] == (want | 0x80)
+    rng = np.random.default_rng(24)
+    x = np.concatenate([rng.standard_normal(4000) * 40, rng.uniform(-463.9, 463.9, 2000),
+                        rng.standard_normal(1000) * 2.0 ** -7])
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(F8.f64_to_e4m3_bits(x), ref)
+    big = np.array([464.0, 500.0, 1e30, -464.0, -7e4])
+    assert list(F8.f64_to_e4m3_bits(big)) == [0x7E, 0x7E, 0x7E, 0xFE, 0xFE]
+
+
+def check_fp8_cache_attention_on_exact_values():
+    """K/V on the e4m3 grid times power-of-two scales (exact in bf16): attention over the
+    coded cache equals the bf16 oracle over the same values; scales differ per kv head
+    and between K and V."""
+    rng = np.random.default_rng(25)
+    sl = [33, 7, 64]
+    H, Hk, D, ps = 8, 2, 16, 16
+    q, kp, vp, bt, _, _ = _random_paged(rng, sl, H, Hk, D, ps)
+    ks = np.array([0.5, 2.0 ** -3])
+    vs = np.array([4.0, 1.0])
+    grid = F8.e4m3_bits_to_f64(np.arange(0, 0x7E, dtype=np.uint8))
+    grid = np.concatenate([grid, -grid])
+    kval = rng.choice(grid, size=kp.shape) * ks[None, :, None, None]
+    vval = rng.choice(grid, size=vp.shape) * vs[None, :, None, None]
+    kc, vc = F8.quantize_pages(kval, ks), F8.quantize_pages(vval, vs)
+    assert np.array_equal(F8.dequantize_pages(kc, ks), kval)
+    got = F8.paged_decode_attention_fp8(q, kc, vc, ks, vs, bt, np.array(sl), 0.3)
+    kb, vb = PA.f64_to_bf16_bits(kval), PA.f64_to_bf16_bits(vval)
+    assert np.array_equal(PA.bf16_bits_to_f64(kb), kval)
+    want = PA.paged_decode_attention(q, kb, vb, bt, np.array(sl), 0.3)
+    assert np.allclose(got, want, rtol=0, atol=1e-12)
+
+
+def check_fp8_quantization_error_bound():
+    """Writing a value costs at most half a step: relative 2^-4 in the normal range
+    (3 mantissa bits), absolute 2^-10 * scale below the smallest normal."""
+    rng = np.random.default_rng(26)
+    s = np.array([0.25, 3.0])
+    x = rng.standard_normal((4, 2, 16, 8)) * np.array([20.0, 300.0])[None, :, None, None]
+    y = F8.dequantize_pages(F8.quantize_pages(x, s), s)
+    r = np.abs(x) / s[None, :, None, None]
+    normal = (r >= 2.0 ** -6) & (r <= 448.0)
+    assert np.all(np.abs(y - x)[normal] <= 2.0 ** -4 * np.abs(x)[normal] + 1e-300)
+    sub = r < 2.0 ** -6
+    assert np.all(np.abs(y - x)[sub] <= 2.0 ** -10 * np.broadcast_to(s[None, :, None, None], x.shape)[sub])
+
+
 ALL_CHECKS = [
     check_bf16_decode,
     check_closed_form_three_tokens,
@@ -455,4 +530,8 @@ ALL_CHECKS = [
     check_multi_query_against_sdpa_causal,
     check_multi_query_single_token_and_newest,
     check_kv_append_multi,
+    check_e4m3_decode_matches_torch,
+    check_e4m3_encode_rounding_and_saturation,
+    check_fp8_cache_attention_on_exact_values,
+    check_fp8_quantization_error_bound,
 ]

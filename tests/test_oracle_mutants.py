@@ -7,6 +7,7 @@ pin catches would mean the pins cannot see that class of mistake.
 import numpy as np
 import pytest
 
+import oracle.fp8_cache as F8
 import oracle.paged_attention as PA
 import oracle_pins as P
 
@@ -111,6 +112,32 @@ def _append_multi_rows_reversed(kp, vp, kn, vn, bt, positions):
     return k, v
 
 
+def _e4m3_bias8(bits):
+    b = np.asarray(bits, dtype=np.uint8).astype(np.int64)
+    sign = np.where(b & 0x80, -1.0, 1.0)
+    e, m = (b >> 3) & 0xF, b & 0x7
+    out = np.where(e == 0, sign * (m / 8.0) * 2.0 ** -7, sign * (1.0 + m / 8.0) * np.exp2(e - 8.0))
+    return np.where((e == 15) & (m == 7), np.nan, out)   # exponent bias 8 instead of 7
+
+
+def _e4m3_truncating(x):
+    a = np.asarray(x, dtype=np.float64)
+    codes = np.arange(0x7F, dtype=np.uint8)
+    vals = F8.e4m3_bits_to_f64(codes)
+    out = np.zeros(a.shape, dtype=np.uint8)
+    for i, v in np.ndenumerate(a):
+        mag = min(abs(v), 448.0)
+        c = codes[np.searchsorted(vals, mag, side="right") - 1]   # rounds toward zero
+        out[i] = c | (0x80 if v < 0 else 0)
+    return out
+
+
+def _fp8_attention_swapped_scales(q, kc, vc, ks, vs, bt, sl, scale):
+    return _ORIG_FP8_ATTN(q, kc, vc, vs, ks, bt, sl, scale)       # K and V scales swapped
+
+
+_ORIG_FP8_ATTN = F8.paged_decode_attention_fp8
+
 MUTANTS = [
     ("kv_head_of", _kv_head_modulo),
     ("gather_sequence_kv", _gather_swapped),
@@ -125,12 +152,18 @@ MUTANTS = [
     ("multi_query_window", _window_excludes_self),
     ("multi_query_window", _window_sees_drafts),
     ("kv_append_multi", _append_multi_reversed),
+    ("F8:e4m3_bits_to_f64", _e4m3_bias8),
+    ("F8:f64_to_e4m3_bits", _e4m3_truncating),
+    ("F8:paged_decode_attention_fp8", _fp8_attention_swapped_scales),
 ]
 
 
 @pytest.mark.parametrize("name,fn", MUTANTS, ids=[f.__name__ for _, f in MUTANTS])
 def test_mutant_is_caught(monkeypatch, name, fn):
-    monkeypatch.setattr(PA, name, fn)
+    if name.startswith("F8:"):
+        monkeypatch.setattr(F8, name[3:], fn)
+    else:
+        monkeypatch.setattr(PA, name, fn)
     caught = []
     for check in P.ALL_CHECKS:
         try:
