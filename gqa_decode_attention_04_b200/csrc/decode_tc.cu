@@ -535,8 +535,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
     const bool pos = sl2 >= 0.f;  // a negative scale turns the row maximum into a minimum
     constexpr int HD = D / 2;     // output columns each warpgroup finishes at a piece end
     float mref = -INFINITY, lsum = 0.f;
-    // MQ: query tokens newer than this row's own (rows past the group's are padding).
-    const int cdrop = MQ ? (r < p.group * p.q_len ? p.q_len - 1 - r / p.group : 0) : 0;
+    // MQ: query tokens newer than this row's own.  Rows past the group's are padding whose
+    // query rows are stale shared memory: their window is empty, so they never trigger an
+    // O rescale (which waits for every earlier P V) and contribute nothing.
+    const int cdrop = MQ ? (r < p.group * p.q_len ? p.q_len - 1 - r / p.group : (1 << 30)) : 0;
     int wg_phase = 0;
     bool failed = false;
     // Every wait outcome is made warp-uniform: the TMEM loads and stores that follow are
