@@ -1,5 +1,5 @@
-// Paged decode attention for large query groups (MQA-like: many query heads per K/V head)
-// on the 5th-generation tensor cores (tcgen05, TMEM accumulators).
+// Paged decode attention for large query groups (MQA-like: more than 16 query rows per K/V
+// head) on the 5th-generation tensor cores (tcgen05, TMEM accumulators).
 //
 // Same result as decode_ws.cu (page "TensorRT对Multi-Query Attention的专项优化支持": decode
 // re-reads all cached K/V; with MQA every query head shares one K/V head, and the plugin
@@ -32,6 +32,13 @@
 //     partials by log-sum-exp weights.  Merging inside the decode (the last CTA of a
 //     segment to finish merges it) put the merge's dependent loads behind the other CTAs'
 //     K/V streams at the very end of every CTA's range.
+//   * Several query tokens per sequence (the MQ instantiation, 17..128 rows per kv head):
+//     a kv head's rows are its group of heads for each query token in turn (row r: token
+//     r / group, head r % group), one segment per kv head.  The query tile comes from a
+//     5-D tensor map (columns, head, token, column group, sequence x kv head) whose last
+//     stride is group x head_dim elements, one box per column group; each softmax thread
+//     masks its row's window (the sequence up to its own token) from the stage's
+//     remaining length, and tile rows past the group get an empty window.
 //   * Safety: every wait is bounded; on a timeout all warps leave their loops, the MMA
 //     warps wait for their issued MMAs, and TMEM is released before exit.
 #include <type_traits>
