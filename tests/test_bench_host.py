@@ -3,20 +3,28 @@ by (checked against the byte counts stated for the workloads), which decode kern
 roofline names, and the rule that committed ncu traffic only counts for the kernel
 sources it was captured from."""
 import json
+from types import SimpleNamespace
 
 import pytest
+import torch
 
 import bench
 from workloads import WORKLOADS, make_inputs
 
 
-@pytest.mark.parametrize("index,kv,qo", [
-    (1, 14_592, 2_048),              # 2 seqs of 17 + 40 tokens, 1 kv head, D 64; q+out 2x2x4x64x2
-    (3, 268_435_456, 3_145_728),     # 64 x 8192 tokens, 1 kv head, D 128; q+out 2x64x96x128x2
-    (4, 2_147_483_648, 131_072),     # 4 x 131072 tokens, 8 kv heads, D 128; q+out 2x4x64x128x2
+def _shape(lens, H, Hk, D, ps):
+    """What the byte accounting reads of a workload: its lengths and shapes."""
+    return SimpleNamespace(num_seqs=len(lens), num_heads=H, num_kv_heads=Hk, head_dim=D, page_size=ps,
+                           seq_lens=torch.tensor(lens, dtype=torch.int32))
+
+
+@pytest.mark.parametrize("shape,kv,qo", [
+    (([17, 40], 4, 1, 64, 16), 14_592, 2_048),                  # tiny MQA; q+out 2x2x4x64x2
+    (([8192] * 64, 96, 1, 128, 64), 268_435_456, 3_145_728),    # MQA batch; q+out 2x64x96x128x2
+    (([131072] * 4, 64, 8, 128, 16), 2_147_483_648, 131_072),   # long context; q+out 2x4x64x128x2
 ])
-def test_algorithmic_bytes_match_the_stated_workload_sizes(index, kv, qo):
-    inp = make_inputs(index, poison=False)
+def test_algorithmic_bytes_match_the_stated_workload_sizes(shape, kv, qo):
+    inp = _shape(*shape)
     b = bench.algorithmic_bytes(inp, with_append=False)
     assert b["kv"] == kv
     pages = int(((inp.seq_lens.long() + inp.page_size - 1) // inp.page_size).sum())
@@ -24,13 +32,18 @@ def test_algorithmic_bytes_match_the_stated_workload_sizes(index, kv, qo):
     assert b["append"] == 0 and b["step"] == b["decode"]
 
 
+def test_the_generated_small_workload_has_the_stated_sizes():
+    inp = make_inputs(1, poison=False)
+    assert bench.algorithmic_bytes(inp, with_append=False)["kv"] == 14_592
+
+
 def test_append_bytes_count_new_rows_and_indices():
-    inp = make_inputs(5, poison=False)
+    inp = _shape(list(range(1, 257)), 32, 8, 128, 16)
     b = bench.algorithmic_bytes(inp, with_append=True)
     B, Hk, D = inp.num_seqs, inp.num_kv_heads, inp.head_dim
     assert b["append"] == 2 * (B * Hk * D * 2) * 2 + 8 * B
     assert b["step"] == b["decode"] + b["append"]
-    assert bench.algorithmic_bytes(inp, with_append=True, num_seqs=10)["kv"] < b["kv"]
+    assert bench.algorithmic_bytes(inp, with_append=True, num_seqs=10)["kv"] == sum(range(1, 11)) * Hk * D * 4
 
 
 def test_roofline_kernel_follows_the_group_size():
