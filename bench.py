@@ -5,27 +5,37 @@
 
 One step = one pass of the whole hot path over one batch: kv_append writes each
 sequence's new K/V token into its page, then paged_decode_attn attends over the
-paged cache (split-KV with its log-sum-exp merge inside the same launch).  The
-default workload is the GQA serving batch (32 sequences, 32 query / 8 KV heads,
-head_dim 128, page_size 16, lengths uniform in [512, 4096]).
+paged cache (split-KV with its log-sum-exp merge).  The headline workload (default
+2) is the GQA serving batch (32 sequences, 32 query / 8 KV heads, head_dim 128,
+page_size 16, lengths uniform in [512, 4096]).
 
-Prints ONE JSON line on rank 0.  `value` is the step's algorithmic HBM bytes
-(all K/V bytes of every context token, plus q, out, the appended rows, block
-table and lengths) divided by the step time, in TB/s, summed over ranks.  Each
-rank runs its own independent batch (weak scaling, no collective on the data
-path).  Inputs are resident in HBM; the working set (two copies of the page
-pools, rotated step by step) is several times the 126 MB L2.
+Prints ONE JSON line on rank 0.  `value` is the step's algorithmic HBM bytes (all
+K/V bytes of every context token, plus q, out, the appended rows, block table and
+lengths) divided by the step time, in TB/s, summed over ranks.  Each rank runs its
+own independent batch (weak scaling, no collective on the data path).  Inputs are
+resident in HBM; the working set (at least two copies of the page pools, rotated
+launch by launch) is several times the 126 MB L2.
+
+On one GPU the line also carries `workloads`: every one of the five synthetic
+workloads measured the same way -- its decode launch and its whole step, each
+replayed from a CUDA graph of back-to-back launches (so host call overhead is not
+what is measured), median over at least five replays and at least 0.2 s of GPU time,
+against the measured HBM copy bandwidth.  With --fp8 (the default) each GQA workload
+also reports the same decode over an e4m3 copy of its cache.
 """
 from __future__ import annotations
 
 import argparse
+import datetime
 import hashlib
 import json
 import math
 import os
+import platform
 import statistics
 import subprocess
 import sys
+import threading
 import time
 
 import torch
@@ -44,6 +54,10 @@ KERNEL_SOURCES = {
     "decode_ws_kernel": [_CSRC + "decode_ws.cu", _CSRC + "ptx.cuh", _CSRC + "internal.cuh"],
     "decode_tc_kernel": [_CSRC + "decode_tc.cu", _CSRC + "ptx.cuh", _CSRC + "internal.cuh"],
 }
+# Each timed loop runs at least this long on the GPU and at least this many replays.
+MIN_LOOP_SECONDS = 0.2
+MIN_REPEATS = 5
+GRAPH_LAUNCHES = 100
 
 
 def decode_kernel_for(inp) -> str:
@@ -54,21 +68,23 @@ def decode_kernel_for(inp) -> str:
 
 # ------------------------------------------------------------------ helpers
 
-def algorithmic_bytes(inp, with_append: bool, num_seqs=None) -> dict:
+def algorithmic_bytes(inp, with_append: bool, num_seqs=None, kv_elem_bytes: int = 2) -> dict:
     """Bytes the step must move: every cached K/V byte once, q in, out back, plus
     the block-table entries and lengths read, and the appended rows.  With
-    num_seqs, only the first num_seqs sequences count."""
+    num_seqs, only the first num_seqs sequences count.  kv_elem_bytes = 1 for an
+    8-bit cache (which also reads one K and one V scale per kv head)."""
     B = inp.num_seqs if num_seqs is None else num_seqs
     H, Hk, D, ps = inp.num_heads, inp.num_kv_heads, inp.head_dim, inp.page_size
     L = inp.seq_lens[:B].to(torch.int64).cpu()
-    kv = int(L.sum()) * Hk * D * 2 * 2
+    kv = int(L.sum()) * Hk * D * kv_elem_bytes * 2
     pages = int(((L + ps - 1) // ps).sum())
     qo = 2 * B * H * D * 2
-    meta = pages * 4 + B * 4
+    meta = pages * 4 + B * 4 + (2 * Hk * 4 if kv_elem_bytes == 1 else 0)
     decode = kv + qo + meta
     append = 0
     if with_append:
-        append = 2 * (B * Hk * D * 2) * 2 + B * 4 + B * 4  # read new rows + write slots, positions, bt
+        # read the new bf16 rows, write them into their slots, positions and block-table entries
+        append = B * Hk * D * 2 * 2 + B * Hk * D * kv_elem_bytes * 2 + B * 4 + B * 4
     return {"kv": kv, "decode": decode, "append": append, "step": decode + append}
 
 
@@ -106,60 +122,108 @@ def profiled_traffic(workload_name: str, kernel: str, units_per_launch: int):
         return None
 
 
-class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return platform.processor() or "unknown"
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons.  Samples are kept only if
+    their own timestamp falls inside one of the timed windows recorded with window():
+    the figures describe the GPU under load, not the set-up around it."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: str, period_ms: int = 25):
         self.gpu_index = gpu_index
+        self.period_ms = period_ms
         self.proc = None
+        self.lines = []
+        self.windows = []
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu_index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", str(self.period_ms)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._reader = threading.Thread(target=self._read, daemon=True)
+            self._reader.start()
         except Exception:
             self.proc = None
-        time.sleep(0.3)
         return self
 
+    def _read(self):
+        for ln in self.proc.stdout:
+            if ln.strip():
+                self.lines.append(ln)
+
+    def window(self):
+        """Context manager marking one timed region (host wall clock, with the GPU busy)."""
+        sampler = self
+
+        class _W:
+            def __enter__(self):
+                self.t0 = time.time()
+
+            def __exit__(self, *exc):
+                sampler.windows.append((self.t0, time.time()))
+                return False
+        return _W()
+
     def __exit__(self, *exc):
-        self.lines = []
         if self.proc is not None:
-            time.sleep(0.25)
+            time.sleep(2.5 * self.period_ms / 1000.0)  # the last window's final sample
             self.proc.terminate()
             try:
-                out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
-                out = ""
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+            self._reader.join(timeout=5)
         return False
 
-    def summary(self):
-        sm, mx, reasons = [], None, set()
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
+    @staticmethod
+    def _stamp(s: str):
+        for fmt in ("%Y/%m/%d %H:%M:%S.%f", "%Y/%m/%d %H:%M:%S"):
             try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
+                return datetime.datetime.strptime(s.strip(), fmt).timestamp()
             except ValueError:
                 continue
-            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-            for n, v in zip(names, parts[5:9]):
+        return None
+
+    def summary(self):
+        sm, mx, reasons, n_all = [], None, set(), 0
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 10:
+                continue
+            n_all += 1
+            t = self._stamp(parts[0])
+            if t is None or not any(a <= t <= b for a, b in self.windows):
+                continue
+            try:
+                sm.append(float(parts[2]))
+                mx = float(parts[3])
+            except ValueError:
+                continue
+            for n, v in zip(self.REASONS, parts[6:10]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0,
+                    "samples_total": n_all}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "samples_total": n_all, "period_ms": self.period_ms,
+                "timed_windows_s": round(sum(b - a for a, b in self.windows), 3)}
 
 
 def setup_dist(n_gpus: int):
@@ -170,7 +234,6 @@ def setup_dist(n_gpus: int):
         backend = "nccl" if torch.cuda.is_available() else "gloo"
         if torch.cuda.is_available():
             torch.cuda.set_device(local)
-        import datetime
         dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
         return rank, world, local
     return 0, 1, 0
@@ -199,6 +262,12 @@ def barrier():
 
 
 # ------------------------------------------------------------------ CPU oracle timing
+
+ONE_CORE_REASON = ("the oracle is timed as it stands: plain per-(sequence, head) loops over numpy "
+                   "vector operations, which one Python thread drives; BLAS threads would not "
+                   "parallelise them, and splitting the batch over processes would be a tuned "
+                   "variant of the oracle, not the oracle")
+
 
 def time_oracle(inp, min_seconds: float, max_seconds: float):
     """Time the fp64 oracle, as it stands, on the same step (its kv_append, then its
@@ -234,6 +303,11 @@ def time_oracle(inp, min_seconds: float, max_seconds: float):
     return step_bytes * passes / elapsed, n * passes / elapsed, desc
 
 
+def _cpu_fields():
+    return {"cpu_model": cpu_model(), "host_cores_available": os.cpu_count(),
+            "why_one_core": ONE_CORE_REASON}
+
+
 # ------------------------------------------------------------------ arms
 
 def run_reference(args, rank, world):
@@ -242,7 +316,6 @@ def run_reference(args, rank, world):
     prefix of the sequences (all of them when that fits the time budget)."""
     if rank != 0:
         return None
-    import numpy as np
     from threadpoolctl import threadpool_limits
     import oracle
 
@@ -285,7 +358,8 @@ def run_reference(args, rank, world):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "tokens_per_s": sum(seqs) / total_t,
         "config": {**_config_keys(inp, world), "l2": "host memory (CPU oracle)"},
-        "cpu_baseline": {"value": value, "unit": "TB/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "TB/s", "cores": 1, "kind": "oracle", "sample": sample,
+                         **_cpu_fields()},
         "e2e": {"value": value, "unit": "TB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -305,10 +379,178 @@ def _with_append(inp, seed):
     (positions = seq_len - 1, already counted in seq_lens)."""
     if inp.positions is None:
         g = torch.Generator().manual_seed(seed + 2)
+        dev = inp.q.device
         inp.positions = (inp.seq_lens - 1).clamp(min=0).to(torch.int32)
-        inp.k_new = torch.randn(inp.num_seqs, inp.num_kv_heads, inp.head_dim, generator=g).to(torch.bfloat16)
-        inp.v_new = torch.randn(inp.num_seqs, inp.num_kv_heads, inp.head_dim, generator=g).to(torch.bfloat16)
+        inp.k_new = torch.randn(inp.num_seqs, inp.num_kv_heads, inp.head_dim, generator=g).to(torch.bfloat16).to(dev)
+        inp.v_new = torch.randn(inp.num_seqs, inp.num_kv_heads, inp.head_dim, generator=g).to(torch.bfloat16).to(dev)
     return inp
+
+
+def _pool_sets(inp_dev, dev):
+    """The batch plus enough further copies of its page pools that the launches, rotating
+    over them, never find their K/V in L2: at least 2 copies and 4x L2 in total (<= 8)."""
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    kv_bytes = 2 * inp_dev.k_pages.numel() * inp_dev.k_pages.element_size()
+    n_sets = min(8, max(2, math.ceil(4 * l2 / max(1, kv_bytes))))
+    sets = [inp_dev]
+    for _ in range(n_sets - 1):
+        s = inp_dev.to(dev)
+        s.k_pages = inp_dev.k_pages.clone()
+        s.v_pages = inp_dev.v_pages.clone()
+        sets.append(s)
+    desc = (f"inputs larger than L2: {n_sets} rotated pool copies of {kv_bytes / 1e6:.1f} MB each "
+            f"vs {l2 / 1e6:.0f} MB L2" if kv_bytes * 2 > l2 else
+            f"{n_sets} rotated pool copies of {kv_bytes / 1e3:.1f} KB each (the batch fits in L2)")
+    return sets, desc
+
+
+def graph_time_us(enqueue, n_calls: int, stream, clocks=None):
+    """Device time of one call: n_calls back-to-back calls captured once in a CUDA graph,
+    the graph replayed at least MIN_REPEATS times and MIN_LOOP_SECONDS, CUDA events on
+    the launching stream around each replay.  Returns (median, min, max) in us."""
+    for i in range(3):  # first calls set up the workspace, tensor maps and attributes
+        enqueue(i)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream()
+    with torch.cuda.graph(g, stream=cap):
+        for i in range(n_calls):
+            enqueue(i)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    one = max(1e-3, e0.elapsed_time(e1) / 1e3)
+    reps = max(MIN_REPEATS, math.ceil(MIN_LOOP_SECONDS / one))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    win = clocks.window() if clocks is not None else None
+    if win is not None:
+        win.__enter__()
+    for a, b in evs:
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+    torch.cuda.synchronize()
+    if win is not None:
+        win.__exit__(None, None, None)
+    per = sorted(a.elapsed_time(b) * 1e3 / n_calls for a, b in evs)
+    del g
+    return statistics.median(per), per[0], per[-1]
+
+
+def measure_workload(gq, inp_dev, dev, peak, clocks, fp8: bool):
+    """One entry of the `workloads` object: the decode launch and the whole step of this
+    batch, each from a CUDA graph of back-to-back calls (see graph_time_us)."""
+    stream = torch.cuda.current_stream(dev)
+    sets, l2_desc = _pool_sets(inp_dev, dev)
+    n = len(sets)
+    B, H, D = inp_dev.num_seqs, inp_dev.num_heads, inp_dev.head_dim
+    out = torch.empty((B, H, D), dtype=torch.bfloat16, device=dev)
+    nb = algorithmic_bytes(inp_dev, with_append=True)
+
+    def decode(i):
+        s = sets[i % n]
+        gq.paged_decode_attn(s.q, s.k_pages, s.v_pages, s.block_table, s.seq_lens, out=out, scale=s.scale)
+
+    def step(i):
+        s = sets[i % n]
+        gq.decode_step(s.q, s.k_new, s.v_new, s.k_pages, s.v_pages, s.block_table, s.positions,
+                       s.seq_lens, out=out, scale=s.scale)
+
+    d_med, d_min, d_max = graph_time_us(decode, GRAPH_LAUNCHES, stream, clocks)
+    s_med, s_min, s_max = graph_time_us(step, GRAPH_LAUNCHES, stream, clocks)
+    gq.check_device_error()
+    achieved = nb["decode"] / (d_med * 1e-6) / 1e9
+    kernel = decode_kernel_for(inp_dev)
+    entry = {
+        "workload": inp_dev.name, "num_seqs": B, "num_heads": H, "num_kv_heads": inp_dev.num_kv_heads,
+        "head_dim": D, "page_size": inp_dev.page_size,
+        "context_tokens": int(inp_dev.seq_lens.to(torch.int64).sum()),
+        "decode_kernel": kernel + (" + merge_tc_kernel" if kernel == "decode_tc_kernel" else ""),
+        "decode_us": d_med, "decode_us_min_max": [d_min, d_max],
+        "step_us": s_med, "step_us_min_max": [s_min, s_max],
+        "algorithmic_bytes_per_decode": nb["decode"], "kv_bytes": nb["kv"],
+        "achieved_gbs": achieved, "frac": achieved / peak,
+        "kv_tbps": nb["kv"] / (d_med * 1e-6) / 1e12,
+        "step_tbps": nb["step"] / (s_med * 1e-6) / 1e12,
+        "tokens_per_s": B / (s_med * 1e-6),
+        "l2": l2_desc, "graph_launches": GRAPH_LAUNCHES,
+    }
+    if fp8 and hasattr(gq, "paged_decode_attn_fp8"):
+        entry["fp8"] = measure_fp8(gq, sets, dev, peak, clocks)
+    del sets, out
+    return entry
+
+
+def measure_fp8(gq, sets, dev, peak, clocks):
+    """The same decode over an e4m3 copy of each pool set (one scale per kv head for K
+    and one for V, from the largest magnitude in the pool), and its step with the
+    quantising append."""
+    stream = torch.cuda.current_stream(dev)
+    s0 = sets[0]
+    Hk = s0.num_kv_heads
+    ks = (s0.k_pages.float().abs().amax(dim=(0, 2, 3)) / 448.0).clamp(min=1e-30).contiguous()
+    vs = (s0.v_pages.float().abs().amax(dim=(0, 2, 3)) / 448.0).clamp(min=1e-30).contiguous()
+    pools = []
+    for s in sets:
+        kq = torch.empty(s.k_pages.shape, dtype=torch.uint8, device=dev)
+        vq = torch.empty(s.v_pages.shape, dtype=torch.uint8, device=dev)
+        gq.quantize_pages_fp8(s.k_pages, kq, ks)
+        gq.quantize_pages_fp8(s.v_pages, vq, vs)
+        pools.append((kq, vq))
+    n = len(sets)
+    B, H, D = s0.num_seqs, s0.num_heads, s0.head_dim
+    out = torch.empty((B, H, D), dtype=torch.bfloat16, device=dev)
+    nb = algorithmic_bytes(s0, with_append=True, kv_elem_bytes=1)
+
+    def decode(i):
+        s, (kq, vq) = sets[i % n], pools[i % n]
+        gq.paged_decode_attn_fp8(s.q, kq, vq, ks, vs, s.block_table, s.seq_lens, out=out, scale=s.scale)
+
+    def step(i):
+        s, (kq, vq) = sets[i % n], pools[i % n]
+        gq.decode_step_fp8(s.q, s.k_new, s.v_new, kq, vq, ks, vs, s.block_table, s.positions, s.seq_lens,
+                           out=out, scale=s.scale)
+
+    d_med, d_min, d_max = graph_time_us(decode, GRAPH_LAUNCHES, stream, clocks)
+    s_med, _, _ = graph_time_us(step, GRAPH_LAUNCHES, stream, clocks)
+    gq.check_device_error()
+    achieved = nb["decode"] / (d_med * 1e-6) / 1e9
+    del pools
+    return {"decode_us": d_med, "decode_us_min_max": [d_min, d_max], "step_us": s_med,
+            "algorithmic_bytes_per_decode": nb["decode"], "kv_bytes": nb["kv"],
+            "achieved_gbs": achieved, "frac": achieved / peak,
+            "kv_tbps": nb["kv"] / (d_med * 1e-6) / 1e12, "tokens_per_s": B / (s_med * 1e-6),
+            "scales": "one fp32 scale per kv head for K and for V: max |x| / 448 over the pool"}
+
+
+class PackedInputs:
+    """The step's per-call inputs (q, k_new, v_new, positions, seq_lens, block table) in
+    one pinned host buffer and one device buffer at 256-byte aligned offsets, so a step
+    moves them with a single host-to-device copy; the device tensors are views."""
+
+    def __init__(self, inp_cpu, dev):
+        srcs = [inp_cpu.q, inp_cpu.k_new, inp_cpu.v_new, inp_cpu.positions, inp_cpu.seq_lens,
+                inp_cpu.block_table]
+        offs, off = [], 0
+        for t in srcs:
+            offs.append(off)
+            off += (t.numel() * t.element_size() + 255) // 256 * 256
+        self.nbytes = off
+        self.host = torch.empty(off, dtype=torch.uint8).pin_memory()
+        self.dev = torch.empty(off, dtype=torch.uint8, device=dev)
+        self.views = []
+        for t, o in zip(srcs, offs):
+            nb = t.numel() * t.element_size()
+            self.host[o:o + nb].copy_(t.contiguous().view(-1).view(torch.uint8))
+            self.views.append(self.dev[o:o + nb].view(t.dtype).view(t.shape))
+        self.payload = sum(t.numel() * t.element_size() for t in srcs)
+
+    def upload(self):
+        self.dev.copy_(self.host, non_blocking=True)
 
 
 def run_ours(args, rank, world, local):
@@ -316,85 +558,76 @@ def run_ours(args, rank, world, local):
 
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    peak, peak_kind = measured_peak()
     seed = rank_seed(args.workload, rank)
     inp_cpu = _with_append(make_inputs(args.workload, seed=seed, poison=False), seed)
     nbytes = algorithmic_bytes(inp_cpu, with_append=True)
-
-    # Rotate between independent copies of the pools so consecutive steps never
-    # find their K/V in L2 (each copy alone is larger than L2 for the default workload).
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    kv_bytes = 2 * inp_cpu.k_pages.numel() * 2
-    n_sets = max(2, math.ceil(4 * l2 / max(1, kv_bytes)))
-    n_sets = min(n_sets, 8)
-    base = inp_cpu.to(dev)
-    sets = [base]
-    for _ in range(n_sets - 1):
-        s = inp_cpu.to(dev)
-        s.k_pages = base.k_pages.clone()
-        s.v_pages = base.v_pages.clone()
-        sets.append(s)
+    sets, l2_desc = _pool_sets(inp_cpu.to(dev), dev)
+    n_sets = len(sets)
     out = torch.empty((inp_cpu.num_seqs, inp_cpu.num_heads, inp_cpu.head_dim), dtype=torch.bfloat16, device=dev)
-    stream = torch.cuda.current_stream(dev)
 
-    def step(s):
+    def step(s, ins=None):
         # one call: kv_append, then the decode (its launch overlaps the append)
-        gq.decode_step(s.q, s.k_new, s.v_new, s.k_pages, s.v_pages, s.block_table, s.positions,
-                       s.seq_lens, out=out, scale=s.scale)
-
-    def decode_only(s):
-        gq.paged_decode_attn(s.q, s.k_pages, s.v_pages, s.block_table, s.seq_lens, out=out, scale=s.scale)
+        q, kn, vn, pos, sl, bt = ins if ins is not None else (s.q, s.k_new, s.v_new, s.positions, s.seq_lens,
+                                                               s.block_table)
+        gq.decode_step(q, kn, vn, s.k_pages, s.v_pages, bt, pos, sl, out=out, scale=s.scale)
 
     for i in range(args.warmup):
         step(sets[i % n_sets])
     torch.cuda.synchronize()
     gq.check_device_error()
 
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    launches0 = gq.launch_count()
     visible = [x for x in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if x.strip()]
     smi_index = visible[local] if local < len(visible) else str(local)
+    workloads = {}
     with ClockSampler(smi_index) as clocks:
+        # ---- headline: exactly K steps through the public API, device-timed
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        launches0 = gq.launch_count()
         barrier()
         torch.cuda.synchronize()
-        start.record(stream)
-        for i in range(args.steps):
-            step(sets[i % n_sets])
-        end.record(stream)
-        torch.cuda.synchronize()
+        with clocks.window():
+            start.record(stream)
+            for i in range(args.steps):
+                step(sets[i % n_sets])
+            end.record(stream)
+            torch.cuda.synchronize()
         barrier()
-    launches = gq.launch_count() - launches0
-    gq.check_device_error()
-    step_ms_local = start.elapsed_time(end) / args.steps
-    # The decode kernel alone (roofline figure): the same launches back to back, timed
-    # with CUDA events on the launching stream; the average interval per launch.
-    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    for i in range(3):
-        decode_only(sets[i % n_sets])
-    torch.cuda.synchronize()
-    d0.record(stream)
-    for i in range(args.steps):
-        decode_only(sets[i % n_sets])
-    d1.record(stream)
-    torch.cuda.synchronize()
-    decode_ms_local = d0.elapsed_time(d1) / args.steps
-    total_ms, total_bytes = reduce_max_sum(step_ms_local * args.steps, nbytes["step"] * args.steps, dev)
-    _, total_seqs = reduce_max_sum(0.0, inp_cpu.num_seqs * args.steps, dev)
+        launches = gq.launch_count() - launches0
+        gq.check_device_error()
+        step_ms_local = start.elapsed_time(end) / args.steps
+        total_ms, total_bytes = reduce_max_sum(step_ms_local * args.steps, nbytes["step"] * args.steps, dev)
+        _, total_seqs = reduce_max_sum(0.0, inp_cpu.num_seqs * args.steps, dev)
+
+        # ---- the decode kernel alone (roofline) and every workload (one GPU)
+        if world == 1 and not args.headline_only:
+            for idx in sorted(WORKLOADS):
+                if idx == args.workload:
+                    entry = measure_workload(gq, sets[0], dev, peak, clocks, fp8=not args.no_fp8)
+                else:
+                    wl = _with_append(make_inputs(idx, seed=1000 + idx, device=dev, poison=False), 1000 + idx)
+                    entry = measure_workload(gq, wl, dev, peak, clocks, fp8=not args.no_fp8)
+                    del wl
+                    torch.cuda.empty_cache()
+                workloads[str(idx)] = entry
+            head = workloads[str(args.workload)]
+        else:
+            head = measure_workload(gq, sets[0], dev, peak, clocks, fp8=False)
+    decode_us = head["decode_us"]
+
     step_ms = total_ms / args.steps
     value_tbps = total_bytes / (total_ms * 1e-3) / 1e12
     tokens_per_s = total_seqs / (total_ms * 1e-3)
 
-    # ---- end to end through the public API: host inputs in, host result out
-    pin = lambda t: t.pin_memory()  # noqa: E731
-    host_in = [pin(inp_cpu.q), pin(inp_cpu.k_new), pin(inp_cpu.v_new), pin(inp_cpu.positions),
-               pin(inp_cpu.seq_lens), pin(inp_cpu.block_table)]
+    # ---- end to end through the public API: host inputs in (one packed copy), host result out
+    packed = PackedInputs(inp_cpu, dev)
     host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in host_in)
     d2h = host_out.numel() * host_out.element_size()
 
     def e2e_step(s):
-        for src, dst in zip(host_in, (s.q, s.k_new, s.v_new, s.positions, s.seq_lens, s.block_table)):
-            dst.copy_(src, non_blocking=True)
-        step(s)
+        packed.upload()
+        step(s, packed.views)
         host_out.copy_(out, non_blocking=True)
         stream.synchronize()
 
@@ -412,8 +645,7 @@ def run_ours(args, rank, world, local):
     e2e_tbps = total_bytes / (e2e_ms * 1e-3) / 1e12
     gq.check_device_error()
 
-    peak, peak_kind = measured_peak()
-    achieved_gbs = nbytes["decode"] / (decode_ms_local * 1e-3) / 1e9
+    achieved_gbs = nbytes["decode"] / (decode_us * 1e-6) / 1e9
     units = int(inp_cpu.seq_lens.to(torch.int64).sum())
     line = {
         "metric": METRIC,
@@ -431,24 +663,27 @@ def run_ours(args, rank, world, local):
         "pct_of_peak": 100.0 * value_tbps * 1e3 / (peak * world),
         "tokens_per_s": tokens_per_s,
         "kv_tbps": nbytes["kv"] * args.steps * world / (total_ms * 1e-3) / 1e12,
-        "config": {**_config_keys(inp_cpu, world),
-                   "l2": f"inputs larger than L2: {n_sets} rotated pool copies of "
-                         f"{kv_bytes / 1e6:.0f} MB each vs {l2 / 1e6:.0f} MB L2"},
-        "e2e": {"value": e2e_tbps, "unit": "TB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": e2e_ms / args.steps},
+        "config": {**_config_keys(inp_cpu, world), "l2": l2_desc},
+        "e2e": {"value": e2e_tbps, "unit": "TB/s", "h2d_bytes_per_step": packed.payload,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps,
+                "copies_per_step": "1 host-to-device (packed inputs) + 1 device-to-host (out)"},
         "gpu_launches": int(launches),
         "roofline": {"bound": "hbm", "kernel": decode_kernel_for(inp_cpu),
                      "achieved": achieved_gbs, "peak": peak, "unit": "GB/s",
-                     "frac": achieved_gbs / peak, "peak_kind": f"{peak_kind} (hbm_gbs)",
+                     "frac": achieved_gbs / peak, "peak_kind": f"{peak_kind} (hbm_gbs, burst copy)",
                      "traffic": profiled_traffic(WORKLOADS[args.workload].name, decode_kernel_for(inp_cpu), units),
                      "algorithmic_bytes_per_launch": nbytes["decode"],
-                     "decode_ms": decode_ms_local},
+                     "decode_us": decode_us, "decode_us_min_max": head["decode_us_min_max"],
+                     "timing": f"CUDA graph of {GRAPH_LAUNCHES} back-to-back decode launches, median over "
+                               f">= {MIN_REPEATS} replays and >= {MIN_LOOP_SECONDS} s"},
         "clocks": clocks.summary(),
     }
+    if workloads:
+        line["workloads"] = workloads
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         bps, sps, desc = time_oracle(inp_cpu, min_seconds=10.0, max_seconds=30.0)
         line["cpu_baseline"] = {"value": bps / 1e12, "unit": "TB/s", "cores": 1, "kind": "oracle",
-                                "sample": desc, "tokens_per_s": sps}
+                                "sample": desc, "tokens_per_s": sps, **_cpu_fields()}
     return line
 
 
@@ -460,6 +695,8 @@ def main():
     ap.add_argument("--workload", type=int, default=2, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the 8-bit cache entries")
+    ap.add_argument("--headline-only", action="store_true", help="skip the other workloads")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -367,7 +367,8 @@ def paged_decode_attn_noalloc(q, k_pages, v_pages, block_table, seq_lens, out: t
 
     Scratch is a fixed array inside the library, shared by every call: calls that
     overlap on the GPU race, and the first call on a device should come before any
-    stream capture.  `out` must be given.  Device-side range errors are not reported.
+    stream capture.  `out` must be given.  Device-side errors (range, timeout) are
+    reported by check_device_error, which reads the array's error word.
     """
     dev = q.device
     for t, n, dt in ((q, "q", torch.bfloat16), (k_pages, "k_pages", torch.bfloat16),

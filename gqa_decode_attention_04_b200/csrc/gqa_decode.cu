@@ -67,6 +67,13 @@ struct DeviceState {
 std::mutex g_mu;
 std::unordered_map<int, DeviceState> g_states;
 
+// The state of the current device if a call has set it up already (never creates it).
+DeviceState* existing_state(int dev) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  auto it = g_states.find(dev);
+  return (it == g_states.end() || it->second.err == nullptr) ? nullptr : &it->second;
+}
+
 gqa_status get_state(DeviceState** out, int* dev_out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -266,11 +273,22 @@ gqa_status noalloc_scratch(int dev, unsigned char** ptr, int* sms) {
     int n = 0;
     e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    // The error word starts at zero; after this it is cleared only when
+    // gqa_check_device_error reads it, so errors of any call stay visible until then.
+    e = cudaMemset(addr, 0, kNoAllocHeaderBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(allocation-free error word)");
     it = g_noalloc_dev.emplace(dev, std::make_pair(static_cast<unsigned char*>(addr), n)).first;
   }
   *ptr = it->second.first;
   *sms = it->second.second;
   return GQA_OK;
+}
+
+// The scratch address of a device whose allocation-free set-up has run, else nullptr.
+unsigned char* noalloc_scratch_if_set_up(int dev) {
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  auto it = g_noalloc_dev.find(dev);
+  return it == g_noalloc_dev.end() ? nullptr : it->second.first;
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t{255}; }
@@ -584,9 +602,10 @@ gqa_status gqa_paged_decode_attn_noalloc(const void* q, const void* k_pages, con
   unsigned char* part_o = part_ml + align256(slots * plan.heads_per_seg * 2 * sizeof(float));
   if (part_o + slots * plan.heads_per_seg * head_dim * sizeof(float) > scratch + kNoAllocScratchBytes)
     return fail(GQA_ERR_UNSUPPORTED, "allocation-free scratch layout does not fit");
-  // The array keeps the previous call's contents: the error word and the arrival
-  // counters must start at zero.
-  e = cudaMemsetAsync(scratch, 0, kNoAllocHeaderBytes + segments * sizeof(int32_t), strm);
+  // The array keeps the previous call's contents: the arrival counters must start at
+  // zero (a call that timed out may leave them set).  The error word is not cleared
+  // here: it accumulates until gqa_check_device_error reads and clears it.
+  e = cudaMemsetAsync(counters, 0, segments * sizeof(int32_t), strm);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(allocation-free scratch)");
 
 
@@ -626,18 +645,40 @@ gqa_status gqa_check_device_error(void* stream) {
   cudaStream_t strm = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaStreamSynchronize(strm);
   if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
-  DeviceState* st;
-  int dev;
-  gqa_status s = get_state(&st, &dev);
-  if (s != GQA_OK) return s;
+  int dev = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  // Two error words may exist on this device: the workspace's (every call but the
+  // allocation-free decode) and the one in the allocation-free call's fixed array.
+  // Only words that calls have set up are read; nothing is allocated here.
   uint32_t word = 0;
-  e = cudaMemcpy(&word, st->err, sizeof(word), cudaMemcpyDeviceToHost);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(error word)");
+  DeviceState* st = existing_state(dev);
+  if (st != nullptr) {
+    uint32_t w = 0;
+    e = cudaMemcpy(&w, st->err, sizeof(w), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(error word)");
+    if (w != 0) {
+      e = cudaMemset(st->err, 0, sizeof(uint32_t));
+      if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(error word)");
+    }
+    word |= w;
+  }
+  unsigned char* na = noalloc_scratch_if_set_up(dev);
+  if (na != nullptr) {
+    uint32_t w = 0;
+    e = cudaMemcpy(&w, na, sizeof(w), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy(allocation-free error word)");
+    if (w != 0) {
+      e = cudaMemset(na, 0, sizeof(uint32_t));
+      if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(allocation-free error word)");
+    }
+    word |= w;
+  }
   if (word == 0) return GQA_OK;
-  e = cudaMemset(st->err, 0, sizeof(uint32_t));
-  if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(error word)");
   if (word & gqa::kErrTimeout) {
-    {
+    // A timed-out launch may leave workspace arrival counters set (the allocation-free
+    // call clears its own at every call).
+    if (st != nullptr) {
       std::lock_guard<std::mutex> lk(g_mu);
       if (st->counters) cudaMemset(st->counters, 0, st->counters_cap * sizeof(int32_t));
     }

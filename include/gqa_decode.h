@@ -201,9 +201,11 @@ gqa_status gqa_multi_query_step(const void* q, const void* k_new, const void* v_
  *     holds 8 or 16 query heads for groups up to 16, up to 128 otherwise); when the
  *     split partials of the default number of workers do not fit, fewer workers are
  *     used.  A call beyond the limits returns GQA_ERR_UNSUPPORTED and launches nothing.
- *   - Device-side range errors (bad page ids, lengths) are skipped as in
- *     gqa_paged_decode_attn but recorded only in the array, so
- *     gqa_check_device_error does not report them.
+ *   - Device-side errors (bad page ids or lengths, a bounded wait that ran out) skip
+ *     the offending work as in gqa_paged_decode_attn and set an error word kept in the
+ *     array itself.  The word accumulates across calls until gqa_check_device_error,
+ *     which reads and clears it together with the regular one (with cudaMemcpy and
+ *     cudaMemset on the array: that call allocates nothing either).
  */
 gqa_status gqa_paged_decode_attn_noalloc(const void* q, const void* k_pages, const void* v_pages,
                                          const int32_t* block_table, const int32_t* seq_lens,
@@ -213,9 +215,11 @@ gqa_status gqa_paged_decode_attn_noalloc(const void* q, const void* k_pages, con
 
 /*
  * gqa_check_device_error -- synchronise `stream`, then read and clear the current
- * device's error word.  Returns GQA_OK, GQA_ERR_DEVICE_BOUNDS, GQA_ERR_TIMEOUT (takes
- * precedence when both are set; it also resets the decode workspace counters a
- * timed-out launch may have left behind) or GQA_ERR_CUDA.
+ * device's error words: the workspace's (every call but the allocation-free decode) and
+ * the allocation-free decode's own, each only if a call has set it up on this device
+ * (this call creates and allocates nothing).  Returns GQA_OK, GQA_ERR_DEVICE_BOUNDS,
+ * GQA_ERR_TIMEOUT (takes precedence when both are set; it also resets the decode
+ * workspace counters a timed-out launch may have left behind) or GQA_ERR_CUDA.
  */
 gqa_status gqa_check_device_error(void* stream);
 

@@ -73,6 +73,91 @@ def test_noalloc_with_many_split_workers(cuda_device):
         gq.set_num_workers(0)
 
 
+def test_noalloc_fit_limit_caps_forced_workers(cuda_device):
+    """With 128 query heads per kv head each worker's two partial slots take
+    2 x 128 x (128 + 2) floats, so the fixed 16 MiB array holds about 125 workers; 1000
+    forced workers (fewer than the 1250 blocks of work) must be cut to what fits, and the
+    result must still agree with the regular entry point and the oracle."""
+    lens = [40000, 40000]
+    inp = make_custom_inputs(lens, 128, 1, 128, 64, seed=8, extra_pages=1)
+    d = inp.to(cuda_device)
+    per_worker = 2 * 128 * (128 + 2) * 4 + 512
+    assert (16 << 20) // per_worker < 1000 <= sum((L + 63) // 64 for L in lens)
+    try:
+        gq.set_num_workers(1000)
+        ref = gq.paged_decode_attn(d.q, d.k_pages, d.v_pages, d.block_table, d.seq_lens, scale=d.scale)
+        gq.check_device_error()
+        out = torch.full_like(ref, float("nan"))
+        assert _noalloc_c_abi(d, out) == 0, gq.load_library().gqa_last_error_string()
+        gq.check_device_error()
+    finally:
+        gq.set_num_workers(0)
+    assert_close(gpu_f64(out), gpu_f64(ref), what="fit-limited workers vs regular")
+    assert_close(gpu_f64(out), oracle_out(host_arrays(inp)), what="fit-limited workers vs oracle")
+
+
+def test_noalloc_reports_device_errors(cuda_device):
+    """A bad page id and a wait that runs out are reported by check_device_error through
+    the fixed array's error word; a normal call afterwards is right again."""
+    inp = make_custom_inputs([300, 90], 16, 4, 128, 16, seed=9)
+    d = inp.to(cuda_device)
+    out = torch.empty((2, 16, 128), dtype=torch.bfloat16, device=cuda_device)
+    gq.check_device_error()  # nothing pending
+    bt = d.block_table.clone()
+    bt[0, 3] = 10 ** 6
+    gq.paged_decode_attn_noalloc(d.q, d.k_pages, d.v_pages, bt, d.seq_lens, out, scale=d.scale)
+    with pytest.raises(gq.GQAError) as ei:
+        gq.check_device_error()
+    assert ei.value.status == -4
+    gq.check_device_error()  # the word was cleared by the read
+    for H, Hk, ps in ((16, 4, 16), (96, 1, 64)):  # both decode kernels
+        inp = make_custom_inputs([700, 90], H, Hk, 128, ps, seed=10 + H)
+        d = inp.to(cuda_device)
+        out = torch.empty((2, H, 128), dtype=torch.bfloat16, device=cuda_device)
+        try:
+            gq.set_num_workers(12)
+            gq.set_wait_limit_ns(2_000_000, arm_without_copy=True)
+            gq.paged_decode_attn_noalloc(d.q, d.k_pages, d.v_pages, d.block_table, d.seq_lens, out,
+                                         scale=d.scale)
+            with pytest.raises(gq.GQAError) as ei:
+                gq.check_device_error()
+            assert ei.value.status == -5
+        finally:
+            gq.set_wait_limit_ns(10 ** 9, False)
+        try:
+            gq.paged_decode_attn_noalloc(d.q, d.k_pages, d.v_pages, d.block_table, d.seq_lens, out,
+                                         scale=d.scale)
+            gq.check_device_error()
+        finally:
+            gq.set_num_workers(0)
+        assert_close(gpu_f64(out), oracle_out(host_arrays(inp)), what=f"after timeout H={H}")
+
+
+def test_noalloc_allocates_no_device_memory(cuda_device):
+    """Free device memory is unchanged across a call with more segments and workers than
+    any earlier call of this process (so a regular workspace would have had to grow)."""
+    small = make_custom_inputs([100, 60], 32, 8, 128, 16, seed=11).to(cuda_device)
+    big_lens = [64] * 2000  # 2000 sequences x 8 kv heads = 16000 segments
+    big = make_custom_inputs(big_lens, 32, 8, 128, 16, seed=12, poison=False).to(cuda_device)
+    out_s = torch.empty((2, 32, 128), dtype=torch.bfloat16, device=cuda_device)
+    out_b = torch.empty((2000, 32, 128), dtype=torch.bfloat16, device=cuda_device)
+    # first call on the device (the set-up) and module loading happen before measuring
+    assert _noalloc_c_abi(small, out_s) == 0
+    gq.check_device_error()
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    try:
+        gq.set_num_workers(5000)
+        for _ in range(2):
+            assert _noalloc_c_abi(big, out_b) == 0, gq.load_library().gqa_last_error_string()
+        gq.check_device_error()
+        torch.cuda.synchronize()
+    finally:
+        gq.set_num_workers(0)
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0, (free0, free1)
+
+
 def test_noalloc_rejects_sizes_beyond_its_limit(cuda_device):
     # 4097 sequences x 4 kv heads = 16388 segments > 16384: refused before any launch
     lib = gq.load_library()
