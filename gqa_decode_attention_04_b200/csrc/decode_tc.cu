@@ -440,6 +440,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
     // S_n = Q K_n^T into TMEM buffer n % kTcBufs once block n's K has landed and the P V of
     // block n - kTcBufs (issued by the P V warp, reading P from the same buffer) is complete.
     constexpr uint32_t idS = ptx::umma_idesc_bf16(kTcRows, kTcBlk, false);
+    bool issued = false;  // a tcgen05.commit is only used to track MMAs this warp issued
     for (int64_t n = 0; n < total; ++n) {
       if (__any_sync(0xffffffffu, aborted())) break;  // warp-uniform
       const int stage = static_cast<int>(n % S);
@@ -467,10 +468,15 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
         ptx::umma_commit(sfull_bar + 8 * sb);
         if (si.flags & kTcLast) ptx::umma_commit(qempty_bar);  // Q tile no longer read
       }
+      issued = true;
       __syncwarp();
     }
-    // Every MMA issued by this warp completes before TMEM can be released.
-    if (lane == 0) ptx::umma_commit(drain_bar);
+    // Every MMA issued by this warp completes before TMEM can be released.  A warp that
+    // issued none (its first wait ran out) arrives directly.
+    if (lane == 0) {
+      if (issued) ptx::umma_commit(drain_bar);
+      else ptx::mbar_arrive(drain_bar);
+    }
     __syncwarp();
     ptx::mbar_wait_bounded(drain_bar, 0, limit);
   } else if (warp == kWarpPV) {
@@ -478,6 +484,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
     // O += P_m V_m as soon as the softmax has written P_m (and, at a piece start, has read
     // the previous piece's O out).
     constexpr uint32_t idPV = ptx::umma_idesc_bf16(kTcRows, D, true);
+    bool issued = false;
     for (int64_t m = 0; m < total; ++m) {
       if (__any_sync(0xffffffffu, aborted())) break;  // warp-uniform
       const int k = static_cast<int>(m % kTcBufs);
@@ -523,9 +530,13 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
         ptx::umma_commit(empty_bar + 8 * stage);  // K_m and V_m are consumed
         ptx::umma_commit(pv_bar + 8 * k);
       }
+      issued = true;
       __syncwarp();
     }
-    if (lane == 0) ptx::umma_commit(drain_bar);
+    if (lane == 0) {
+      if (issued) ptx::umma_commit(drain_bar);
+      else ptx::mbar_arrive(drain_bar);
+    }
     __syncwarp();
     ptx::mbar_wait_bounded(drain_bar, 0, limit);
   } else {
