@@ -26,4 +26,8 @@ from .fp8_cache import (  # noqa: F401
     quantize_pages,
     dequantize_pages,
     paged_decode_attention_fp8,
+    paged_decode_attention_fp8_rows,
+    encode_fp32_quotient,
+    quantize_bf16_pages,
+    kv_append_fp8,
 )

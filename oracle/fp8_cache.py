@@ -18,7 +18,12 @@ Readings where the pages are silent (restated in the design notes):
   * K and V each carry one float scale per kv head (a per-tensor scale is the case of
     equal scales); a cached value is decode(code) * scale;
   * writing a value x stores the code nearest to x / scale, ties to the even code, and
-    magnitudes beyond the format saturate to +-448 (not NaN).
+    magnitudes beyond the format saturate to +-448 (not NaN);
+  * when bf16 values are written into the cache (kv_append, or converting a whole bf16
+    pool), the quotient x / scale is formed in IEEE fp32 (round to nearest even) and the
+    code is the one nearest to that fp32 quotient: a quantised code is an integer decided
+    by floating point, so the oracle takes that decision in the precision the kernels
+    use.  A NaN input gives a NaN code.
 """
 from __future__ import annotations
 
@@ -35,6 +40,10 @@ __all__ = [
     "quantize_pages",
     "dequantize_pages",
     "paged_decode_attention_fp8",
+    "paged_decode_attention_fp8_rows",
+    "encode_fp32_quotient",
+    "quantize_bf16_pages",
+    "kv_append_fp8",
 ]
 
 E4M3_MAX = 448.0
@@ -106,3 +115,57 @@ def paged_decode_attention_fp8(q_bits, k_codes, v_codes, k_scales, v_scales, blo
             kvh = kv_head_of(h, H, Hk)
             out[b, h] = attend_one_query(q[b, h], K[page, kvh, slot, :], V[page, kvh, slot, :], scale)
     return out
+
+
+def paged_decode_attention_fp8_rows(q_bits, k_codes, v_codes, k_scales, v_scales, block_table,
+                                    seq_lens, scale: float, rows) -> np.ndarray:
+    """The same attention for selected (b, h) rows only, decoding just the codes those rows
+    read (full-size pools hold billions of codes).  Returns [len(rows), D]."""
+    Hk, ps = k_codes.shape[1], k_codes.shape[2]
+    H = q_bits.shape[1]
+    q = bf16_bits_to_f64(q_bits)
+    out = np.zeros((len(rows), q_bits.shape[2]), dtype=np.float64)
+    for i, (b, h) in enumerate(rows):
+        L = int(seq_lens[b])
+        t = np.arange(L, dtype=np.int64)
+        page = np.asarray(block_table[b], dtype=np.int64)[t // ps]
+        slot = t % ps
+        kvh = kv_head_of(h, H, Hk)
+        K = e4m3_bits_to_f64(k_codes[page, kvh, slot, :]) * float(k_scales[kvh])
+        V = e4m3_bits_to_f64(v_codes[page, kvh, slot, :]) * float(v_scales[kvh])
+        out[i] = attend_one_query(q[b, h], K, V, scale)
+    return out
+
+
+def encode_fp32_quotient(x, scale) -> np.ndarray:
+    """Codes of x / scale: the quotient in IEEE fp32 (x and scale as fp32, round to nearest
+    even), then the e4m3 code nearest to that fp32 value (f64_to_e4m3_bits)."""
+    quotient = np.asarray(x, dtype=np.float32) / np.asarray(scale, dtype=np.float32)
+    return f64_to_e4m3_bits(quotient.astype(np.float64))
+
+
+def quantize_bf16_pages(pages_bits, scales) -> np.ndarray:
+    """Codes of a bf16 pool [P, Hk, ps, D] (raw bits) with one fp32 scale per kv head:
+    element [p, kvh, t, d] becomes encode_fp32_quotient(x, scales[kvh])."""
+    x = bf16_bits_to_f64(pages_bits)
+    s = np.asarray(scales, dtype=np.float32)[None, :, None, None]
+    return encode_fp32_quotient(x, np.broadcast_to(s, x.shape))
+
+
+def kv_append_fp8(k_codes, v_codes, k_new_bits, v_new_bits, k_scales, v_scales, block_table,
+                  positions):
+    """kv_append into a coded cache: the slot of position positions[b] of sequence b takes
+    the codes of k_new[b, kvh, :] / k_scales[kvh] (V likewise with v_scales); every other
+    byte is unchanged.  k_new, v_new [B, Hk, D] are bf16 bits; returns new (K, V) pools."""
+    kc = np.array(k_codes, dtype=np.uint8, copy=True)
+    vc = np.array(v_codes, dtype=np.uint8, copy=True)
+    ps = kc.shape[2]
+    ks = np.asarray(k_scales, dtype=np.float32)[:, None]
+    vs = np.asarray(v_scales, dtype=np.float32)[:, None]
+    for b in range(len(positions)):
+        pos = int(positions[b])
+        page = int(block_table[b][pos // ps])
+        slot = pos % ps
+        kc[page, :, slot, :] = encode_fp32_quotient(bf16_bits_to_f64(k_new_bits[b]), np.broadcast_to(ks, kc.shape[1:2] + kc.shape[3:]))
+        vc[page, :, slot, :] = encode_fp32_quotient(bf16_bits_to_f64(v_new_bits[b]), np.broadcast_to(vs, vc.shape[1:2] + vc.shape[3:]))
+    return kc, vc

@@ -509,6 +509,97 @@ def check_fp8_quantization_error_bound():
     assert np.all(np.abs(y - x)[sub] <= 2.0 ** -10 * np.broadcast_to(s[None, :, None, None], x.shape)[sub])
 
 
+def check_fp8_encode_of_the_fp32_quotient():
+    """Writing bf16 values into the coded cache: the code of x / scale is decided on the
+    IEEE fp32 quotient.  torch's fp32 division followed by its float8_e4m3fn cast (a
+    library routine) gives the same codes below the overflow midpoint; 41 / fp32(6.56)
+    is exactly 6.25 in fp32, a tie that goes to the even code 0x4C, while the fp64
+    quotient lies just above the tie (code 0x4D); NaN gives a NaN code."""
+    rng = np.random.default_rng(27)
+    x = PA.bf16_bits_to_f64(_rand_bits(rng, 6000, scale=30.0))
+    sc = rng.uniform(0.01, 4.0, 6000).astype(np.float32)
+    got = F8.encode_fp32_quotient(x, sc)
+    qt = torch.from_numpy(x.astype(np.float32)) / torch.from_numpy(sc)
+    ok = qt.abs() < 464.0
+    ref = qt[ok].to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(got[ok.numpy()], ref)
+    sat = (~ok).numpy()
+    assert np.all((got[sat] & 0x7F) == 0x7E) and np.array_equal(got[sat] >> 7, (x[sat] < 0).astype(np.uint8))
+    s656 = np.float32(6.56)
+    assert F8.encode_fp32_quotient([41.0], s656)[0] == 0x4C
+    assert F8.f64_to_e4m3_bits([41.0 / float(s656)])[0] == 0x4D
+    c = F8.encode_fp32_quotient([np.nan, -0.0, 0.0], np.float32(1.0))
+    assert (c[0] & 0x7F) == 0x7F and c[1] == 0x80 and c[2] == 0x00
+
+
+def check_fp8_quantize_bf16_pool_per_kv_head():
+    """A whole bf16 pool becomes codes with its own kv head's scale: every element's code
+    is the fp32-quotient encode with scales[kvh] (kv heads on axis 1 of [P, Hk, ps, D]),
+    and decoding gives the value back within half a step."""
+    rng = np.random.default_rng(28)
+    P_, Hk, ps, D = 5, 3, 16, 8
+    mags = np.array([0.05, 1.0, 40.0])
+    bits = PA.f64_to_bf16_bits(rng.standard_normal((P_, Hk, ps, D)) * mags[None, :, None, None])
+    x = PA.bf16_bits_to_f64(bits)
+    scales = (np.abs(x).max(axis=(0, 2, 3)) / 448.0).astype(np.float32)
+    codes = F8.quantize_bf16_pages(bits, scales)
+    assert codes.shape == bits.shape and codes.dtype == np.uint8
+    for kvh in range(Hk):
+        want = F8.encode_fp32_quotient(x[:, kvh], np.float32(scales[kvh]))
+        assert np.array_equal(codes[:, kvh], want)
+    y = F8.dequantize_pages(codes, scales.astype(np.float64))
+    r = np.abs(x) / scales.astype(np.float64)[None, :, None, None]
+    normal = r >= 2.0 ** -6
+    assert np.all(np.abs(y - x)[normal] <= 2.0 ** -4 * np.abs(x)[normal] * (1 + 2.0 ** -20))
+    assert np.abs(F8.e4m3_bits_to_f64(codes)).max() == 448.0  # the largest magnitude maps to the top code
+
+
+def check_kv_append_fp8():
+    """The coded append writes exactly the target slot of every sequence -- K with the K
+    scales, V with the V scales -- and leaves every other byte of both pools unchanged."""
+    rng = np.random.default_rng(29)
+    B, Hk, D, ps, P_ = 3, 2, 8, 16, 7
+    kc = rng.integers(0, 256, (P_, Hk, ps, D), dtype=np.uint8)
+    vc = rng.integers(0, 256, (P_, Hk, ps, D), dtype=np.uint8)
+    bt = np.array([[4, 1, -1], [0, -1, -1], [6, 2, 5]])
+    pos = np.array([17, 3, 40])
+    kn = _rand_bits(rng, (B, Hk, D), scale=3.0)
+    vn = _rand_bits(rng, (B, Hk, D), scale=0.2)
+    ks = np.array([0.05, 0.5], dtype=np.float32)     # no appended value saturates
+    vs = np.array([0.004, 0.03], dtype=np.float32)
+    k2, v2 = F8.kv_append_fp8(kc, vc, kn, vn, ks, vs, bt, pos)
+    touched = np.zeros(kc.shape, dtype=bool)
+    for b in range(B):
+        page, slot = bt[b][pos[b] // ps], pos[b] % ps
+        touched[page, :, slot, :] = True
+        for kvh in range(Hk):
+            assert np.array_equal(k2[page, kvh, slot], F8.encode_fp32_quotient(PA.bf16_bits_to_f64(kn[b, kvh]), ks[kvh]))
+            assert np.array_equal(v2[page, kvh, slot], F8.encode_fp32_quotient(PA.bf16_bits_to_f64(vn[b, kvh]), vs[kvh]))
+    assert np.array_equal(k2[~touched], kc[~touched]) and np.array_equal(v2[~touched], vc[~touched])
+    # the appended rows read back within half a step of the bf16 values
+    for b in range(B):
+        page, slot = bt[b][pos[b] // ps], pos[b] % ps
+        y = F8.e4m3_bits_to_f64(k2[page, :, slot, :]) * ks[:, None]
+        xk = PA.bf16_bits_to_f64(kn[b])
+        assert np.all(np.abs(y - xk) <= 2.0 ** -4 * np.abs(xk) * (1 + 2.0 ** -20) + 2.0 ** -10 * ks[:, None])
+
+
+def check_fp8_rows_match_full():
+    """The row-subset attention over a coded cache equals the full one on those rows."""
+    rng = np.random.default_rng(30)
+    sl = [40, 3, 70]
+    H, Hk, D, ps = 6, 2, 8, 16
+    q, kp, vp, bt, _, _ = _random_paged(rng, sl, H, Hk, D, ps)
+    ks = np.array([0.01, 0.02], dtype=np.float32)
+    vs = np.array([0.005, 0.04], dtype=np.float32)
+    kc = F8.quantize_bf16_pages(kp, ks)
+    vc = F8.quantize_bf16_pages(vp, vs)
+    full = F8.paged_decode_attention_fp8(q, kc, vc, ks, vs, bt, np.array(sl), 0.4)
+    rows = [(0, 5), (2, 0), (1, 3), (2, 4)]
+    got = F8.paged_decode_attention_fp8_rows(q, kc, vc, ks, vs, bt, np.array(sl), 0.4, rows)
+    assert np.allclose(got, np.stack([full[b, h] for b, h in rows]), rtol=0, atol=1e-13)
+
+
 ALL_CHECKS = [
     check_bf16_decode,
     check_closed_form_three_tokens,
@@ -534,4 +625,8 @@ ALL_CHECKS = [
     check_e4m3_encode_rounding_and_saturation,
     check_fp8_cache_attention_on_exact_values,
     check_fp8_quantization_error_bound,
+    check_fp8_encode_of_the_fp32_quotient,
+    check_fp8_quantize_bf16_pool_per_kv_head,
+    check_kv_append_fp8,
+    check_fp8_rows_match_full,
 ]

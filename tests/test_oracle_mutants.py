@@ -138,6 +138,33 @@ def _fp8_attention_swapped_scales(q, kc, vc, ks, vs, bt, sl, scale):
 
 _ORIG_FP8_ATTN = F8.paged_decode_attention_fp8
 
+def _encode_fp64_quotient(x, scale):
+    return F8.f64_to_e4m3_bits(np.asarray(x, dtype=np.float64) /
+                               np.asarray(scale, dtype=np.float32).astype(np.float64))  # fp64 quotient
+
+
+_ORIG_QUANT = F8.quantize_bf16_pages
+
+
+def _quantize_scale_by_page(pages_bits, scales):
+    s = np.asarray(scales, dtype=np.float32)
+    P_ = pages_bits.shape[0]
+    per_page = np.resize(s, P_)[:, None, None, None]          # scale indexed by page, not kv head
+    x = PA.bf16_bits_to_f64(pages_bits)
+    return F8.encode_fp32_quotient(x, np.broadcast_to(per_page, x.shape))
+
+
+_ORIG_APPEND8 = F8.kv_append_fp8
+
+
+def _append_fp8_swapped_scales(kc, vc, kn, vn, ks, vs, bt, pos):
+    return _ORIG_APPEND8(kc, vc, kn, vn, vs, ks, bt, pos)       # K and V scales swapped
+
+
+def _append_fp8_next_slot(kc, vc, kn, vn, ks, vs, bt, pos):
+    return _ORIG_APPEND8(kc, vc, kn, vn, ks, vs, bt, np.asarray(pos) + 1)  # one slot late
+
+
 MUTANTS = [
     ("kv_head_of", _kv_head_modulo),
     ("gather_sequence_kv", _gather_swapped),
@@ -155,6 +182,10 @@ MUTANTS = [
     ("F8:e4m3_bits_to_f64", _e4m3_bias8),
     ("F8:f64_to_e4m3_bits", _e4m3_truncating),
     ("F8:paged_decode_attention_fp8", _fp8_attention_swapped_scales),
+    ("F8:encode_fp32_quotient", _encode_fp64_quotient),
+    ("F8:quantize_bf16_pages", _quantize_scale_by_page),
+    ("F8:kv_append_fp8", _append_fp8_swapped_scales),
+    ("F8:kv_append_fp8", _append_fp8_next_slot),
 ]
 
 
