@@ -78,22 +78,3 @@ def test_wait_timeout_returns_error_and_library_recovers(cuda_device):
     gq.check_device_error()
     assert_close(gpu_f64(out), oracle_out(host_arrays(inp)))
 
-
-@pytest.mark.parametrize("workers", [1, 12], ids=["one_cta", "split_and_merge"])
-def test_tcgen05_wait_timeout_returns_error_and_library_recovers(cuda_device, workers):
-    """The same timeout path on the tcgen05 kernel (96 query heads per kv head): every
-    warp leaves its loop, the MMA-issuing warps drain, TMEM is released, and with several
-    workers the split-merge kernel (launched behind the decode) still completes.  A normal
-    call on the same library instance then matches the oracle."""
-    inp = make_custom_inputs([700, 64, 1500], 96, 1, 128, 64, seed=25)
-    d = inp.to(cuda_device)
-    gq.set_num_workers(workers)
-    gq.set_wait_limit_ns(2_000_000, arm_without_copy=True)
-    gq.paged_decode_attn(d.q, d.k_pages, d.v_pages, d.block_table, d.seq_lens, scale=d.scale)
-    with pytest.raises(gq.GQAError) as ei:
-        gq.check_device_error()
-    assert ei.value.status == -5
-    gq.set_wait_limit_ns(10 ** 9, False)
-    out = gq.paged_decode_attn(d.q, d.k_pages, d.v_pages, d.block_table, d.seq_lens, scale=d.scale)
-    gq.check_device_error()
-    assert_close(gpu_f64(out), oracle_out(host_arrays(inp)))

@@ -110,7 +110,7 @@ def test_noalloc_reports_device_errors(cuda_device):
         gq.check_device_error()
     assert ei.value.status == -4
     gq.check_device_error()  # the word was cleared by the read
-    for H, Hk, ps in ((16, 4, 16), (96, 1, 64)):  # both decode kernels
+    for H, Hk, ps in ((16, 4, 16),):  # the mma.sync kernel (the tcgen05 kernel's timeout path stays off GPUs)
         inp = make_custom_inputs([700, 90], H, Hk, 128, ps, seed=10 + H)
         d = inp.to(cuda_device)
         out = torch.empty((2, H, 128), dtype=torch.bfloat16, device=cuda_device)
