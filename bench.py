@@ -479,8 +479,11 @@ def measure_workload(gq, inp_dev, dev, peak, clocks, fp8: bool):
         "tokens_per_s": B / (s_med * 1e-6),
         "l2": l2_desc, "graph_launches": GRAPH_LAUNCHES,
     }
-    if fp8 and hasattr(gq, "paged_decode_attn_fp8"):
-        entry["fp8"] = measure_fp8(gq, sets, dev, peak, clocks)
+    if fp8:
+        try:
+            entry["fp8"] = measure_fp8(gq, sets, dev, peak, clocks)
+        except gq.GQAError as e:  # a shape the 8-bit path does not serve
+            entry["fp8"] = {"unavailable": str(e)}
     del sets, out
     return entry
 

@@ -25,6 +25,10 @@ __all__ = [
     "paged_decode_attn",
     "decode_step",
     "paged_decode_attn_noalloc",
+    "quantize_pages_fp8",
+    "kv_append_fp8",
+    "paged_decode_attn_fp8",
+    "decode_step_fp8",
     "kv_append_multi",
     "paged_multi_query_attn",
     "multi_query_step",
@@ -51,6 +55,10 @@ EXPORTED_SYMBOLS = (
     "gqa_paged_decode_attn",
     "gqa_decode_step",
     "gqa_paged_decode_attn_noalloc",
+    "gqa_kv_quantize_fp8",
+    "gqa_kv_append_fp8",
+    "gqa_paged_decode_attn_fp8",
+    "gqa_decode_step_fp8",
     "gqa_kv_append_multi",
     "gqa_paged_multi_query_attn",
     "gqa_multi_query_step",
@@ -108,6 +116,16 @@ def load_library() -> ctypes.CDLL:
     lib.gqa_decode_step.restype = i32
     lib.gqa_paged_decode_attn_noalloc.argtypes = lib.gqa_paged_decode_attn.argtypes
     lib.gqa_paged_decode_attn_noalloc.restype = i32
+    lib.gqa_kv_quantize_fp8.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp]
+    lib.gqa_kv_quantize_fp8.restype = i32
+    lib.gqa_kv_append_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, vp]
+    lib.gqa_kv_append_fp8.restype = i32
+    lib.gqa_paged_decode_attn_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32,
+                                              i32, i32, vp]
+    lib.gqa_paged_decode_attn_fp8.restype = i32
+    lib.gqa_decode_step_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32,
+                                        i32, i32, vp]
+    lib.gqa_decode_step_fp8.restype = i32
     lib.gqa_kv_append_multi.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, i32, vp]
     lib.gqa_kv_append_multi.restype = i32
     lib.gqa_paged_multi_query_attn.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32, f32,
@@ -389,6 +407,109 @@ def paged_decode_attn_noalloc(q, k_pages, v_pages, block_table, seq_lens, out: t
             q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(), block_table.data_ptr(),
             seq_lens.data_ptr(), out.data_ptr(), B, H, Hk, D, ps, float(scale),
             block_table.shape[1], P, _stream_ptr(stream)))
+    return out
+
+
+def _pools_fp8(k_pages, v_pages, k_scales, v_scales, dev):
+    for t, n, dt in ((k_pages, "k_pages", torch.uint8), (v_pages, "v_pages", torch.uint8),
+                     (k_scales, "k_scales", torch.float32), (v_scales, "v_scales", torch.float32)):
+        _need(t, n, dt, dev)
+    if k_pages.dim() != 4 or tuple(v_pages.shape) != tuple(k_pages.shape):
+        raise ValueError("e4m3 pools must both be [num_pages, num_kv_heads, page_size, head_dim] uint8")
+    P, Hk, ps, D = k_pages.shape
+    if tuple(k_scales.shape) != (Hk,) or tuple(v_scales.shape) != (Hk,):
+        raise ValueError("k_scales / v_scales must be [num_kv_heads] float32")
+    return P, Hk, ps, D
+
+
+def quantize_pages_fp8(src, dst, scales, stream=None) -> torch.Tensor:
+    """e4m3 codes of a bf16 pool: dst[p, kvh] = code of src[p, kvh] / scales[kvh]."""
+    dev = src.device
+    _need(src, "src", torch.bfloat16, dev)
+    _need(dst, "dst", torch.uint8, dev)
+    _need(scales, "scales", torch.float32, dev)
+    if src.dim() != 4 or tuple(dst.shape) != tuple(src.shape):
+        raise ValueError("src and dst must both be [num_pages, num_kv_heads, page_size, head_dim]")
+    P, Hk, ps, D = src.shape
+    if tuple(scales.shape) != (Hk,):
+        raise ValueError("scales must be [num_kv_heads] float32")
+    with torch.cuda.device(dev):
+        _check(load_library().gqa_kv_quantize_fp8(src.data_ptr(), dst.data_ptr(), scales.data_ptr(), P, Hk, ps, D,
+                                                  _stream_ptr(stream)))
+    return dst
+
+
+def kv_append_fp8(k_new, v_new, k_pages, v_pages, k_scales, v_scales, block_table, positions,
+                  stream=None) -> None:
+    """Write k_new/v_new [B, Hk, D] (bf16) into the e4m3 pools at positions[b]."""
+    dev = k_pages.device
+    P, Hk, ps, D = _pools_fp8(k_pages, v_pages, k_scales, v_scales, dev)
+    for t, n, dt in ((k_new, "k_new", torch.bfloat16), (v_new, "v_new", torch.bfloat16),
+                     (block_table, "block_table", torch.int32), (positions, "positions", torch.int32)):
+        _need(t, n, dt, dev)
+    B = k_new.shape[0]
+    if tuple(k_new.shape) != (B, Hk, D) or tuple(v_new.shape) != (B, Hk, D):
+        raise ValueError("k_new / v_new must be [num_seqs, num_kv_heads, head_dim]")
+    if block_table.dim() != 2 or block_table.shape[0] != B or tuple(positions.shape) != (B,):
+        raise ValueError("block_table must be [num_seqs, max_blocks], positions [num_seqs]")
+    with torch.cuda.device(dev):
+        _check(load_library().gqa_kv_append_fp8(
+            k_new.data_ptr(), v_new.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(), k_scales.data_ptr(),
+            v_scales.data_ptr(), block_table.data_ptr(), positions.data_ptr(), B, Hk, D, ps, block_table.shape[1], P,
+            _stream_ptr(stream)))
+
+
+def paged_decode_attn_fp8(q, k_pages, v_pages, k_scales, v_scales, block_table, seq_lens,
+                          out: Optional[torch.Tensor] = None, scale: Optional[float] = None,
+                          stream=None) -> torch.Tensor:
+    """paged_decode_attn over e4m3 pools (cached value = code * scale of its kv head)."""
+    dev = q.device
+    _need(q, "q", torch.bfloat16, dev)
+    P, Hk, ps, D = _pools_fp8(k_pages, v_pages, k_scales, v_scales, dev)
+    _need(block_table, "block_table", torch.int32, dev)
+    _need(seq_lens, "seq_lens", torch.int32, dev)
+    B, H, D2 = q.shape
+    if D2 != D:
+        raise ValueError("q's head_dim differs from the pools'")
+    if block_table.dim() != 2 or block_table.shape[0] != B or tuple(seq_lens.shape) != (B,):
+        raise ValueError("block_table must be [num_seqs, max_blocks], seq_lens [num_seqs]")
+    out = _multi_out(out, (B, H, D), dev)
+    if scale is None:
+        scale = 1.0 / (D ** 0.5)
+    with torch.cuda.device(dev):
+        _check(load_library().gqa_paged_decode_attn_fp8(
+            q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(), k_scales.data_ptr(), v_scales.data_ptr(),
+            block_table.data_ptr(), seq_lens.data_ptr(), out.data_ptr(), B, H, Hk, D, ps, float(scale),
+            block_table.shape[1], P, _stream_ptr(stream)))
+    return out
+
+
+def decode_step_fp8(q, k_new, v_new, k_pages, v_pages, k_scales, v_scales, block_table, positions, seq_lens,
+                    out: Optional[torch.Tensor] = None, scale: Optional[float] = None,
+                    stream=None) -> torch.Tensor:
+    """kv_append_fp8 of k_new/v_new at positions, then paged_decode_attn_fp8 (one call)."""
+    dev = q.device
+    _need(q, "q", torch.bfloat16, dev)
+    P, Hk, ps, D = _pools_fp8(k_pages, v_pages, k_scales, v_scales, dev)
+    for t, n, dt in ((k_new, "k_new", torch.bfloat16), (v_new, "v_new", torch.bfloat16),
+                     (block_table, "block_table", torch.int32), (positions, "positions", torch.int32),
+                     (seq_lens, "seq_lens", torch.int32)):
+        _need(t, n, dt, dev)
+    B, H, D2 = q.shape
+    if D2 != D or tuple(k_new.shape) != (B, Hk, D) or tuple(v_new.shape) != (B, Hk, D):
+        raise ValueError("q [B, H, D], k_new / v_new [B, Hk, D] must match the pools")
+    if (block_table.dim() != 2 or block_table.shape[0] != B or tuple(seq_lens.shape) != (B,)
+            or tuple(positions.shape) != (B,)):
+        raise ValueError("block_table must be [num_seqs, max_blocks]; seq_lens, positions [num_seqs]")
+    out = _multi_out(out, (B, H, D), dev)
+    if scale is None:
+        scale = 1.0 / (D ** 0.5)
+    with torch.cuda.device(dev):
+        _check(load_library().gqa_decode_step_fp8(
+            q.data_ptr(), k_new.data_ptr(), v_new.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(),
+            k_scales.data_ptr(), v_scales.data_ptr(), block_table.data_ptr(), positions.data_ptr(),
+            seq_lens.data_ptr(), out.data_ptr(), B, H, Hk, D, ps, float(scale), block_table.shape[1], P,
+            _stream_ptr(stream)))
     return out
 
 

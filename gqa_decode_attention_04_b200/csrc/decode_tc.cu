@@ -39,6 +39,11 @@
 //     stride is group x head_dim elements, one box per column group; each softmax thread
 //     masks its row's window (the sequence up to its own token) from the stage's
 //     remaining length, and tile rows past the group get an empty window.
+//   * 8-bit cache (the F8 instantiation): the producers copy each block's e4m3 codes into
+//     a ring of raw stages; two converter warps widen them (exactly) to fp16 in the stage
+//     layout the MMAs read, and convert each piece's query tile from bf16 to fp16 in
+//     place, so both MMAs run kind::f16 on fp16 operands (P is packed as fp16).  The kv
+//     head's K scale joins the score scale of a piece, its V scale the piece-end output.
 //   * Safety: every wait is bounded; on a timeout all warps leave their loops, the MMA
 //     warps wait for their issued MMAs, and TMEM is released before exit.
 #include <type_traits>
@@ -62,17 +67,26 @@ constexpr int kStgFloats = 16 * 36;  // piece-end staging per softmax warp
 constexpr int kTcWarps = 12;
 constexpr int kTcThreads = 32 * kTcWarps;
 constexpr int kWarpProducer = 8, kWarpS = 9, kWarpPV = 10, kWarpProducer2 = 11;
+// 8-bit cache: warps 12 and 13 convert codes (even and odd blocks).
+constexpr int kTcWarpsF8 = 14;
+constexpr int kTcThreadsF8 = 32 * kTcWarpsF8;
+constexpr int kWarpConv = 12;
 constexpr float kTcRescale = 8.0f;
 
-template <int D>
+template <int D, bool F8 = false>
 struct TcGeo {
   static constexpr int kGroups = D / 64;                 // 64-column (128-byte) groups
   static constexpr int kGroupBytes = kTcBlk * 128;       // 64 rows x 128 bytes
-  static constexpr int kTile = kGroups * kGroupBytes;    // K (or V) of one block
+  static constexpr int kTile = kGroups * kGroupBytes;    // K (or V) of one block (16-bit)
   static constexpr int kStage = 2 * kTile;
   static constexpr int kQGroup = kTcRows * 128;
   static constexpr int kQTile = kGroups * kQGroup;
-  static constexpr int kStages = D == 128 ? 5 : 10;
+  static constexpr int kStages = F8 ? (D == 128 ? 3 : 5) : (D == 128 ? 5 : 10);
+  // 8-bit cache: a block's codes (64 tokens x D bytes per tensor, as 128-byte swizzled
+  // rows) land in a ring of raw stages before the converters widen them.
+  static constexpr int kRawTile = kTcBlk * D;
+  static constexpr int kRawStage = 2 * kRawTile;
+  static constexpr int kRawStages = F8 ? (D == 128 ? 4 : 8) : 0;
   // TMEM columns: S/P buffer k at 64 k (64 fp32 columns each; the bf16 pairs of P of
   // tokens 0-31 overwrite columns 0-15, of tokens 32-63 columns 32-47), then one O
   // accumulator (D columns) per softmax warpgroup.
@@ -100,20 +114,30 @@ struct TcCursor {
 // MQ: several query tokens per sequence (p.q_len): a kv head's rows are its group of
 // heads for each query token in turn (row r: token r / group, head r % group), all in one
 // segment (at most 128 rows); row r sees the sequence up to its own token.
-template <int D, bool MQ>
-__global__ void __launch_bounds__(kTcThreads, 1)
+// F8: the cache holds e4m3 codes with one scale per kv head for K and for V.
+template <int D, bool MQ, bool F8 = false>
+__global__ void __launch_bounds__(F8 ? kTcThreadsF8 : kTcThreads, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                  const __grid_constant__ CUtensorMap tmap_q, const DecodeParams p) {
-  using GE = TcGeo<D>;
+  using GE = TcGeo<D, F8>;
   constexpr int S = GE::kStages;
+  constexpr int RS = GE::kRawStages;
+  constexpr int NW = F8 ? kTcWarpsF8 : kTcWarps;
+  static_assert(!(F8 && MQ), "the 8-bit cache serves one query token per sequence");
   extern __shared__ uint8_t smem_raw[];
-  __shared__ int64_t s_wtot[kTcWarps];
+  __shared__ int64_t s_wtot[NW];
   __shared__ float s_xmax[2][kTcRows];  // per-piece row references of each warpgroup
   __shared__ float s_xsum[2][kTcRows];  // per-piece row sums of each warpgroup
   __shared__ int s_start_b;
   __shared__ int64_t s_start_base;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
+  // Pieces whose query copy has been issued (producers) and, with the 8-bit cache,
+  // converted (converters).  A parity wait on an mbarrier is only exact if the waiter
+  // is at most one phase ahead; the two producers (and the two converters) take pieces
+  // in turns, so the one starting piece k first waits for these counters to show that
+  // piece k - 1 went through, which puts the barrier at most one phase behind.
+  __shared__ int s_qissued, s_qconverted;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int B = p.num_seqs;
@@ -143,10 +167,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
   if (threadIdx.x == 0) {
     s_start_b = -1;
     s_abort = 0;
+    s_qissued = 0;
+    s_qconverted = 0;
   }
   __syncthreads();
   int64_t T = 0;
-  for (int i = 0; i < kTcWarps; ++i) T += s_wtot[i];
+  for (int i = 0; i < NW; ++i) T += s_wtot[i];
   const int64_t W = min(static_cast<int64_t>(p.num_workers), T);
   const int64_t w = blockIdx.x;
   if (w >= W) return;
@@ -167,7 +193,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
       if (lane == 31) s_wtot[warp] = incl;
       __syncthreads();
       int64_t pre = 0, tot = 0;
-      for (int i = 0; i < kTcWarps; ++i) {
+      for (int i = 0; i < NW; ++i) {
         if (i < warp) pre += s_wtot[i];
         tot += s_wtot[i];
       }
@@ -190,10 +216,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
   const uint32_t pad = (1024u - (smem0 & 1023u)) & 1023u;
   uint8_t* base_ptr = smem_raw + pad;
   const uint32_t ring = smem0 + pad;                        // S stages of K | V
-  const uint32_t qbuf = ring + S * GE::kStage;              // Q tile of the current piece
+  const uint32_t raw = ring + S * GE::kStage;               // F8: RS raw stages of K | V codes
+  const uint32_t qbuf = raw + RS * GE::kRawStage;           // Q tile of the current piece
   uint8_t* vring = base_ptr;                                // generic view of the ring
-  TcStageInfo* info = reinterpret_cast<TcStageInfo*>(base_ptr + S * GE::kStage + GE::kQTile);
-  const uint32_t bar0 = ptx::smem_u32(info + S);
+  TcStageInfo* info = reinterpret_cast<TcStageInfo*>(base_ptr + S * GE::kStage + RS * GE::kRawStage + GE::kQTile);
+  TcStageInfo* rinfo = info + S;                            // F8: descriptors of the raw stages
+  const uint32_t bar0 = ptx::smem_u32(rinfo + RS);
   const uint32_t full_bar = bar0;                 // [S] producer -> MMA (K/V landed)
   const uint32_t empty_bar = full_bar + 8 * S;    // [S] MMA commit -> producer
   const uint32_t qfull_bar = empty_bar + 8 * S;   // producer -> S warp (piece k: phase k)
@@ -204,9 +232,13 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
   const uint32_t ofree_bar = pv_bar + 8 * kTcBufs;       // softmax (256) -> P V warp, a piece's O is read
   const uint32_t drain_bar = ofree_bar + 8;       // MMA commit at exit
   const uint32_t wg_bar = drain_bar + 8;          // rendezvous of both softmax warpgroups (256)
+  const uint32_t raw_full = wg_bar + 8;           // F8: [RS] producer -> converter (codes landed)
+  const uint32_t raw_empty = raw_full + 8 * RS;   // F8: [RS] converter -> producer
+  const uint32_t qconv_bar = raw_empty + 8 * RS;  // F8: converter -> S warp (piece k's Q in fp16: phase k)
+  const uint32_t bars_end = qconv_bar + (F8 ? 8 : 0);
   // Piece-end staging: per softmax warp 16 rows x 36 floats, so a warp writes whole
   // 128-byte row segments of its 32 rows (16 rows per round) instead of one row per lane.
-  float* const stg_all = reinterpret_cast<float*>(base_ptr + ((wg_bar + 8 - ring + 127u) & ~127u));
+  float* const stg_all = reinterpret_cast<float*>(base_ptr + ((bars_end - ring + 127u) & ~127u));
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -223,6 +255,13 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
     ptx::mbar_init(ofree_bar, kTcSoftThreads);
     ptx::mbar_init(drain_bar, 2);  // both MMA-issuing warps
     ptx::mbar_init(wg_bar, kTcSoftThreads);
+    if constexpr (F8) {
+      for (int s = 0; s < RS; ++s) {
+        ptx::mbar_init(raw_full + 8 * s, 1);
+        ptx::mbar_init(raw_empty + 8 * s, 1);
+      }
+      ptx::mbar_init(qconv_bar, 1);
+    }
     ptx::fence_mbarrier_init();
   }
   if (warp == kWarpS) ptx::tmem_alloc(ptx::smem_u32(&s_tmem), kTmemCols);
@@ -268,14 +307,20 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
     // A 64-row box carries every 64-column group at once (its shared-memory image is the
     // [group][64 rows][128 B] tile the MMAs read); shorter boxes carry one group each.
     const int box_groups = R == kTcBlk ? GE::kGroups : 1;
-    const int gsteps = GE::kGroups / box_groups;
+    // (8-bit cache: one box of R * D / 128 code rows carries a chunk's every column)
+    const int gsteps = F8 ? 1 : GE::kGroups / box_groups;
     const int nops = 2 * nchunks * gsteps;   // copies per block, one per lane
     // This lane's copy: tensor (K or V), chunk and column group.
     const int op_t = lane / (nchunks * gsteps);
     const int op_c = (lane % (nchunks * gsteps)) / gsteps;
     const int op_g = (lane % gsteps) * box_groups;
     const int cl = lane & (nchunks - 1);     // chunk whose page this lane tracks
-    const uint32_t tile_bytes = 2u * GE::kGroups * R * 128u;  // K + V bytes of one chunk
+    const uint32_t tile_bytes = F8 ? 2u * R * D : 2u * GE::kGroups * R * 128u;  // K + V bytes of one chunk
+    // The ring the copies land in: the MMA stages, or with the 8-bit cache the raw ones.
+    constexpr int PS = F8 ? RS : S;
+    const uint32_t p_full = F8 ? raw_full : full_bar;
+    const uint32_t p_empty = F8 ? raw_empty : empty_bar;
+    TcStageInfo* const p_info = F8 ? rinfo : info;
     // Block-table rows are read 32 entries at a time (one per lane) into a register window,
     // with the window needed next already in flight, so no copy waits on a dependent load.
     // Window boundaries (entry 32 k starts at token 32 k ps, a multiple of 512) fall on
@@ -331,7 +376,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
       if (mine) {
       if (__any_sync(0xffffffffu, aborted())) break;  // warp-uniform
       if (round > 0) {
-        const bool ok = ptx::mbar_wait_bounded(empty_bar + 8 * stage, (round - 1) & 1u, limit);
+        const bool ok = ptx::mbar_wait_bounded(p_empty + 8 * stage, (round - 1) & 1u, limit);
         if (!__all_sync(0xffffffffu, ok)) {
           if (lane == 0) abort_all(kErrTimeout);
           break;
@@ -339,9 +384,13 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
       }
       if (first) {
         // Q rows of this piece's segment (the previous piece's S MMAs must be done with it).
+        // Piece - 1's copy was issued only after the phase of piece - 2 completed, so once
+        // it has been issued the parity wait can only be met by the phase of piece - 1.
         bool ok = true;
-        if (piece >= 1)
-          ok = ptx::mbar_wait_bounded(qempty_bar, static_cast<uint32_t>((piece - 1) & 1), limit);
+        if (piece >= 1) {
+          ok = ptx::wait_counter(&s_qissued, piece, limit);
+          if (ok) ok = ptx::mbar_wait_bounded(qempty_bar, static_cast<uint32_t>((piece - 1) & 1), limit);
+        }
         if (!__all_sync(0xffffffffu, ok)) {
           if (lane == 0) abort_all(kErrTimeout);
           break;
@@ -361,6 +410,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
             if (!p.arm_without_copy)  // one box: 128 rows x every column group
               ptx::tma_load_3d(qbuf, &tmap_q, qfull_bar, 0, q_row0, 0, 0);
           }
+          *reinterpret_cast<volatile int*>(&s_qissued) = piece + 1;
         }
       }
       const int nvalid = min(kTcBlk, cu.len - cu.blk * kTcBlk);
@@ -377,7 +427,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
         for (int c = 0; c < nchunks; ++c)
           if ((okbits >> c) & 1u) vmask |= chunk_mask << (c * R);
         if (nvalid < kTcBlk) vmask &= (1ull << nvalid) - 1ull;
-        TcStageInfo& si = info[stage];
+        TcStageInfo& si = p_info[stage];
         si.vmask = vmask;
         si.b = cu.b;
         si.seg = cu.seg;
@@ -389,18 +439,23 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
                    ((last && piece_blk0 == 0 && cu.blk + 1 == cu.nblk) ? kTcSole : 0) |
                    (first_piece ? kTcFirstPieceOfCta : 0);
         const uint32_t bytes = p.arm_without_copy ? 0u : __popc(okbits) * tile_bytes;
-        if (bytes) ptx::mbar_arrive_expect_tx(full_bar + 8 * stage, bytes);
-        else if (p.arm_without_copy) ptx::mbar_arrive_expect_tx(full_bar + 8 * stage, 1u);
-        else ptx::mbar_arrive(full_bar + 8 * stage);
+        if (bytes) ptx::mbar_arrive_expect_tx(p_full + 8 * stage, bytes);
+        else if (p.arm_without_copy) ptx::mbar_arrive_expect_tx(p_full + 8 * stage, 1u);
+        else ptx::mbar_arrive(p_full + 8 * stage);
       }
       __syncwarp();
       if (lane < nops && ((okbits >> op_c) & 1u) && !p.arm_without_copy) {
         const int row = (op_page * p.num_kv_heads + kvh) * ps + op_po;
-        const uint32_t dst = ring + stage * GE::kStage + op_t * GE::kTile + op_g * GE::kGroupBytes + op_c * R * 128;
-        ptx::tma_load_3d(dst, op_t ? &tmap_v : &tmap_k, full_bar + 8 * stage, 0, row, op_g, policy);
+        if constexpr (F8) {  // codes: R tokens are R * D / 128 rows of 128 bytes
+          const uint32_t dst = raw + stage * GE::kRawStage + op_t * GE::kRawTile + op_c * R * D;
+          ptx::tma_load_2d(dst, op_t ? &tmap_v : &tmap_k, p_full + 8 * stage, 0, row / (128 / D), policy);
+        } else {
+          const uint32_t dst = ring + stage * GE::kStage + op_t * GE::kTile + op_g * GE::kGroupBytes + op_c * R * 128;
+          ptx::tma_load_3d(dst, op_t ? &tmap_v : &tmap_k, full_bar + 8 * stage, 0, row, op_g, policy);
+        }
       }
       }  // mine
-      if (++stage == S) {
+      if (++stage == PS) {
         stage = 0;
         ++round;
       }
@@ -432,22 +487,22 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
       }
     }
     // Let this producer's copies still in flight land before the CTA can exit.
-    for (int64_t j = (i > S ? i - S : 0); j < i; ++j)
+    for (int64_t j = (i > PS ? i - PS : 0); j < i; ++j)
       if ((static_cast<uint32_t>(j) & 1u) == pid)
-        ptx::mbar_wait_bounded(full_bar + 8 * (j % S), static_cast<uint32_t>((j / S) & 1), limit);
+        ptx::mbar_wait_bounded(p_full + 8 * (j % PS), static_cast<uint32_t>((j / PS) & 1), limit);
   } else if (warp == kWarpS) {
     // ============================================================ S warp
     // S_n = Q K_n^T into TMEM buffer n % kTcBufs once block n's K has landed and the P V of
     // block n - kTcBufs (issued by the P V warp, reading P from the same buffer) is complete.
-    constexpr uint32_t idS = ptx::umma_idesc_bf16(kTcRows, kTcBlk, false);
+    constexpr uint32_t idS = F8 ? ptx::umma_idesc_f16(kTcRows, kTcBlk, false) : ptx::umma_idesc_bf16(kTcRows, kTcBlk, false);
     bool issued = false;  // a tcgen05.commit is only used to track MMAs this warp issued
     for (int64_t n = 0; n < total; ++n) {
       if (__any_sync(0xffffffffu, aborted())) break;  // warp-uniform
       const int stage = static_cast<int>(n % S);
       bool ok = ptx::mbar_wait_bounded(full_bar + 8 * stage, static_cast<uint32_t>((n / S) & 1), limit);
       const TcStageInfo si = info[stage];
-      if (ok && (si.flags & kTcFirst))
-        ok = ptx::mbar_wait_bounded(qfull_bar, static_cast<uint32_t>(si.piece & 1), limit);
+      if (ok && (si.flags & kTcFirst))  // (8-bit cache: once the converters have made Q fp16)
+        ok = ptx::mbar_wait_bounded(F8 ? qconv_bar : qfull_bar, static_cast<uint32_t>(si.piece & 1), limit);
       if (ok && n >= kTcBufs)
         ok = ptx::mbar_wait_bounded(pv_bar + 8 * (n % kTcBufs),
                                     static_cast<uint32_t>(((n - kTcBufs) / kTcBufs) & 1), limit);
@@ -483,7 +538,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
     // ============================================================ P V warp
     // O += P_m V_m as soon as the softmax has written P_m (and, at a piece start, has read
     // the previous piece's O out).
-    constexpr uint32_t idPV = ptx::umma_idesc_bf16(kTcRows, D, true);
+    constexpr uint32_t idPV = F8 ? ptx::umma_idesc_f16(kTcRows, D, true) : ptx::umma_idesc_bf16(kTcRows, D, true);
     bool issued = false;
     for (int64_t m = 0; m < total; ++m) {
       if (__any_sync(0xffffffffu, aborted())) break;  // warp-uniform
@@ -539,6 +594,94 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
     }
     __syncwarp();
     ptx::mbar_wait_bounded(drain_bar, 0, limit);
+  } else if (F8 && warp >= kWarpConv) {
+    // ============================================================ converter warps (8-bit cache)
+    // Converter c takes the blocks i with i % 2 == c: once the block's codes have landed
+    // (raw stage i % RS) and the MMA stage i % S is free (the P V of block i - S is
+    // complete), it widens the K and V codes to fp16 in the tile layout the MMAs read,
+    // copies the block's descriptor, and publishes the stage after a proxy fence (the MMAs
+    // read shared memory through the async proxy).  At a piece start it first converts
+    // the piece's query tile from bf16 to fp16 in place.
+    const uint32_t cid = static_cast<uint32_t>(warp - kWarpConv);
+    constexpr int CPT = D / 16;               // 16-code chunks per token
+    constexpr int ITERS = kTcBlk * CPT / 32;  // chunks per lane, block and tensor
+    const int tlo = lane & 7, cq = lane >> 3;
+    int rstage = 0, stage = 0;
+    uint32_t rround = 0, round = 0;
+    for (int64_t i = 0; i < total; ++i) {
+      if ((static_cast<uint32_t>(i) & 1u) == cid) {
+        if (__any_sync(0xffffffffu, aborted())) break;  // warp-uniform
+        bool ok = ptx::mbar_wait_bounded(raw_full + 8 * rstage, rround & 1u, limit);
+        if (ok && round > 0) ok = ptx::mbar_wait_bounded(empty_bar + 8 * stage, (round - 1) & 1u, limit);
+        if (!__all_sync(0xffffffffu, ok)) {
+          if (lane == 0) abort_all(kErrTimeout);
+          break;
+        }
+        const TcStageInfo si = rinfo[rstage];
+        if (si.flags & kTcFirst) {
+          // The producer loads a piece's Q only after the previous piece's S MMAs are done.
+          // Once piece - 1's Q has been converted (its copy landed), the parity wait can
+          // only be met by this piece's copy.
+          ok = ptx::wait_counter(&s_qconverted, si.piece, limit);
+          if (ok) ok = ptx::mbar_wait_bounded(qfull_bar, static_cast<uint32_t>(si.piece & 1), limit);
+          if (!__all_sync(0xffffffffu, ok)) {
+            if (lane == 0) abort_all(kErrTimeout);
+            break;
+          }
+          uint4* qv = reinterpret_cast<uint4*>(base_ptr + (qbuf - ring));
+          for (int k = lane; k < GE::kQTile / 16; k += 32) {
+            uint4 x = qv[k];
+            x.x = ptx::bf16x2_to_f16x2(x.x);
+            x.y = ptx::bf16x2_to_f16x2(x.y);
+            x.z = ptx::bf16x2_to_f16x2(x.z);
+            x.w = ptx::bf16x2_to_f16x2(x.w);
+            qv[k] = x;
+          }
+          ptx::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            ptx::mbar_arrive(qconv_bar);
+            *reinterpret_cast<volatile int*>(&s_qconverted) = si.piece + 1;
+          }
+        }
+        const uint8_t* rb = base_ptr + (raw - ring) + rstage * GE::kRawStage;
+        uint8_t* fb = base_ptr + stage * GE::kStage;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {  // K, then V
+#pragma unroll 4
+          for (int it = 0; it < ITERS; ++it) {
+            // 16-code chunk c (head dims 16 c .. 16 c + 15) of token tok: 8 lanes take 8
+            // tokens of one chunk, so the swizzled reads and writes hit distinct banks
+            const int c = cq + 4 * (it % (CPT / 4));
+            const int tok = 8 * (it / (CPT / 4)) + tlo;
+            const int rrow = tok / (128 / D);
+            const int rc = (tok % (128 / D)) * CPT + c;
+            const uint4 x = *reinterpret_cast<const uint4*>(rb + t * GE::kRawTile + rrow * 128 + ((rc ^ (rrow & 7)) << 4));
+            const int cc = 2 * (c % 4);  // 8-value chunk of its 64-column group
+            uint8_t* dst = fb + t * GE::kTile + (c / 4) * GE::kGroupBytes + tok * 128;
+            *reinterpret_cast<uint4*>(dst + ((cc ^ (tok & 7)) << 4)) =
+                make_uint4(ptx::e4m3x2_lo(x.x), ptx::e4m3x2_hi(x.x), ptx::e4m3x2_lo(x.y), ptx::e4m3x2_hi(x.y));
+            *reinterpret_cast<uint4*>(dst + (((cc + 1) ^ (tok & 7)) << 4)) =
+                make_uint4(ptx::e4m3x2_lo(x.z), ptx::e4m3x2_hi(x.z), ptx::e4m3x2_lo(x.w), ptx::e4m3x2_hi(x.w));
+          }
+        }
+        if (lane == 0) info[stage] = si;
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          ptx::mbar_arrive(full_bar + 8 * stage);
+          ptx::mbar_arrive(raw_empty + 8 * rstage);
+        }
+      }
+      if (++rstage == RS) {
+        rstage = 0;
+        ++rround;
+      }
+      if (++stage == S) {
+        stage = 0;
+        ++round;
+      }
+    }
   } else {
     // ============================================================ softmax warpgroups
     // Thread t: warpgroup g = t / 128 owns tokens [32 g, 32 g + 32) of every block and its
@@ -549,8 +692,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
     const int g = t >> 7, r = t & (kTcRows - 1);
     const uint32_t lane_off = static_cast<uint32_t>(32 * (warp & 3)) << 16;
     const uint32_t o_mine = tmem + lane_off + (g ? GE::kO1 : GE::kO0);
-    const float sl2 = p.scale_log2;
-    const bool pos = sl2 >= 0.f;  // a negative scale turns the row maximum into a minimum
+    float sl2 = p.scale_log2;     // (8-bit cache: times the kv head's K scale, set per piece)
+    bool pos = sl2 >= 0.f;        // a negative scale turns the row maximum into a minimum
     constexpr int HD = D / 2;     // output columns each warpgroup finishes at a piece end
     float mref = -INFINITY, lsum = 0.f;
     // MQ: query tokens newer than this row's own.  Rows past the group's are padding whose
@@ -604,6 +747,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
       if (first) {
         mref = -INFINITY;
         lsum = 0.f;
+        if constexpr (F8) {
+          sl2 = p.scale_log2 * __ldg(p.k_scales + info[stg].seg / p.n_ht);
+          pos = sl2 >= 0.f;
+        }
       }
       const uint32_t st = tmem + lane_off + 64 * sb;
       uint32_t u[32];
@@ -714,7 +861,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
         lsum += s0 + s1;
       }
 #pragma unroll
-      for (int c = 0; c < 32; c += 2) pk[c / 2] = ptx::pack_bf16x2(e[c], e[c + 1]);
+      for (int c = 0; c < 32; c += 2) pk[c / 2] = F8 ? ptx::pack_f16x2(e[c], e[c + 1]) : ptx::pack_bf16x2(e[c], e[c + 1]);
       ptx::tmem_st16(st + 32 * g, pk);
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
@@ -748,7 +895,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
       const bool sole = flags & kTcSole;
       const int64_t slot = w * 2 + ((flags & kTcFirstPieceOfCta) ? 0 : 1);
       const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
-      const float f0 = sole ? w0 * inv : w0, f1 = sole ? w1 * inv : w1;
+      float f0 = sole ? w0 * inv : w0, f1 = sole ? w1 * inv : w1;
+      if constexpr (F8) {  // cached V values are codes x the kv head's V scale
+        const float vs = __ldg(p.v_scales + kvh);
+        f0 *= vs;
+        f1 *= vs;
+      }
       float* const rows_buf = stg_all + warp * kStgFloats;
 #pragma unroll
       for (int c0 = 0; c0 < HD; c0 += 32) {
@@ -974,19 +1126,22 @@ __global__ void __launch_bounds__(kMergeThreads, 6) merge_tc_kernel(const Decode
 
 // ------------------------------------------------------------------ host side
 namespace {
-template <int D>
+template <int D, bool F8 = false>
 constexpr size_t tc_smem_bytes() {
-  using GE = TcGeo<D>;
-  return 1024 + static_cast<size_t>(GE::kStages) * GE::kStage + GE::kQTile +
-         GE::kStages * sizeof(TcStageInfo) + 16 * GE::kStages + 24 * kTcBufs + 64 + 128 +
-         kTcSoftThreads / 32 * kStgFloats * sizeof(float);
+  using GE = TcGeo<D, F8>;
+  return 1024 + static_cast<size_t>(GE::kStages) * GE::kStage + static_cast<size_t>(GE::kRawStages) * GE::kRawStage +
+         GE::kQTile + (GE::kStages + GE::kRawStages) * sizeof(TcStageInfo) + 16 * GE::kStages +
+         16 * GE::kRawStages + 8 + 24 * kTcBufs + 64 + 128 + kTcSoftThreads / 32 * kStgFloats * sizeof(float);
 }
+static_assert(tc_smem_bytes<128, true>() <= 227 * 1024 && tc_smem_bytes<64, true>() <= 227 * 1024 &&
+                  tc_smem_bytes<128>() <= 227 * 1024 && tc_smem_bytes<64>() <= 227 * 1024,
+              "shared memory per CTA");
 
-template <int D, bool MQ>
+template <int D, bool MQ, bool F8 = false>
 cudaError_t launch_tc_t(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
                         const CUtensorMap& tq, int grid, cudaStream_t stream, bool overlap) {
-  auto kern = decode_tc_kernel<D, MQ>;
-  constexpr size_t smem = tc_smem_bytes<D>();
+  auto kern = decode_tc_kernel<D, MQ, F8>;
+  constexpr size_t smem = tc_smem_bytes<D, F8>();
   static thread_local int configured_device = -1;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -997,7 +1152,7 @@ cudaError_t launch_tc_t(const DecodeParams& p, const CUtensorMap& tk, const CUte
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kTcThreads);
+  cfg.blockDim = dim3(F8 ? kTcThreadsF8 : kTcThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -1019,12 +1174,16 @@ cudaError_t launch_tc_t(const DecodeParams& p, const CUtensorMap& tk, const CUte
 }
 }  // namespace
 
-size_t decode_tc_smem_bytes(int head_dim) {
+size_t decode_tc_smem_bytes(int head_dim, bool fp8) {
+  if (fp8) return head_dim == 64 ? tc_smem_bytes<64, true>() : tc_smem_bytes<128, true>();
   return head_dim == 64 ? tc_smem_bytes<64>() : tc_smem_bytes<128>();
 }
 
 cudaError_t launch_decode_tc(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
                              const CUtensorMap& tq, int grid, cudaStream_t stream, bool overlap) {
+  if (p.k_scales != nullptr)
+    return p.head_dim == 64 ? launch_tc_t<64, false, true>(p, tk, tv, tq, grid, stream, overlap)
+                            : launch_tc_t<128, false, true>(p, tk, tv, tq, grid, stream, overlap);
   if (p.q_len > 1)
     return p.head_dim == 64 ? launch_tc_t<64, true>(p, tk, tv, tq, grid, stream, overlap)
                             : launch_tc_t<128, true>(p, tk, tv, tq, grid, stream, overlap);

@@ -44,13 +44,18 @@ namespace gqa {
 
 namespace {
 
-template <int D>
+// F8: the cache holds e4m3 codes (one byte per element) instead of bf16.
+template <int D, bool F8 = false>
 struct Geo {
-  static constexpr int kBoxes = D / 64;                      // 64-column (128-byte) boxes
-  static constexpr int kBoxBytes = kChunk * 128;             // 16 rows x 128 bytes
-  static constexpr int kSubBytes = kBoxes * kBoxBytes;       // one 16-token K (or V) tile
+  static constexpr int kElem = F8 ? 1 : 2;
+  static constexpr int kBoxes = D / 64;                      // bf16: 64-column (128-byte) boxes
+  static constexpr int kBoxBytes = kChunk * 128;             // bf16: 16 rows x 128 bytes
+  static constexpr int kSubBytes = kChunk * D * kElem;       // one 16-token K (or V) tile
   static constexpr int kTileBytes = kSubChunks * kSubBytes;  // 64-token K (or V) tile
   static constexpr int kStageBytes = 2 * kTileBytes;
+  // Query heads whose fp32 partial O (D floats each) fit one sub-chunk tile: a consumer
+  // hands its partial to the epilogue in its own K and V sub-chunk tiles.
+  static constexpr int kHeadsPerSub = kSubBytes / (4 * D);
 };
 
 constexpr float kRescaleThreshold = 8.0f;
@@ -225,6 +230,117 @@ __device__ __forceinline__ void attend_subchunk(uint32_t kb, uint32_t vb, int nv
   }
 }
 
+// The same sub-chunk over an e4m3 cache, on fp16 MMAs (e4m3 -> fp16 is exact; q is
+// converted to fp16 when its fragments are loaded, P is packed as fp16).  One 16-byte
+// ldmatrix row is 16 head-dim values of one token, so thread (g, q) receives values
+// 4q .. 4q + 3 of a 16-value chunk: the contraction over head_dim uses that order for
+// K (the q fragments follow it), and for V^T each converted pair is transposed with
+// movmatrix, which puts dimension 16 mt + 4 (g >> 1) + (g & 1) (+ 2 for row g + 8) on
+// M-row g of O^T tile mt.
+template <int D, int NT>
+__device__ __forceinline__ void attend_subchunk_f8(uint32_t kb, uint32_t vb, int nvalid,
+                                                   const uint32_t (&ofs)[D / 32], const uint32_t (&qf)[D / 16][NT][2],
+                                                   float (&o)[D / 16][NT][4], float (&mref)[NT][2],
+                                                   float (&lsum)[NT][2], float sl2, int g, int q) {
+  constexpr int MT = D / 16;
+  float s[2][NT][4];
+#pragma unroll
+  for (int c = 0; c < 2; ++c)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) s[c][nt][0] = s[c][nt][1] = s[c][nt][2] = s[c][nt][3] = 0.f;
+#pragma unroll
+  for (int kx = 0; kx < D / 32; ++kx) {
+    uint32_t r[4];
+    ptx::ldmatrix_x4(kb + ofs[kx], r[0], r[1], r[2], r[3]);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {  // k-step 2 kx + h: chunk 2 kx + h (r[2h]: token g, r[2h+1]: g + 8)
+      const uint32_t a[4] = {ptx::e4m3x2_lo(r[2 * h]), ptx::e4m3x2_lo(r[2 * h + 1]), ptx::e4m3x2_hi(r[2 * h]),
+                             ptx::e4m3x2_hi(r[2 * h + 1])};
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) ptx::mma_f16_16816(s[h][nt], a, qf[2 * kx + h][nt][0], qf[2 * kx + h][nt][1]);
+    }
+  }
+  float sc[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) sc[nt][e] = (s[0][nt][e] + s[1][nt][e]) * sl2;
+  if (nvalid < kChunk) {
+    const bool v0 = g < nvalid, v1 = g + 8 < nvalid;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      if (!v0) sc[nt][0] = sc[nt][1] = -INFINITY;
+      if (!v1) sc[nt][2] = sc[nt][3] = -INFINITY;
+    }
+  }
+  float mx[NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      float m = fmaxf(sc[nt][e], sc[nt][e + 2]);
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+      mx[nt][e] = m;
+    }
+  bool need = false;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) need |= mx[nt][e] > mref[nt][e] + kRescaleThreshold;
+  if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float mn = fmaxf(mref[nt][e], mx[nt][e]);
+        const float alpha = (mn == mref[nt][e]) ? 1.f : ptx::ex2(mref[nt][e] - mn);
+        mref[nt][e] = mn;
+        lsum[nt][e] *= alpha;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          o[mt][nt][e] *= alpha;
+          o[mt][nt][e + 2] *= alpha;
+        }
+      }
+  }
+  uint32_t pb[NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    const float mu0 = (mref[nt][0] == -INFINITY) ? 0.f : mref[nt][0];
+    const float mu1 = (mref[nt][1] == -INFINITY) ? 0.f : mref[nt][1];
+    const float p0 = ptx::ex2(sc[nt][0] - mu0), p1 = ptx::ex2(sc[nt][1] - mu1);
+    const float p2 = ptx::ex2(sc[nt][2] - mu0), p3 = ptx::ex2(sc[nt][3] - mu1);
+    lsum[nt][0] += p0 + p2;
+    lsum[nt][1] += p1 + p3;
+    pb[nt][0] = ptx::movmatrix_trans(ptx::pack_f16x2(p0, p1));
+    pb[nt][1] = ptx::movmatrix_trans(ptx::pack_f16x2(p2, p3));
+  }
+  // Codes past the sequence end may be anything (NaN included): zeroed after conversion.
+  uint32_t vm0 = 0xffffffffu, vm1 = 0xffffffffu;
+  if (nvalid < kChunk) {
+    const int t0 = 2 * q, t1 = 8 + 2 * q;
+    vm0 = (t0 < nvalid ? 0x0000ffffu : 0u) | (t0 + 1 < nvalid ? 0xffff0000u : 0u);
+    vm1 = (t1 < nvalid ? 0x0000ffffu : 0u) | (t1 + 1 < nvalid ? 0xffff0000u : 0u);
+  }
+#pragma unroll
+  for (int vx = 0; vx < D / 32; ++vx) {
+    uint32_t r[4];
+    ptx::ldmatrix_x4(vb + ofs[vx], r[0], r[1], r[2], r[3]);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {  // O^T tile mt = 2 vx + h
+      uint32_t a[4];
+      a[0] = ptx::movmatrix_trans(ptx::e4m3x2_lo(r[2 * h])) & vm0;      // dims d(g), tokens 2q, 2q+1
+      a[1] = ptx::movmatrix_trans(ptx::e4m3x2_hi(r[2 * h])) & vm0;      // dims d(g) + 2
+      a[2] = ptx::movmatrix_trans(ptx::e4m3x2_lo(r[2 * h + 1])) & vm1;  // dims d(g), tokens 8 + 2q, ..
+      a[3] = ptx::movmatrix_trans(ptx::e4m3x2_hi(r[2 * h + 1])) & vm1;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) ptx::mma_f16_16816(o[2 * vx + h][nt], a, pb[nt][0], pb[nt][1]);
+    }
+  }
+}
+
 }  // namespace
 
 // Launch shape: CTAs per SM (several producer warps per SM keep more TMA copies in
@@ -242,14 +358,20 @@ constexpr int kWsCtasPerSm = GQA_CTAS_TOKEN_SPLIT;
 // sub-chunk of every stage for all rows).  C: consumer warps.  S: stages.  MQ:
 // several query tokens per sequence (p.q_len): a kv head's rows are its group of heads
 // for each query token in turn (row r: token r / group, head r % group), one segment.
-template <int D, int NT, int C, int S, bool MQ>
+// F8: the cache holds e4m3 codes with one scale per kv head for K and for V
+// (p.k_scales, p.v_scales); the K scale joins the score scale of a piece, the V scale
+// the output of its combine.
+template <int D, int NT, int C, int S, bool MQ, bool F8>
 __global__ void __launch_bounds__((C + 2) * 32, kWsCtasPerSm)
 decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
                  const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
-  using G_ = Geo<D>;
+  using G_ = Geo<D, F8>;
   constexpr int MT = D / 16;
   constexpr int NH = 8 * NT;             // heads one consumer covers
+  constexpr int HS = G_::kHeadsPerSub;   // partial rows that fit one sub-chunk tile
   static_assert(C == kSubChunks, "one consumer per sub-chunk");
+  static_assert(NH <= 2 * HS, "a consumer's partial must fit its K and V sub-chunk tiles");
+  static_assert(!(F8 && MQ), "the 8-bit cache serves one query token per sequence");
 
   extern __shared__ uint8_t smem_raw[];
   __shared__ int64_t s_wtot[kMaxWarps];
@@ -363,7 +485,6 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
   // Token split: at a piece end each consumer leaves its partial O^T in the part of the
   // stage only it read (its sub-chunk's K tile, and V tile for a second n-tile) and its
   // (max, sum) pairs in cml[stage]; the epilogue warp combines them and releases the stage.
-  static_assert(8 * D * 4 == G_::kSubBytes, "an 8-head partial fills one sub-chunk tile");
   constexpr int kCml = S * C * NH * 2;  // floats
   float* cml = reinterpret_cast<float*>(base_ptr + S * G_::kStageBytes);
   // Token split: the query rows of a piece arrive with its first block (bulk copy).
@@ -517,9 +638,16 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const uint32_t kdst = ring + stage * G_::kStageBytes + lane * G_::kSubBytes;
         const uint32_t vdst = kdst + G_::kTileBytes;
         const uint32_t bar = full_bar + 8 * stage;
-        // one copy per tensor brings all head_dim/64 column boxes of the 16 rows
-        ptx::tma_load_3d(kdst, &tmap_k, bar, 0, row, 0, policy);
-        ptx::tma_load_3d(vdst, &tmap_v, bar, 0, row, 0, policy);
+        if constexpr (F8) {
+          // the codes viewed as 128-byte rows: a sub-chunk is 16 * D / 128 of them
+          const int row8 = row / (128 / D);
+          ptx::tma_load_2d(kdst, &tmap_k, bar, 0, row8, policy);
+          ptx::tma_load_2d(vdst, &tmap_v, bar, 0, row8, policy);
+        } else {
+          // one copy per tensor brings all head_dim/64 column boxes of the 16 rows
+          ptx::tma_load_3d(kdst, &tmap_k, bar, 0, row, 0, policy);
+          ptx::tma_load_3d(vdst, &tmap_v, bar, 0, row, 0, policy);
+        }
       }
       if (last) first_piece = false;
       if (i + 1 < total) {
@@ -557,6 +685,7 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const int kvh = si.seg / p.n_ht, ht = si.seg % p.n_ht;
         const int nrows = min(hps, grp - ht * hps);
         const bool sole = si.flags & kSole;
+        const float vscale = F8 ? __ldg(p.v_scales + kvh) : 1.f;
         const int64_t slot = w * 2 + ((si.flags & kFirstPieceOfCta) ? 0 : 1);
         for (int h = 0; h < nrows; ++h) {
           float mj[C], wj[C];
@@ -576,10 +705,14 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
           for (int c = 0; c < CPL; ++c) acc[c] = 0.f;
 #pragma unroll
           for (int jj = 0; jj < C; ++jj) {
-            const float* src = reinterpret_cast<const float*>(st + (h >= 8 ? G_::kTileBytes : 0) +
-                                                              jj * G_::kSubBytes) + (h & 7) * D + d0;
+            const float* src = reinterpret_cast<const float*>(st + (h >= HS ? G_::kTileBytes : 0) +
+                                                              jj * G_::kSubBytes) + (h % HS) * D + d0;
 #pragma unroll
             for (int c = 0; c < CPL; ++c) acc[c] += wj[jj] * src[c];
+          }
+          if constexpr (F8) {  // the cached V values are codes x the kv head's V scale
+#pragma unroll
+            for (int c = 0; c < CPL; ++c) acc[c] *= vscale;
           }
           if (sole) {
             const float inv = L > 0.f ? 1.f / L : 0.f;
@@ -684,6 +817,20 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
   const int g = lane >> 2;
   const int q = lane & 3;
   uint32_t kofs[4], vofs[4];
+  uint32_t ofs8[D / 32];  // F8: ldmatrix row addresses, K and V alike
+  if constexpr (F8) {
+    // lane l addresses row l % 8 of matrix l / 8: token (l % 8) + 8 ((l / 8) & 1), 16-value
+    // chunk 2 x + (l / 16) of the x-th 32 values; a token's D codes are D / 128 of a
+    // 128-byte swizzled row
+    const int tok = (lane & 7) + (((lane >> 3) & 1) << 3);
+#pragma unroll
+    for (int x = 0; x < D / 32; ++x) {
+      const int chunk = 2 * x + (lane >> 4);
+      const int row = tok / (128 / D);
+      const int c = (tok % (128 / D)) * (D / 16) + chunk;
+      ofs8[x] = static_cast<uint32_t>(row * 128 + ((c ^ (row & 7)) << 4));
+    }
+  }
   {
     // K as the A operand: matrices (t0-7, d), (t8-15, d), (t0-7, d+8), (t8-15, d+8).
     const int tokK = (lane & 7) + (((lane >> 3) & 1) << 3);
@@ -705,11 +852,12 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
   int nrows_c = 0;    // valid heads of this consumer's tile
   int cdrop[NT][2];   // MQ: query tokens newer than each column's own
   const int max_drop = MQ ? p.q_len - 1 : 0;
-  const float sl2 = p.scale_log2;
+  float sl2 = p.scale_log2;
 
   auto load_q = [&](int b, int seg, int stage) {
     const int kvh = seg / p.n_ht;
     const int ht = seg % p.n_ht;
+    if constexpr (F8) sl2 = p.scale_log2 * __ldg(p.k_scales + kvh);
     nrows_seg = min(p.heads_per_seg, grp - ht * p.heads_per_seg);
     nrows_c = min(NH, nrows_seg);
     const int r0 = ht * p.heads_per_seg;  // first row of the segment
@@ -726,8 +874,13 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
       const uint32_t* qrow = reinterpret_cast<const uint32_t*>(qbuf + stage * kQBytes) + (v ? h : 0) * (D / 2);
 #pragma unroll
       for (int ks = 0; ks < MT; ++ks) {
-        qf[ks][nt][0] = v ? qrow[ks * 8 + q] : 0u;
-        qf[ks][nt][1] = v ? qrow[ks * 8 + 4 + q] : 0u;
+        if constexpr (F8) {  // fp16, values 16 ks + 4q, +1 and 16 ks + 4q + 2, +3 (the K order)
+          qf[ks][nt][0] = v ? ptx::bf16x2_to_f16x2(qrow[ks * 8 + 2 * q]) : 0u;
+          qf[ks][nt][1] = v ? ptx::bf16x2_to_f16x2(qrow[ks * 8 + 2 * q + 1]) : 0u;
+        } else {
+          qf[ks][nt][0] = v ? qrow[ks * 8 + q] : 0u;
+          qf[ks][nt][1] = v ? qrow[ks * 8 + 4 + q] : 0u;
+        }
       }
     }
 #pragma unroll
@@ -755,9 +908,13 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const uint32_t kst = ring + stage * G_::kStageBytes;
     if ((si.submask >> j) & 1) {
       const uint32_t kb = kst + j * G_::kSubBytes;
-      attend_subchunk<D, NT, MQ>(kb, kb + G_::kTileBytes, min(kChunk, si.nvalid - j * kChunk),
-                                 kofs, vofs, qf, o, mref, lsum, sl2, g, q, si.rem - j * kChunk, max_drop,
-                                 cdrop);
+      if constexpr (F8)
+        attend_subchunk_f8<D, NT>(kb, kb + G_::kTileBytes, min(kChunk, si.nvalid - j * kChunk), ofs8, qf, o, mref,
+                                  lsum, sl2, g, q);
+      else
+        attend_subchunk<D, NT, MQ>(kb, kb + G_::kTileBytes, min(kChunk, si.nvalid - j * kChunk),
+                                   kofs, vofs, qf, o, mref, lsum, sl2, g, q, si.rem - j * kChunk, max_drop,
+                                   cdrop);
     }
     const bool piece_end = si.flags & kLastOfPiece;
     __syncwarp();
@@ -800,17 +957,22 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
             mlj[h * 2 + 1] = lt[nt][e];
           }
       }
+      // Head h of this consumer goes to its K sub-chunk tile (h < HS) or its V one.
+      // O^T M-row g of tile mt is dimension 16 mt + g (bf16), or 16 mt + dg with the
+      // 8-bit cache's order (row g + 8: 16 mt + g + 8, or 16 mt + dg + 2).
+      const int dg = F8 ? 4 * (g >> 1) + (g & 1) : g;
+      constexpr int d8 = F8 ? 2 : 8;
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        float* reg = reinterpret_cast<float*>(base_ptr + stage * G_::kStageBytes +
-                                              (nt ? G_::kTileBytes : 0) + j * G_::kSubBytes);
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          float* row = reg + (2 * q + e) * D;
+          const int h = nt * 8 + 2 * q + e;
+          float* row = reinterpret_cast<float*>(base_ptr + stage * G_::kStageBytes + (h >= HS ? G_::kTileBytes : 0) +
+                                                j * G_::kSubBytes) + (h % HS) * D;
 #pragma unroll
           for (int mt = 0; mt < MT; ++mt) {
-            row[mt * 16 + g] = o[mt][nt][e];
-            row[mt * 16 + g + 8] = o[mt][nt][e + 2];
+            row[mt * 16 + dg] = o[mt][nt][e];
+            row[mt * 16 + dg + d8] = o[mt][nt][e + 2];
           }
         }
       }
@@ -825,7 +987,7 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
 namespace {
 
 
-template <int D, int NT, int C>
+template <int D, int NT, int C, bool F8 = false>
 struct Cfg {
   static constexpr int kNH = 8 * NT;
   // per-stage (max, sum) hand-off area, sized for up to 8 stages
@@ -833,17 +995,17 @@ struct Cfg {
   static constexpr size_t kBudget = static_cast<size_t>(GQA_SMEM_PER_SM_KB) * 1024 / kWsCtasPerSm;
   static constexpr size_t kQBytes = static_cast<size_t>(kNH) * D * 2;
   static constexpr int kStagesRaw =
-      static_cast<int>((kBudget - kMerge) / (Geo<D>::kStageBytes + kQBytes));
+      static_cast<int>((kBudget - kMerge) / (Geo<D, F8>::kStageBytes + kQBytes));
   static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
-  static constexpr size_t kSmem = 1024 + static_cast<size_t>(kStages) * (Geo<D>::kStageBytes + kQBytes) + kMerge +
-                                  kStages * (sizeof(StageInfo) + 24);
+  static constexpr size_t kSmem = 1024 + static_cast<size_t>(kStages) * (Geo<D, F8>::kStageBytes + kQBytes) +
+                                  kMerge + kStages * (sizeof(StageInfo) + 24);
 };
 
-template <int D, int NT, int C, bool MQ>
+template <int D, int NT, int C, bool MQ, bool F8 = false>
 cudaError_t launch_t(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int grid,
                      cudaStream_t stream, bool overlap) {
-  using CF = Cfg<D, NT, C>;
-  auto kern = decode_ws_kernel<D, NT, C, CF::kStages, MQ>;
+  using CF = Cfg<D, NT, C, F8>;
+  auto kern = decode_ws_kernel<D, NT, C, CF::kStages, MQ, F8>;
   static thread_local int configured_device = -1;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -877,9 +1039,9 @@ cudaError_t launch_d(const DecodeParams& p, const DecodePlan& pl, const CUtensor
   return pl.n_tiles == 1 ? launch_t<D, 1, 4, MQ>(p, tk, tv, grid, s, o) : launch_t<D, 2, 4, MQ>(p, tk, tv, grid, s, o);
 }
 
-template <int D, int NT, int C>
+template <int D, int NT, int C, bool F8 = false>
 void fill(DecodePlan& pl) {
-  using CF = Cfg<D, NT, C>;
+  using CF = Cfg<D, NT, C, F8>;
   pl.stages = CF::kStages;
   pl.smem_bytes = CF::kSmem;
 }
@@ -892,9 +1054,21 @@ void fill(DecodePlan& pl) {
 // the mma.sync kernel's, whose work grows with the heads (measured: 24 and 32 heads per
 // kv head, 29-49 us against 46-73 us).  Rows of several query tokens per sequence
 // (mq_rows) follow the same rule; on the tcgen05 kernel they form one segment (<= 128).
-DecodePlan plan_decode(int head_dim, int group, bool mq_rows) {
+DecodePlan plan_decode(int head_dim, int group, bool mq_rows, bool fp8) {
   DecodePlan pl{};
   (void)mq_rows;
+  if (fp8 && group <= 16) {
+    // 8-bit cache: a consumer's 8-head partial fills both its K and V sub-chunk tiles, so
+    // a segment is one 8-head tile; 9 to 16 heads per kv head take two segments (each
+    // reads the kv head's codes).
+    pl.n_tiles = 1;
+    pl.consumers = 4;
+    pl.heads_per_seg = 8;
+    pl.n_ht = (group + 7) / 8;
+    pl.ctas_per_sm = kWsCtasPerSm;
+    if (head_dim == 64) fill<64, 1, 4, true>(pl); else fill<128, 1, 4, true>(pl);
+    return pl;
+  }
   if (group > 16) {
     // Dense enough for the 5th-generation tensor cores: one 128-row MMA tile of heads.
     pl.tensor_cores = 1;
@@ -902,7 +1076,7 @@ DecodePlan plan_decode(int head_dim, int group, bool mq_rows) {
     pl.n_ht = (group + pl.heads_per_seg - 1) / pl.heads_per_seg;
     pl.ctas_per_sm = 1;
     pl.consumers = 4;
-    pl.smem_bytes = decode_tc_smem_bytes(head_dim);
+    pl.smem_bytes = decode_tc_smem_bytes(head_dim, fp8);
     return pl;
   }
   pl.n_tiles = group <= 8 ? 1 : 2;
@@ -920,6 +1094,9 @@ DecodePlan plan_decode(int head_dim, int group, bool mq_rows) {
 
 cudaError_t launch_decode(const DecodeParams& p, const DecodePlan& pl, const CUtensorMap& tk,
                           const CUtensorMap& tv, int grid, cudaStream_t stream, bool overlap) {
+  if (p.k_scales != nullptr)
+    return p.head_dim == 64 ? launch_t<64, 1, 4, false, true>(p, tk, tv, grid, stream, overlap)
+                            : launch_t<128, 1, 4, false, true>(p, tk, tv, grid, stream, overlap);
   if (p.q_len > 1)
     return p.head_dim == 64 ? launch_d<64, true>(p, pl, tk, tv, grid, stream, overlap)
                             : launch_d<128, true>(p, pl, tk, tv, grid, stream, overlap);

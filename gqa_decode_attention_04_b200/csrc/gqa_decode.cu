@@ -159,9 +159,10 @@ struct MapKey {
   int dev;
   int box_rows;
   int box_groups;
+  int codes;  // 1: an e4m3 pool (make_map_codes), 0: bf16
   bool operator==(const MapKey& o) const {
     return ptr == o.ptr && rows == o.rows && d == o.d && dev == o.dev && box_rows == o.box_rows &&
-           box_groups == o.box_groups;
+           box_groups == o.box_groups && codes == o.codes;
   }
 };
 
@@ -174,7 +175,7 @@ gqa_status make_map(CUtensorMap* m, const void* base, int64_t rows, int d, int d
   static thread_local MapKey keys[8];
   static thread_local CUtensorMap maps[8];
   static thread_local int next = 0;
-  MapKey k{base, rows, d, dev, box_rows, box_groups};
+  MapKey k{base, rows, d, dev, box_rows, box_groups, 0};
   for (int i = 0; i < 8; ++i)
     if (keys[i] == k) {
       *m = maps[i];
@@ -193,6 +194,35 @@ gqa_status make_map(CUtensorMap* m, const void* base, int64_t rows, int d, int d
   keys[next] = k;
   maps[next] = *m;
   next = (next + 1) % 8;
+  return GQA_OK;
+}
+
+// An e4m3 pool [P * Hk * ps, D] (one byte per element) viewed as 128-byte rows: a 2-D
+// uint8 tensor of 128 columns x rows * D / 128 rows.  One box is box_rows of those rows,
+// 128-byte swizzle (16 tokens of codes are 16 * D / 128 rows).
+gqa_status make_map_codes(CUtensorMap* m, const void* base, int64_t rows, int d, int dev, int box_rows) {
+  static thread_local MapKey keys[4];
+  static thread_local CUtensorMap maps[4];
+  static thread_local int next = 0;
+  MapKey k{base, rows, d, dev, box_rows, 1, 1};
+  for (int i = 0; i < 4; ++i)
+    if (keys[i] == k) {
+      *m = maps[i];
+      return GQA_OK;
+    }
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return fail(GQA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(rows * d / 128)};
+  cuuint64_t strides[1] = {128};
+  cuuint32_t box[2] = {128, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(GQA_ERR_CUDA, "cuTensorMapEncodeTiled (e4m3 pool) failed (%d)", (int)r);
+  keys[next] = k;
+  maps[next] = *m;
+  next = (next + 1) % 4;
   return GQA_OK;
 }
 
@@ -226,8 +256,13 @@ cudaError_t launch_with_maps(const gqa::DecodeParams& p, const gqa::DecodePlan& 
   if (plan.tensor_cores) {
     const int br = gqa::tc_box_rows(p.page_size);
     const int bg = br == 64 ? hd / 64 : 1;  // a 64-row box carries every column group
-    *st = make_map(&tk, k_pages, rows, hd, dev, br, bg);
-    if (*st == GQA_OK) *st = make_map(&tv, v_pages, rows, hd, dev, br, bg);
+    if (p.k_scales != nullptr) {  // e4m3 codes: br tokens are br * D / 128 rows of 128 bytes
+      *st = make_map_codes(&tk, k_pages, rows, hd, dev, br * hd / 128);
+      if (*st == GQA_OK) *st = make_map_codes(&tv, v_pages, rows, hd, dev, br * hd / 128);
+    } else {
+      *st = make_map(&tk, k_pages, rows, hd, dev, br, bg);
+      if (*st == GQA_OK) *st = make_map(&tv, v_pages, rows, hd, dev, br, bg);
+    }
     if (*st == GQA_OK)
       *st = p.q_len > 1
                 ? make_qmap_multi(&tq, q, p.num_seqs, p.q_len, p.num_kv_heads, p.group, hd)
@@ -235,8 +270,13 @@ cudaError_t launch_with_maps(const gqa::DecodeParams& p, const gqa::DecodePlan& 
     if (*st != GQA_OK) return cudaSuccess;
     return gqa::launch_decode_tc(p, tk, tv, tq, grid, strm, overlap);
   }
-  *st = make_map(&tk, k_pages, rows, hd, dev, gqa::kChunk, hd / 64);
-  if (*st == GQA_OK) *st = make_map(&tv, v_pages, rows, hd, dev, gqa::kChunk, hd / 64);
+  if (p.k_scales != nullptr) {  // e4m3 codes: a 16-token sub-chunk is 16 * D / 128 rows of 128 bytes
+    *st = make_map_codes(&tk, k_pages, rows, hd, dev, gqa::kChunk * hd / 128);
+    if (*st == GQA_OK) *st = make_map_codes(&tv, v_pages, rows, hd, dev, gqa::kChunk * hd / 128);
+  } else {
+    *st = make_map(&tk, k_pages, rows, hd, dev, gqa::kChunk, hd / 64);
+    if (*st == GQA_OK) *st = make_map(&tv, v_pages, rows, hd, dev, gqa::kChunk, hd / 64);
+  }
   if (*st != GQA_OK) return cudaSuccess;
   return gqa::launch_decode(p, plan, tk, tv, grid, strm, overlap);
 }
@@ -297,7 +337,9 @@ gqa_status decode_impl(const void* q, const void* k_pages, const void* v_pages,
                        const int32_t* block_table, const int32_t* seq_lens, void* out,
                        int num_seqs, int num_heads, int num_kv_heads, int head_dim, int page_size,
                        float scale, int max_blocks_per_seq, int num_pages, void* stream,
-                       bool overlap_previous, int q_len = 1) {
+                       bool overlap_previous, int q_len = 1, const float* k_scales = nullptr,
+                       const float* v_scales = nullptr) {
+  const bool fp8 = k_scales != nullptr || v_scales != nullptr;
   if (num_seqs < 0) return fail(GQA_ERR_INVALID_ARG, "num_seqs < 0");
   if (num_seqs > 65536) return fail(GQA_ERR_UNSUPPORTED, "num_seqs > 65536");
   if (q_len < 1) return fail(GQA_ERR_INVALID_ARG, "q_len %d < 1", q_len);
@@ -329,6 +371,13 @@ gqa_status decode_impl(const void* q, const void* k_pages, const void* v_pages,
     return fail(GQA_ERR_INVALID_ARG, "k_pages / v_pages must be 16-byte aligned");
   if (!aligned(q, 16) || !aligned(out, 8))
     return fail(GQA_ERR_INVALID_ARG, "q must be 16-byte and out 8-byte aligned");
+  if (fp8) {
+    if (k_scales == nullptr || v_scales == nullptr)
+      return fail(GQA_ERR_INVALID_ARG, "k_scales and v_scales are both required");
+    if (!aligned(k_scales, 4) || !aligned(v_scales, 4))
+      return fail(GQA_ERR_INVALID_ARG, "k_scales / v_scales must be 4-byte aligned");
+    if (q_len != 1) return fail(GQA_ERR_UNSUPPORTED, "the 8-bit cache serves one query token per sequence");
+  }
 
   DeviceState* st;
   int dev;
@@ -337,7 +386,7 @@ gqa_status decode_impl(const void* q, const void* k_pages, const void* v_pages,
   cudaStream_t strm = static_cast<cudaStream_t>(stream);
 
   const int group = num_heads / num_kv_heads;
-  const gqa::DecodePlan plan = gqa::plan_decode(head_dim, group * q_len, q_len > 1);
+  const gqa::DecodePlan plan = gqa::plan_decode(head_dim, group * q_len, q_len > 1, fp8);
   // Upper bound on the block count (seq_lens are device data).
   const int64_t blocks_per_seq =
       (static_cast<int64_t>(max_blocks_per_seq) * page_size + gqa::kBlock - 1) / gqa::kBlock;
@@ -356,11 +405,13 @@ gqa_status decode_impl(const void* q, const void* k_pages, const void* v_pages,
   if (s != GQA_OK) return s;
 
 
-  gqa::DecodeParams p;
+  gqa::DecodeParams p{};
   p.q = static_cast<const uint16_t*>(q);
   p.out = static_cast<uint16_t*>(out);
   p.block_table = block_table;
   p.seq_lens = seq_lens;
+  p.k_scales = k_scales;
+  p.v_scales = v_scales;
   p.part_o = st->part_o;
   p.part_ml = st->part_ml;
   p.counters = st->counters;
@@ -429,6 +480,49 @@ gqa_status append_impl(const void* k_new, const void* v_new, void* k_pages, void
   p.q_len = q_len;
   cudaError_t e = gqa::launch_kv_append(p, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "kv_append launch");
+  g_launches.fetch_add(1);
+  return GQA_OK;
+}
+
+gqa_status append_fp8_impl(const void* k_new, const void* v_new, void* k_pages, void* v_pages,
+                           const float* k_scales, const float* v_scales, const int32_t* block_table,
+                           const int32_t* positions, int num_seqs, int num_kv_heads, int head_dim, int page_size,
+                           int max_blocks_per_seq, int num_pages, void* stream) {
+  if (num_seqs < 0) return fail(GQA_ERR_INVALID_ARG, "num_seqs < 0");
+  if (num_kv_heads < 1 || head_dim < 1 || page_size < 1 || max_blocks_per_seq < 1 || num_pages < 1)
+    return fail(GQA_ERR_INVALID_ARG, "sizes must be positive");
+  if (head_dim % 16 != 0) return fail(GQA_ERR_UNSUPPORTED, "head_dim must be a multiple of 16");
+  if (static_cast<int64_t>(max_blocks_per_seq) * page_size > INT32_MAX)
+    return fail(GQA_ERR_UNSUPPORTED, "max_blocks_per_seq * page_size exceeds 2^31");
+  if (num_seqs == 0) return GQA_OK;
+  if (!k_new || !v_new || !k_pages || !v_pages || !k_scales || !v_scales || !block_table || !positions)
+    return fail(GQA_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(k_pages, 16) || !aligned(v_pages, 16))
+    return fail(GQA_ERR_INVALID_ARG, "k_new, v_new and the pools must be 16-byte aligned");
+  if (!aligned(k_scales, 4) || !aligned(v_scales, 4))
+    return fail(GQA_ERR_INVALID_ARG, "k_scales / v_scales must be 4-byte aligned");
+  DeviceState* st;
+  int dev;
+  gqa_status s = get_state(&st, &dev);
+  if (s != GQA_OK) return s;
+  gqa::AppendFp8Params p{};
+  p.k_new = static_cast<const uint4*>(k_new);
+  p.v_new = static_cast<const uint4*>(v_new);
+  p.k_pages = static_cast<uint4*>(k_pages);
+  p.v_pages = static_cast<uint4*>(v_pages);
+  p.k_scales = k_scales;
+  p.v_scales = v_scales;
+  p.block_table = block_table;
+  p.positions = positions;
+  p.err = st->err;
+  p.num_seqs = num_seqs;
+  p.num_kv_heads = num_kv_heads;
+  p.groups_per_row = head_dim / 16;
+  p.page_size = page_size;
+  p.max_blocks = max_blocks_per_seq;
+  p.num_pages = num_pages;
+  cudaError_t e = gqa::launch_kv_append_fp8(p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "kv_append_fp8 launch");
   g_launches.fetch_add(1);
   return GQA_OK;
 }
@@ -532,6 +626,54 @@ gqa_status gqa_multi_query_step(const void* q, const void* k_new, const void* v_
                      stream, true, q_len);
 }
 
+gqa_status gqa_kv_quantize_fp8(const void* src, void* dst, const float* scales, int num_pages,
+                               int num_kv_heads, int page_size, int head_dim, void* stream) {
+  if (num_pages < 0) return fail(GQA_ERR_INVALID_ARG, "num_pages < 0");
+  if (num_kv_heads < 1 || page_size < 1 || head_dim < 1) return fail(GQA_ERR_INVALID_ARG, "sizes must be positive");
+  if (head_dim % 16 != 0) return fail(GQA_ERR_UNSUPPORTED, "head_dim must be a multiple of 16");
+  if (num_pages == 0) return GQA_OK;
+  if (!src || !dst || !scales) return fail(GQA_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned(src, 16) || !aligned(dst, 16) || !aligned(scales, 4))
+    return fail(GQA_ERR_INVALID_ARG, "src and dst must be 16-byte and scales 4-byte aligned");
+  const int64_t groups = static_cast<int64_t>(num_pages) * num_kv_heads * page_size * (head_dim / 16);
+  cudaError_t e = gqa::launch_kv_quantize(static_cast<const uint4*>(src), static_cast<uint4*>(dst), scales, groups,
+                                          head_dim / 16, page_size, num_kv_heads, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "kv_quantize launch");
+  g_launches.fetch_add(1);
+  return GQA_OK;
+}
+
+gqa_status gqa_kv_append_fp8(const void* k_new, const void* v_new, void* k_pages, void* v_pages,
+                             const float* k_scales, const float* v_scales, const int32_t* block_table,
+                             const int32_t* positions, int num_seqs, int num_kv_heads, int head_dim, int page_size,
+                             int max_blocks_per_seq, int num_pages, void* stream) {
+  return append_fp8_impl(k_new, v_new, k_pages, v_pages, k_scales, v_scales, block_table, positions, num_seqs,
+                         num_kv_heads, head_dim, page_size, max_blocks_per_seq, num_pages, stream);
+}
+
+gqa_status gqa_paged_decode_attn_fp8(const void* q, const void* k_pages, const void* v_pages, const float* k_scales,
+                                     const float* v_scales, const int32_t* block_table, const int32_t* seq_lens,
+                                     void* out, int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                     int page_size, float scale, int max_blocks_per_seq, int num_pages,
+                                     void* stream) {
+  if (!k_scales || !v_scales) return fail(GQA_ERR_INVALID_ARG, "k_scales and v_scales are required");
+  return decode_impl(q, k_pages, v_pages, block_table, seq_lens, out, num_seqs, num_heads, num_kv_heads, head_dim,
+                     page_size, scale, max_blocks_per_seq, num_pages, stream, false, 1, k_scales, v_scales);
+}
+
+gqa_status gqa_decode_step_fp8(const void* q, const void* k_new, const void* v_new, void* k_pages, void* v_pages,
+                               const float* k_scales, const float* v_scales, const int32_t* block_table,
+                               const int32_t* positions, const int32_t* seq_lens, void* out, int num_seqs,
+                               int num_heads, int num_kv_heads, int head_dim, int page_size, float scale,
+                               int max_blocks_per_seq, int num_pages, void* stream) {
+  if (!k_scales || !v_scales) return fail(GQA_ERR_INVALID_ARG, "k_scales and v_scales are required");
+  gqa_status s = append_fp8_impl(k_new, v_new, k_pages, v_pages, k_scales, v_scales, block_table, positions,
+                                 num_seqs, num_kv_heads, head_dim, page_size, max_blocks_per_seq, num_pages, stream);
+  if (s != GQA_OK) return s;
+  return decode_impl(q, k_pages, v_pages, block_table, seq_lens, out, num_seqs, num_heads, num_kv_heads, head_dim,
+                     page_size, scale, max_blocks_per_seq, num_pages, stream, true, 1, k_scales, v_scales);
+}
+
 gqa_status gqa_paged_decode_attn_noalloc(const void* q, const void* k_pages, const void* v_pages,
                                          const int32_t* block_table, const int32_t* seq_lens,
                                          void* out, int num_seqs, int num_heads, int num_kv_heads,
@@ -609,7 +751,7 @@ gqa_status gqa_paged_decode_attn_noalloc(const void* q, const void* k_pages, con
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(allocation-free scratch)");
 
 
-  gqa::DecodeParams p;
+  gqa::DecodeParams p{};
   p.q = static_cast<const uint16_t*>(q);
   p.out = static_cast<uint16_t*>(out);
   p.block_table = block_table;

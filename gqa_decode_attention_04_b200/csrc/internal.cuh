@@ -53,6 +53,10 @@ struct DecodeParams {
   uint64_t wait_limit_ns;
   int arm_without_copy;
   int q_len;                  // query tokens per sequence (q, out: [B, q_len, H, D]); 1 = decode
+  // 8-bit cache: k_pages / v_pages hold e4m3 codes; a cached value is code * scale of its
+  // kv head (k_scales, v_scales [Hk] fp32).  nullptr for a bf16 cache.
+  const float* k_scales;
+  const float* v_scales;
 };
 
 struct AppendParams {
@@ -67,8 +71,26 @@ struct AppendParams {
   int q_len;                  // rows per sequence: k_new [B, q_len, Hk, D] to positions[b] + i
 };
 
+// The append into an 8-bit (e4m3) cache: 16 elements per thread.
+struct AppendFp8Params {
+  const uint4* k_new;         // [B, Hk, D] bf16
+  const uint4* v_new;
+  uint4* k_pages;             // [P, Hk, ps, D] e4m3
+  uint4* v_pages;
+  const float* k_scales;      // [Hk]
+  const float* v_scales;
+  const int32_t* block_table;
+  const int32_t* positions;
+  uint32_t* err;
+  int num_seqs, num_kv_heads, groups_per_row, page_size, max_blocks, num_pages;
+};
+
 // Launchers (return the cudaError_t of the launch).
 cudaError_t launch_kv_append(const AppendParams& p, cudaStream_t stream);
+cudaError_t launch_kv_append_fp8(const AppendFp8Params& p, cudaStream_t stream);
+// Codes of a bf16 pool, groups of 16 elements (groups_per_row = head_dim / 16).
+cudaError_t launch_kv_quantize(const uint4* src, uint4* dst, const float* scales, int64_t groups,
+                               int groups_per_row, int page_size, int num_kv_heads, cudaStream_t stream);
 
 // How a (head_dim, group) problem is mapped onto the decode kernel.
 struct DecodePlan {
@@ -82,8 +104,9 @@ struct DecodePlan {
   size_t smem_bytes;
 };
 
-// group: query rows per kv head; mq_rows: they are several query tokens' heads.
-DecodePlan plan_decode(int head_dim, int group, bool mq_rows = false);
+// group: query rows per kv head; mq_rows: they are several query tokens' heads; fp8: the
+// cache holds e4m3 codes.
+DecodePlan plan_decode(int head_dim, int group, bool mq_rows = false, bool fp8 = false);
 // overlap_previous: launch with programmatic stream serialization, so the prologue
 // overlaps the preceding kernel of the stream (which must write nothing the decode reads
 // except the K/V pools); the producer waits for that kernel before its first K/V copy.
@@ -92,7 +115,7 @@ DecodePlan plan_decode(int head_dim, int group, bool mq_rows = false);
 // [num_seqs * num_heads, head_dim] with boxes of 128 rows x every column group.
 cudaError_t launch_decode_tc(const DecodeParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
                              const CUtensorMap& tq, int grid, cudaStream_t stream, bool overlap);
-size_t decode_tc_smem_bytes(int head_dim);
+size_t decode_tc_smem_bytes(int head_dim, bool fp8 = false);
 
 cudaError_t launch_decode(const DecodeParams& p, const DecodePlan& plan, const CUtensorMap& tmap_k,
                           const CUtensorMap& tmap_v, int grid, cudaStream_t stream,

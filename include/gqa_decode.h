@@ -178,6 +178,55 @@ gqa_status gqa_multi_query_step(const void* q, const void* k_new, const void* v_
                                 float scale, int max_blocks_per_seq, int num_pages, void* stream);
 
 /*
+ * 8-bit (e4m3) K/V cache.  The TensorRT MQA page calibrates Q, K and V separately with
+ * their own per-tensor scales in 8-bit mode (one shared scale loses precision to their
+ * different ranges); the TensorRT-LLM guide names FP8 for throughput.  Here the pools
+ * hold e4m3 codes (1 sign, 4 exponent bits with bias 7, 3 mantissa bits; no infinities;
+ * S.1111.111 is NaN; largest value 448) and K and V each carry one fp32 scale per kv
+ * head (k_scales, v_scales: [num_kv_heads] device arrays; a per-tensor scale is the case
+ * of equal entries).  A cached value is code * scale of its kv head.  The pools take
+ * half the bytes of bf16 ones, the quantity decode attention is bound by.
+ *
+ *     k_pages, v_pages   [num_pages, num_kv_heads, page_size, head_dim]   e4m3 codes (uint8)
+ *
+ * Writing a bf16 value x stores the code nearest to the fp32 quotient x / scale (IEEE
+ * division, round to nearest even), saturating to +-448; NaN stays NaN.  q, out,
+ * k_new, v_new stay bf16.
+ *
+ * gqa_kv_quantize_fp8 -- codes of a whole bf16 pool: dst[p, kvh, t, :] = code of
+ *   src[p, kvh, t, :] / scales[kvh] (src [num_pages, num_kv_heads, page_size, head_dim]
+ *   bf16, dst the same shape in e4m3; both 16-byte aligned; head_dim % 16 == 0).
+ * gqa_kv_append_fp8 -- gqa_kv_append into coded pools, K rows with k_scales and V rows
+ *   with v_scales; same arguments otherwise (head_dim % 16 == 0, pools 16-byte aligned).
+ * gqa_paged_decode_attn_fp8 -- gqa_paged_decode_attn over coded pools: the definition at
+ *   the top of this file with K_b, V_b the cached values code * scale.  The kernel widens
+ *   codes to fp16 (exactly), converts q to fp16 (round to nearest: exact for 2^-17 <=
+ *   |q| <= 65504, saturating above) and accumulates in fp32.  Requirements as
+ *   gqa_paged_decode_attn, and num_heads / num_kv_heads <= 16 (GQA_ERR_UNSUPPORTED
+ *   otherwise).
+ * gqa_decode_step_fp8 -- gqa_kv_append_fp8, then gqa_paged_decode_attn_fp8, as
+ *   gqa_decode_step does for a bf16 cache.
+ */
+gqa_status gqa_kv_quantize_fp8(const void* src, void* dst, const float* scales, int num_pages,
+                               int num_kv_heads, int page_size, int head_dim, void* stream);
+gqa_status gqa_kv_append_fp8(const void* k_new, const void* v_new, void* k_pages, void* v_pages,
+                             const float* k_scales, const float* v_scales, const int32_t* block_table,
+                             const int32_t* positions, int num_seqs, int num_kv_heads, int head_dim,
+                             int page_size, int max_blocks_per_seq, int num_pages, void* stream);
+gqa_status gqa_paged_decode_attn_fp8(const void* q, const void* k_pages, const void* v_pages,
+                                     const float* k_scales, const float* v_scales,
+                                     const int32_t* block_table, const int32_t* seq_lens, void* out,
+                                     int num_seqs, int num_heads, int num_kv_heads, int head_dim,
+                                     int page_size, float scale, int max_blocks_per_seq, int num_pages,
+                                     void* stream);
+gqa_status gqa_decode_step_fp8(const void* q, const void* k_new, const void* v_new, void* k_pages,
+                               void* v_pages, const float* k_scales, const float* v_scales,
+                               const int32_t* block_table, const int32_t* positions,
+                               const int32_t* seq_lens, void* out, int num_seqs, int num_heads,
+                               int num_kv_heads, int head_dim, int page_size, float scale,
+                               int max_blocks_per_seq, int num_pages, void* stream);
+
+/*
  * gqa_paged_decode_attn_noalloc -- the same decode attention as gqa_paged_decode_attn
  * (same arguments, layouts and result), for callers that cannot allocate device memory:
  * an engine that has already reserved nearly all of the GPU for its own caching

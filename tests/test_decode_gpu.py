@@ -410,3 +410,15 @@ def test_large_group_forced_splits(cuda_device, workers):
     gq.set_num_workers(workers)
     d, out = _run(inp, cuda_device)
     assert_close(gpu_f64(out), oracle_out(host_arrays(inp)), what=f"workers={workers}")
+
+
+@pytest.mark.parametrize("workers", [1, 2, 3])
+def test_large_group_many_short_pieces_in_one_cta(cuda_device, workers):
+    """Many one-block sequences in a row inside one CTA's range on the tcgen05 kernel: the
+    query tile is reloaded for every piece, by the two producers in turns, and each load
+    must wait for the previous piece's S MMAs."""
+    lens = [64, 1, 5, 64, 3, 130, 1, 1, 1, 200, 2, 64, 1, 9]
+    inp = make_custom_inputs(lens, 96, 1, 128, 64, seed=45, extra_pages=2)
+    gq.set_num_workers(workers)
+    d, out = _run(inp, cuda_device)
+    assert_close(gpu_f64(out), oracle_out(host_arrays(inp)), what=f"workers={workers}")
