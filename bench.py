@@ -54,9 +54,11 @@ KERNEL_SOURCES = {
     "decode_ws_kernel": [_CSRC + "decode_ws.cu", _CSRC + "ptx.cuh", _CSRC + "internal.cuh"],
     "decode_tc_kernel": [_CSRC + "decode_tc.cu", _CSRC + "ptx.cuh", _CSRC + "internal.cuh"],
 }
-# Each timed loop runs at least this long on the GPU and at least this many replays.
-MIN_LOOP_SECONDS = 0.2
-MIN_REPEATS = 5
+# Each timed loop: at least MIN_REPEATS replays of a graph of GRAPH_LAUNCHES calls, and at
+# least MIN_LOOP_SECONDS of GPU time (short, so that a compute-heavy decode is timed at
+# the clocks it starts with rather than after seconds under the power cap).
+MIN_LOOP_SECONDS = 0.03
+MIN_REPEATS = 7
 GRAPH_LAUNCHES = 100
 
 
@@ -200,7 +202,10 @@ class ClockSampler:
                 continue
         return None
 
-    def summary(self):
+    def summary(self, windows=None):
+        """Median SM clock and throttle reasons over the samples inside `windows` (all
+        timed windows by default)."""
+        windows = self.windows if windows is None else windows
         sm, mx, reasons, n_all = [], None, set(), 0
         for ln in self.lines:
             parts = [p.strip() for p in ln.split(",")]
@@ -208,7 +213,7 @@ class ClockSampler:
                 continue
             n_all += 1
             t = self._stamp(parts[0])
-            if t is None or not any(a <= t <= b for a, b in self.windows):
+            if t is None or not any(a <= t <= b for a, b in windows):
                 continue
             try:
                 sm.append(float(parts[2]))
@@ -223,7 +228,7 @@ class ClockSampler:
                     "samples_total": n_all}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
                 "samples": len(sm), "samples_total": n_all, "period_ms": self.period_ms,
-                "timed_windows_s": round(sum(b - a for a, b in self.windows), 3)}
+                "timed_windows_s": round(sum(b - a for a, b in windows), 3)}
 
 
 def setup_dist(n_gpus: int):
@@ -448,6 +453,7 @@ def measure_workload(gq, inp_dev, dev, peak, clocks, fp8: bool):
     sets, l2_desc = _pool_sets(inp_dev, dev)
     n = len(sets)
     B, H, D = inp_dev.num_seqs, inp_dev.num_heads, inp_dev.head_dim
+    w0 = len(clocks.windows) if clocks is not None else 0
     out = torch.empty((B, H, D), dtype=torch.bfloat16, device=dev)
     nb = algorithmic_bytes(inp_dev, with_append=True)
 
@@ -465,6 +471,7 @@ def measure_workload(gq, inp_dev, dev, peak, clocks, fp8: bool):
     gq.check_device_error()
     achieved = nb["decode"] / (d_med * 1e-6) / 1e9
     kernel = decode_kernel_for(inp_dev)
+    units = int(inp_dev.seq_lens.to(torch.int64).sum())
     entry = {
         "workload": inp_dev.name, "num_seqs": B, "num_heads": H, "num_kv_heads": inp_dev.num_kv_heads,
         "head_dim": D, "page_size": inp_dev.page_size,
@@ -477,11 +484,14 @@ def measure_workload(gq, inp_dev, dev, peak, clocks, fp8: bool):
         "kv_tbps": nb["kv"] / (d_med * 1e-6) / 1e12,
         "step_tbps": nb["step"] / (s_med * 1e-6) / 1e12,
         "tokens_per_s": B / (s_med * 1e-6),
+        "traffic": profiled_traffic(inp_dev.name, kernel, units),
         "l2": l2_desc, "graph_launches": GRAPH_LAUNCHES,
+        "clocks": clocks.summary(clocks.windows[w0:]) if clocks is not None else None,
     }
     if fp8:
         try:
             entry["fp8"] = measure_fp8(gq, sets, dev, peak, clocks)
+            entry["fp8"]["traffic"] = profiled_traffic(inp_dev.name + "_fp8", kernel, units)
         except gq.GQAError as e:  # a shape the 8-bit path does not serve
             entry["fp8"] = {"unavailable": str(e)}
     del sets, out
@@ -628,25 +638,48 @@ def run_ours(args, rank, world, local):
     host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     d2h = host_out.numel() * host_out.element_size()
 
-    def e2e_step(s):
+    def e2e_eager(s):
         packed.upload()
         step(s, packed.views)
         host_out.copy_(out, non_blocking=True)
         stream.synchronize()
 
-    for i in range(args.warmup):
-        e2e_step(sets[i % n_sets])
-    barrier()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(args.steps):
-        e2e_step(sets[i % n_sets])
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms, _ = reduce_max_sum(e0.elapsed_time(e1), 0.0, dev)
+    # The same step as a serving loop runs it: the upload, the public decode_step call and
+    # the download captured once in a CUDA graph per pool copy, then one replay and one
+    # synchronisation per step (host inputs refreshed in the pinned buffer in between).
+    graphs = []
+    cap = torch.cuda.Stream(dev)
+    for s in sets:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            packed.upload()
+            step(s, packed.views)
+            host_out.copy_(out, non_blocking=True)
+        graphs.append(g)
+
+    def e2e_graph(i):
+        graphs[i % n_sets].replay()
+        stream.synchronize()
+
+    def timed(fn, arg_of):
+        for i in range(args.warmup):
+            fn(arg_of(i))
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(args.steps):
+            fn(arg_of(i))
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms, _ = reduce_max_sum(e0.elapsed_time(e1), 0.0, dev)
+        return ms
+
+    e2e_ms = timed(e2e_graph, lambda i: i)
+    eager_ms = timed(e2e_eager, lambda i: sets[i % n_sets])
     e2e_tbps = total_bytes / (e2e_ms * 1e-3) / 1e12
     gq.check_device_error()
+    del graphs
 
     achieved_gbs = nbytes["decode"] / (decode_us * 1e-6) / 1e9
     units = int(inp_cpu.seq_lens.to(torch.int64).sum())
@@ -669,7 +702,11 @@ def run_ours(args, rank, world, local):
         "config": {**_config_keys(inp_cpu, world), "l2": l2_desc},
         "e2e": {"value": e2e_tbps, "unit": "TB/s", "h2d_bytes_per_step": packed.payload,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps,
-                "copies_per_step": "1 host-to-device (packed inputs) + 1 device-to-host (out)"},
+                "copies_per_step": "1 host-to-device (packed inputs) + 1 device-to-host (out)",
+                "how": "upload, decode_step and download captured in a CUDA graph; one replay and one "
+                       "stream synchronisation per step",
+                "eager_ms_per_step": eager_ms / args.steps,
+                "eager_value": total_bytes / (eager_ms * 1e-3) / 1e12},
         "gpu_launches": int(launches),
         "roofline": {"bound": "hbm", "kernel": decode_kernel_for(inp_cpu),
                      "achieved": achieved_gbs, "peak": peak, "unit": "GB/s",
@@ -690,6 +727,40 @@ def run_ours(args, rank, world, local):
     return line
 
 
+def run_profile(args):
+    """Only --warmup + --steps decode launches of the workload (bf16 or e4m3 cache) on two
+    rotated pool copies: the small, self-contained case ncu captures are taken of.
+    Prints no JSON line."""
+    import gqa_decode_attention_04_b200 as gq
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    inp = make_inputs(args.workload, seed=1000 + args.workload, device=dev, poison=False)
+    sets, _ = _pool_sets(inp, dev)
+    sets = sets[:2]
+    out = torch.empty((inp.num_seqs, inp.num_heads, inp.head_dim), dtype=torch.bfloat16, device=dev)
+    if args.profile == "fp8":
+        ks = (inp.k_pages.float().abs().amax(dim=(0, 2, 3)) / 448.0).clamp(min=1e-30).contiguous()
+        vs = (inp.v_pages.float().abs().amax(dim=(0, 2, 3)) / 448.0).clamp(min=1e-30).contiguous()
+        pools = []
+        for st in sets:
+            kq = torch.empty(st.k_pages.shape, dtype=torch.uint8, device=dev)
+            vq = torch.empty(st.v_pages.shape, dtype=torch.uint8, device=dev)
+            gq.quantize_pages_fp8(st.k_pages, kq, ks)
+            gq.quantize_pages_fp8(st.v_pages, vq, vs)
+            pools.append((kq, vq))
+        del sets[1:]
+        st = sets[0]
+        for i in range(args.warmup + args.steps):
+            kq, vq = pools[i % 2]
+            gq.paged_decode_attn_fp8(st.q, kq, vq, ks, vs, st.block_table, st.seq_lens, out=out, scale=st.scale)
+    else:
+        for i in range(args.warmup + args.steps):
+            st = sets[i % 2]
+            gq.paged_decode_attn(st.q, st.k_pages, st.v_pages, st.block_table, st.seq_lens, out=out, scale=st.scale)
+    torch.cuda.synchronize()
+    gq.check_device_error()
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -700,6 +771,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fp8", action="store_true", help="skip the 8-bit cache entries")
     ap.add_argument("--headline-only", action="store_true", help="skip the other workloads")
+    ap.add_argument("--profile", choices=["bf16", "fp8"],
+                    help="only run --warmup + --steps decode launches of --workload (ncu captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -713,6 +786,9 @@ def main():
         return
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA GPU for --impl ours")
+    if args.profile:
+        run_profile(args)
+        return
     rank, world, local = setup_dist(args.gpus)
     try:
         line = run_ours(args, rank, world, local)
