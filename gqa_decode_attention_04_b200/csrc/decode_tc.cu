@@ -40,10 +40,12 @@
 //     masks its row's window (the sequence up to its own token) from the stage's
 //     remaining length, and tile rows past the group get an empty window.
 //   * 8-bit cache (the F8 instantiation): the producers copy each block's e4m3 codes into
-//     a ring of raw stages; two converter warps widen them (exactly) to fp16 in the stage
-//     layout the MMAs read, and convert each piece's query tile from bf16 to fp16 in
-//     place, so both MMAs run kind::f16 on fp16 operands (P is packed as fp16).  The kv
-//     head's K scale joins the score scale of a piece, its V scale the piece-end output.
+//     a ring of raw stages; the S warp widens K (exactly) to fp16 in the tile layout its
+//     MMA reads, and converts each piece's query tile from bf16 to fp16 in place, just
+//     before issuing; the P V warp widens V for a block while the softmax works on it.
+//     Both MMAs run kind::f16 on fp16 operands (P is packed as fp16).  The kv head's K
+//     scale joins the score scale of a piece, its V scale the piece-end output.  (Two
+//     extra converter warps measured slower: 14 warps cap registers at 128.)
 //   * Safety: every wait is bounded; on a timeout all warps leave their loops, the MMA
 //     warps wait for their issued MMAs, and TMEM is released before exit.
 #include <type_traits>
@@ -67,10 +69,6 @@ constexpr int kStgFloats = 16 * 36;  // piece-end staging per softmax warp
 constexpr int kTcWarps = 12;
 constexpr int kTcThreads = 32 * kTcWarps;
 constexpr int kWarpProducer = 8, kWarpS = 9, kWarpPV = 10, kWarpProducer2 = 11;
-// 8-bit cache: warps 12 and 13 convert codes (even and odd blocks).
-constexpr int kTcWarpsF8 = 14;
-constexpr int kTcThreadsF8 = 32 * kTcWarpsF8;
-constexpr int kWarpConv = 12;
 constexpr float kTcRescale = 8.0f;
 
 template <int D, bool F8 = false>
@@ -116,13 +114,13 @@ struct TcCursor {
 // segment (at most 128 rows); row r sees the sequence up to its own token.
 // F8: the cache holds e4m3 codes with one scale per kv head for K and for V.
 template <int D, bool MQ, bool F8 = false>
-__global__ void __launch_bounds__(F8 ? kTcThreadsF8 : kTcThreads, 1)
+__global__ void __launch_bounds__(kTcThreads, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                  const __grid_constant__ CUtensorMap tmap_q, const DecodeParams p) {
   using GE = TcGeo<D, F8>;
   constexpr int S = GE::kStages;
   constexpr int RS = GE::kRawStages;
-  constexpr int NW = F8 ? kTcWarpsF8 : kTcWarps;
+  constexpr int NW = kTcWarps;
   static_assert(!(F8 && MQ), "the 8-bit cache serves one query token per sequence");
   extern __shared__ uint8_t smem_raw[];
   __shared__ int64_t s_wtot[NW];
@@ -132,12 +130,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
   __shared__ int64_t s_start_base;
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
-  // Pieces whose query copy has been issued (producers) and, with the 8-bit cache,
-  // converted (converters).  A parity wait on an mbarrier is only exact if the waiter
-  // is at most one phase ahead; the two producers (and the two converters) take pieces
-  // in turns, so the one starting piece k first waits for these counters to show that
-  // piece k - 1 went through, which puts the barrier at most one phase behind.
-  __shared__ int s_qissued, s_qconverted;
+  // Pieces whose query copy has been issued.  A parity wait on an mbarrier is only exact
+  // if the waiter is at most one phase ahead; the two producers take pieces in turns, so
+  // the one starting piece k first waits for this counter to show that piece k - 1's
+  // copy was issued, which puts the barrier at most one phase behind.
+  __shared__ int s_qissued;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int B = p.num_seqs;
@@ -168,7 +165,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
     s_start_b = -1;
     s_abort = 0;
     s_qissued = 0;
-    s_qconverted = 0;
   }
   __syncthreads();
   int64_t T = 0;
@@ -232,10 +228,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
   const uint32_t ofree_bar = pv_bar + 8 * kTcBufs;       // softmax (256) -> P V warp, a piece's O is read
   const uint32_t drain_bar = ofree_bar + 8;       // MMA commit at exit
   const uint32_t wg_bar = drain_bar + 8;          // rendezvous of both softmax warpgroups (256)
-  const uint32_t raw_full = wg_bar + 8;           // F8: [RS] producer -> converter (codes landed)
-  const uint32_t raw_empty = raw_full + 8 * RS;   // F8: [RS] converter -> producer
-  const uint32_t qconv_bar = raw_empty + 8 * RS;  // F8: converter -> S warp (piece k's Q in fp16: phase k)
-  const uint32_t bars_end = qconv_bar + (F8 ? 8 : 0);
+  const uint32_t raw_full = wg_bar + 8;           // F8: [RS] producer -> S and P V warps (codes landed)
+  const uint32_t raw_empty = raw_full + 8 * RS;   // F8: [RS] S warp (K) and P V warp (V) converted -> producer
+  const uint32_t bars_end = raw_empty + 8 * RS;
   // Piece-end staging: per softmax warp 16 rows x 36 floats, so a warp writes whole
   // 128-byte row segments of its 32 rows (16 rows per round) instead of one row per lane.
   float* const stg_all = reinterpret_cast<float*>(base_ptr + ((bars_end - ring + 127u) & ~127u));
@@ -258,9 +253,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
     if constexpr (F8) {
       for (int s = 0; s < RS; ++s) {
         ptx::mbar_init(raw_full + 8 * s, 1);
-        ptx::mbar_init(raw_empty + 8 * s, 1);
+        ptx::mbar_init(raw_empty + 8 * s, 2);
       }
-      ptx::mbar_init(qconv_bar, 1);
     }
     ptx::fence_mbarrier_init();
   }
@@ -285,6 +279,43 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
   auto abort_all = [&](uint32_t bit) {
     atomicOr(p.err, bit);
     atomicExch(&s_abort, 1);
+  };
+  // 8-bit cache: one warp widens one tensor's codes of a block (raw stage, 128-byte
+  // swizzled rows) into the 16-bit tile its MMA reads ([group][64 rows][128 B], swizzled).
+  // Lane (t, c): 8 lanes take 8 tokens of one 16-code chunk, so the swizzled reads and
+  // writes hit distinct banks.
+  auto convert_tile = [&](uint32_t raw_tile, uint32_t tile) {
+    constexpr int CPT = D / 16;               // 16-code chunks per token
+    constexpr int ITERS = kTcBlk * CPT / 32;  // chunks per lane
+    constexpr int BATCH = 8;                  // chunks loaded before any is converted (latency)
+    const uint8_t* rb = base_ptr + (raw_tile - ring);
+    uint8_t* fb = base_ptr + (tile - ring);
+    const int tlo = lane & 7, cq = lane >> 3;
+#pragma unroll
+    for (int i0 = 0; i0 < ITERS; i0 += BATCH) {
+      uint4 x[BATCH];
+#pragma unroll
+      for (int j = 0; j < BATCH; ++j) {
+        const int it = i0 + j;
+        const int c = cq + 4 * (it % (CPT / 4));  // head dims 16 c .. 16 c + 15
+        const int tok = 8 * (it / (CPT / 4)) + tlo;
+        const int rrow = tok / (128 / D);
+        const int rc = (tok % (128 / D)) * CPT + c;
+        x[j] = *reinterpret_cast<const uint4*>(rb + rrow * 128 + ((rc ^ (rrow & 7)) << 4));
+      }
+#pragma unroll
+      for (int j = 0; j < BATCH; ++j) {
+        const int it = i0 + j;
+        const int c = cq + 4 * (it % (CPT / 4));
+        const int tok = 8 * (it / (CPT / 4)) + tlo;
+        const int cc = 2 * (c % 4);  // 8-value chunk of its 64-column group
+        uint8_t* dst = fb + (c / 4) * GE::kGroupBytes + tok * 128;
+        *reinterpret_cast<uint4*>(dst + ((cc ^ (tok & 7)) << 4)) =
+            make_uint4(ptx::e4m3x2_lo(x[j].x), ptx::e4m3x2_hi(x[j].x), ptx::e4m3x2_lo(x[j].y), ptx::e4m3x2_hi(x[j].y));
+        *reinterpret_cast<uint4*>(dst + (((cc + 1) ^ (tok & 7)) << 4)) =
+            make_uint4(ptx::e4m3x2_lo(x[j].z), ptx::e4m3x2_hi(x[j].z), ptx::e4m3x2_lo(x[j].w), ptx::e4m3x2_hi(x[j].w));
+      }
+    }
   };
 
   if (warp == kWarpProducer || warp == kWarpProducer2) {
@@ -499,13 +530,51 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
     for (int64_t n = 0; n < total; ++n) {
       if (__any_sync(0xffffffffu, aborted())) break;  // warp-uniform
       const int stage = static_cast<int>(n % S);
-      bool ok = ptx::mbar_wait_bounded(full_bar + 8 * stage, static_cast<uint32_t>((n / S) & 1), limit);
-      const TcStageInfo si = info[stage];
-      if (ok && (si.flags & kTcFirst))  // (8-bit cache: once the converters have made Q fp16)
-        ok = ptx::mbar_wait_bounded(F8 ? qconv_bar : qfull_bar, static_cast<uint32_t>(si.piece & 1), limit);
-      if (ok && n >= kTcBufs)
-        ok = ptx::mbar_wait_bounded(pv_bar + 8 * (n % kTcBufs),
-                                    static_cast<uint32_t>(((n - kTcBufs) / kTcBufs) & 1), limit);
+      bool ok;
+      TcStageInfo si;
+      if constexpr (F8) {
+        // Block n's codes have landed and the stage's previous block is consumed (its P V is
+        // complete); at a piece start also the piece's Q copy (pieces in order: exact parity).
+        const int rst = static_cast<int>(n % RS);
+        ok = ptx::mbar_wait_bounded(raw_full + 8 * rst, static_cast<uint32_t>((n / RS) & 1), limit);
+        if (ok && n >= S) ok = ptx::mbar_wait_bounded(empty_bar + 8 * stage, static_cast<uint32_t>((n / S - 1) & 1), limit);
+        si = rinfo[rst];
+        if (ok && (si.flags & kTcFirst)) ok = ptx::mbar_wait_bounded(qfull_bar, static_cast<uint32_t>(si.piece & 1), limit);
+        if (!__all_sync(0xffffffffu, ok)) {
+          if (lane == 0) abort_all(kErrTimeout);
+          break;
+        }
+        if (si.flags & kTcFirst) {  // the piece's query tile, bf16 -> fp16 in place
+          uint4* qv = reinterpret_cast<uint4*>(base_ptr + (qbuf - ring));
+          for (int k = lane; k < GE::kQTile / 16; k += 32) {
+            uint4 x = qv[k];
+            x.x = ptx::bf16x2_to_f16x2(x.x);
+            x.y = ptx::bf16x2_to_f16x2(x.y);
+            x.z = ptx::bf16x2_to_f16x2(x.z);
+            x.w = ptx::bf16x2_to_f16x2(x.w);
+            qv[k] = x;
+          }
+        }
+        convert_tile(raw + rst * GE::kRawStage, ring + stage * GE::kStage);
+        if (lane == 0) {
+          info[stage] = si;
+          __threadfence_block();
+        }
+        ptx::fence_proxy_async_smem();  // the MMA reads the converted tiles through the async proxy
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(raw_empty + 8 * rst);
+        if (n >= kTcBufs)
+          ok = ptx::mbar_wait_bounded(pv_bar + 8 * (n % kTcBufs),
+                                      static_cast<uint32_t>(((n - kTcBufs) / kTcBufs) & 1), limit);
+      } else {
+        ok = ptx::mbar_wait_bounded(full_bar + 8 * stage, static_cast<uint32_t>((n / S) & 1), limit);
+        si = info[stage];
+        if (ok && (si.flags & kTcFirst))
+          ok = ptx::mbar_wait_bounded(qfull_bar, static_cast<uint32_t>(si.piece & 1), limit);
+        if (ok && n >= kTcBufs)
+          ok = ptx::mbar_wait_bounded(pv_bar + 8 * (n % kTcBufs),
+                                      static_cast<uint32_t>(((n - kTcBufs) / kTcBufs) & 1), limit);
+      }
       if (!__all_sync(0xffffffffu, ok)) {
         if (lane == 0) abort_all(kErrTimeout);
         break;
@@ -544,10 +613,28 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
       if (__any_sync(0xffffffffu, aborted())) break;  // warp-uniform
       const int k = static_cast<int>(m % kTcBufs);
       const int stage = static_cast<int>(m % S);
-      bool ok = ptx::mbar_wait_bounded(pfull_bar + 8 * k, static_cast<uint32_t>((m / kTcBufs) & 1), limit);
-      // V_m landed before S_m was issued; observing the copy barrier here as well orders
-      // the TMA writes before this warp's own stores and MMAs (it has already completed).
-      if (ok) ok = ptx::mbar_wait_bounded(full_bar + 8 * stage, static_cast<uint32_t>((m / S) & 1), limit);
+      bool ok;
+      if constexpr (F8) {
+        // Widen V_m while the softmax works on block m: its codes have landed and this
+        // warp's P V of the stage's previous block is complete.
+        const int rst = static_cast<int>(m % RS);
+        ok = ptx::mbar_wait_bounded(raw_full + 8 * rst, static_cast<uint32_t>((m / RS) & 1), limit);
+        if (ok && m >= S) ok = ptx::mbar_wait_bounded(empty_bar + 8 * stage, static_cast<uint32_t>((m / S - 1) & 1), limit);
+        if (!__all_sync(0xffffffffu, ok)) {
+          if (lane == 0) abort_all(kErrTimeout);
+          break;
+        }
+        convert_tile(raw + rst * GE::kRawStage + GE::kRawTile, ring + stage * GE::kStage + GE::kTile);
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(raw_empty + 8 * rst);
+        ok = ptx::mbar_wait_bounded(pfull_bar + 8 * k, static_cast<uint32_t>((m / kTcBufs) & 1), limit);
+      } else {
+        ok = ptx::mbar_wait_bounded(pfull_bar + 8 * k, static_cast<uint32_t>((m / kTcBufs) & 1), limit);
+        // V_m landed before S_m was issued; observing the copy barrier here as well orders
+        // the TMA writes before this warp's own stores and MMAs (it has already completed).
+        if (ok) ok = ptx::mbar_wait_bounded(full_bar + 8 * stage, static_cast<uint32_t>((m / S) & 1), limit);
+      }
       const TcStageInfo si = info[stage];  // the stage is held until this P V completes
       const bool first = si.flags & kTcFirst;
       if (ok && first && si.piece > 0)
@@ -594,94 +681,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
     }
     __syncwarp();
     ptx::mbar_wait_bounded(drain_bar, 0, limit);
-  } else if (F8 && warp >= kWarpConv) {
-    // ============================================================ converter warps (8-bit cache)
-    // Converter c takes the blocks i with i % 2 == c: once the block's codes have landed
-    // (raw stage i % RS) and the MMA stage i % S is free (the P V of block i - S is
-    // complete), it widens the K and V codes to fp16 in the tile layout the MMAs read,
-    // copies the block's descriptor, and publishes the stage after a proxy fence (the MMAs
-    // read shared memory through the async proxy).  At a piece start it first converts
-    // the piece's query tile from bf16 to fp16 in place.
-    const uint32_t cid = static_cast<uint32_t>(warp - kWarpConv);
-    constexpr int CPT = D / 16;               // 16-code chunks per token
-    constexpr int ITERS = kTcBlk * CPT / 32;  // chunks per lane, block and tensor
-    const int tlo = lane & 7, cq = lane >> 3;
-    int rstage = 0, stage = 0;
-    uint32_t rround = 0, round = 0;
-    for (int64_t i = 0; i < total; ++i) {
-      if ((static_cast<uint32_t>(i) & 1u) == cid) {
-        if (__any_sync(0xffffffffu, aborted())) break;  // warp-uniform
-        bool ok = ptx::mbar_wait_bounded(raw_full + 8 * rstage, rround & 1u, limit);
-        if (ok && round > 0) ok = ptx::mbar_wait_bounded(empty_bar + 8 * stage, (round - 1) & 1u, limit);
-        if (!__all_sync(0xffffffffu, ok)) {
-          if (lane == 0) abort_all(kErrTimeout);
-          break;
-        }
-        const TcStageInfo si = rinfo[rstage];
-        if (si.flags & kTcFirst) {
-          // The producer loads a piece's Q only after the previous piece's S MMAs are done.
-          // Once piece - 1's Q has been converted (its copy landed), the parity wait can
-          // only be met by this piece's copy.
-          ok = ptx::wait_counter(&s_qconverted, si.piece, limit);
-          if (ok) ok = ptx::mbar_wait_bounded(qfull_bar, static_cast<uint32_t>(si.piece & 1), limit);
-          if (!__all_sync(0xffffffffu, ok)) {
-            if (lane == 0) abort_all(kErrTimeout);
-            break;
-          }
-          uint4* qv = reinterpret_cast<uint4*>(base_ptr + (qbuf - ring));
-          for (int k = lane; k < GE::kQTile / 16; k += 32) {
-            uint4 x = qv[k];
-            x.x = ptx::bf16x2_to_f16x2(x.x);
-            x.y = ptx::bf16x2_to_f16x2(x.y);
-            x.z = ptx::bf16x2_to_f16x2(x.z);
-            x.w = ptx::bf16x2_to_f16x2(x.w);
-            qv[k] = x;
-          }
-          ptx::fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            ptx::mbar_arrive(qconv_bar);
-            *reinterpret_cast<volatile int*>(&s_qconverted) = si.piece + 1;
-          }
-        }
-        const uint8_t* rb = base_ptr + (raw - ring) + rstage * GE::kRawStage;
-        uint8_t* fb = base_ptr + stage * GE::kStage;
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {  // K, then V
-#pragma unroll 4
-          for (int it = 0; it < ITERS; ++it) {
-            // 16-code chunk c (head dims 16 c .. 16 c + 15) of token tok: 8 lanes take 8
-            // tokens of one chunk, so the swizzled reads and writes hit distinct banks
-            const int c = cq + 4 * (it % (CPT / 4));
-            const int tok = 8 * (it / (CPT / 4)) + tlo;
-            const int rrow = tok / (128 / D);
-            const int rc = (tok % (128 / D)) * CPT + c;
-            const uint4 x = *reinterpret_cast<const uint4*>(rb + t * GE::kRawTile + rrow * 128 + ((rc ^ (rrow & 7)) << 4));
-            const int cc = 2 * (c % 4);  // 8-value chunk of its 64-column group
-            uint8_t* dst = fb + t * GE::kTile + (c / 4) * GE::kGroupBytes + tok * 128;
-            *reinterpret_cast<uint4*>(dst + ((cc ^ (tok & 7)) << 4)) =
-                make_uint4(ptx::e4m3x2_lo(x.x), ptx::e4m3x2_hi(x.x), ptx::e4m3x2_lo(x.y), ptx::e4m3x2_hi(x.y));
-            *reinterpret_cast<uint4*>(dst + (((cc + 1) ^ (tok & 7)) << 4)) =
-                make_uint4(ptx::e4m3x2_lo(x.z), ptx::e4m3x2_hi(x.z), ptx::e4m3x2_lo(x.w), ptx::e4m3x2_hi(x.w));
-          }
-        }
-        if (lane == 0) info[stage] = si;
-        ptx::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          ptx::mbar_arrive(full_bar + 8 * stage);
-          ptx::mbar_arrive(raw_empty + 8 * rstage);
-        }
-      }
-      if (++rstage == RS) {
-        rstage = 0;
-        ++rround;
-      }
-      if (++stage == S) {
-        stage = 0;
-        ++round;
-      }
-    }
   } else {
     // ============================================================ softmax warpgroups
     // Thread t: warpgroup g = t / 128 owns tokens [32 g, 32 g + 32) of every block and its
@@ -734,21 +733,22 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_consta
       ptx::tc_fence_after();
       const int stg = is;
       if (++is == S) is = 0;
-      const int flags = info[stg].flags;
-      const uint64_t vmask = info[stg].vmask;
+      const TcStageInfo* const ip = &info[stg];
+      const int flags = ip->flags;
+      const uint64_t vmask = ip->vmask;
       // What a piece end needs of this block, read while its stage is held (the stage is
       // refilled once the block's P V completes, which needs this thread's P).
       int pe_b = 0, pe_seg = 0;
       if (flags & kTcLast) {
-        pe_b = info[stg].b;
-        pe_seg = info[stg].seg;
+        pe_b = ip->b;
+        pe_seg = ip->seg;
       }
       const bool first = flags & kTcFirst;
       if (first) {
         mref = -INFINITY;
         lsum = 0.f;
         if constexpr (F8) {
-          sl2 = p.scale_log2 * __ldg(p.k_scales + info[stg].seg / p.n_ht);
+          sl2 = p.scale_log2 * __ldg(p.k_scales + ip->seg / p.n_ht);
           pos = sl2 >= 0.f;
         }
       }
@@ -1131,7 +1131,7 @@ constexpr size_t tc_smem_bytes() {
   using GE = TcGeo<D, F8>;
   return 1024 + static_cast<size_t>(GE::kStages) * GE::kStage + static_cast<size_t>(GE::kRawStages) * GE::kRawStage +
          GE::kQTile + (GE::kStages + GE::kRawStages) * sizeof(TcStageInfo) + 16 * GE::kStages +
-         16 * GE::kRawStages + 8 + 24 * kTcBufs + 64 + 128 + kTcSoftThreads / 32 * kStgFloats * sizeof(float);
+         16 * GE::kRawStages + 24 * kTcBufs + 64 + 128 + kTcSoftThreads / 32 * kStgFloats * sizeof(float);
 }
 static_assert(tc_smem_bytes<128, true>() <= 227 * 1024 && tc_smem_bytes<64, true>() <= 227 * 1024 &&
                   tc_smem_bytes<128>() <= 227 * 1024 && tc_smem_bytes<64>() <= 227 * 1024,
@@ -1152,7 +1152,7 @@ cudaError_t launch_tc_t(const DecodeParams& p, const CUtensorMap& tk, const CUte
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(F8 ? kTcThreadsF8 : kTcThreads);
+  cfg.blockDim = dim3(kTcThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];

@@ -236,7 +236,9 @@ __device__ __forceinline__ void attend_subchunk(uint32_t kb, uint32_t vb, int nv
 // 4q .. 4q + 3 of a 16-value chunk: the contraction over head_dim uses that order for
 // K (the q fragments follow it), and for V^T each converted pair is transposed with
 // movmatrix, which puts dimension 16 mt + 4 (g >> 1) + (g & 1) (+ 2 for row g + 8) on
-// M-row g of O^T tile mt.
+// M-row g of O^T tile mt.  (V^T from the transposing ldmatrix with one byte permute per
+// register instead -- fewer instructions -- measured slower: 270.5 against 262.6 us on
+// the long-context batch.)
 template <int D, int NT>
 __device__ __forceinline__ void attend_subchunk_f8(uint32_t kb, uint32_t vb, int nvalid,
                                                    const uint32_t (&ofs)[D / 32], const uint32_t (&qf)[D / 16][NT][2],
@@ -353,6 +355,17 @@ __device__ __forceinline__ void attend_subchunk_f8(uint32_t kb, uint32_t vb, int
 #define GQA_SMEM_PER_SM_KB 212
 #endif
 constexpr int kWsCtasPerSm = GQA_CTAS_TOKEN_SPLIT;
+// The 8-bit cache moves half the bytes per stage; its launch shape is set on its own.
+// Three CTAs per SM (3 stages each, 96 registers) measured faster than two (5 stages):
+// 242.5 against 263.6 us on the long-context batch, 320 against 354 us on the
+// continuous batch, 45.8 against 45.2 us on the GQA serving batch.
+#ifndef GQA_F8_CTAS
+#define GQA_F8_CTAS 3
+#endif
+#ifndef GQA_F8_SMEM_PER_SM_KB
+#define GQA_F8_SMEM_PER_SM_KB 220
+#endif
+constexpr int kWsCtasPerSmF8 = GQA_F8_CTAS;
 
 // D: head_dim.  NT: 8-head n-tiles per consumer (each consumer takes one 16-token
 // sub-chunk of every stage for all rows).  C: consumer warps.  S: stages.  MQ:
@@ -362,7 +375,7 @@ constexpr int kWsCtasPerSm = GQA_CTAS_TOKEN_SPLIT;
 // (p.k_scales, p.v_scales); the K scale joins the score scale of a piece, the V scale
 // the output of its combine.
 template <int D, int NT, int C, int S, bool MQ, bool F8>
-__global__ void __launch_bounds__((C + 2) * 32, kWsCtasPerSm)
+__global__ void __launch_bounds__((C + 2) * 32, F8 ? kWsCtasPerSmF8 : kWsCtasPerSm)
 decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
                  const __grid_constant__ CUtensorMap tmap_v, const DecodeParams p) {
   using G_ = Geo<D, F8>;
@@ -958,8 +971,8 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
           }
       }
       // Head h of this consumer goes to its K sub-chunk tile (h < HS) or its V one.
-      // O^T M-row g of tile mt is dimension 16 mt + g (bf16), or 16 mt + dg with the
-      // 8-bit cache's order (row g + 8: 16 mt + g + 8, or 16 mt + dg + 2).
+      // O^T M-row g of tile mt is dimension 16 mt + g (bf16; row g + 8: 16 mt + g + 8),
+      // with the 8-bit cache 16 mt + dg (row g + 8: 16 mt + dg + d8).
       const int dg = F8 ? 4 * (g >> 1) + (g & 1) : g;
       constexpr int d8 = F8 ? 2 : 8;
 #pragma unroll
@@ -992,7 +1005,8 @@ struct Cfg {
   static constexpr int kNH = 8 * NT;
   // per-stage (max, sum) hand-off area, sized for up to 8 stages
   static constexpr size_t kMerge = static_cast<size_t>(8 * C * kNH * 2) * sizeof(float);
-  static constexpr size_t kBudget = static_cast<size_t>(GQA_SMEM_PER_SM_KB) * 1024 / kWsCtasPerSm;
+  static constexpr size_t kBudget = F8 ? static_cast<size_t>(GQA_F8_SMEM_PER_SM_KB) * 1024 / kWsCtasPerSmF8
+                                      : static_cast<size_t>(GQA_SMEM_PER_SM_KB) * 1024 / kWsCtasPerSm;
   static constexpr size_t kQBytes = static_cast<size_t>(kNH) * D * 2;
   static constexpr int kStagesRaw =
       static_cast<int>((kBudget - kMerge) / (Geo<D, F8>::kStageBytes + kQBytes));
@@ -1065,7 +1079,7 @@ DecodePlan plan_decode(int head_dim, int group, bool mq_rows, bool fp8) {
     pl.consumers = 4;
     pl.heads_per_seg = 8;
     pl.n_ht = (group + 7) / 8;
-    pl.ctas_per_sm = kWsCtasPerSm;
+    pl.ctas_per_sm = kWsCtasPerSmF8;
     if (head_dim == 64) fill<64, 1, 4, true>(pl); else fill<128, 1, 4, true>(pl);
     return pl;
   }
