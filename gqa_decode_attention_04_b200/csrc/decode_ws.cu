@@ -354,6 +354,7 @@ __device__ __forceinline__ void attend_subchunk_f8(uint32_t kb, uint32_t vb, int
 #ifndef GQA_SMEM_PER_SM_KB
 #define GQA_SMEM_PER_SM_KB 212
 #endif
+
 constexpr int kWsCtasPerSm = GQA_CTAS_TOKEN_SPLIT;
 // The 8-bit cache moves half the bytes per stage; its launch shape is set on its own.
 // Three CTAs per SM (3 stages each, 96 registers) measured faster than two (5 stages):
@@ -634,33 +635,39 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
           if constexpr (MQ) {
             // One copy per query token (its group's rows are contiguous in q); a
             // segment is the whole kv head (ht == 0) when there are several tokens.
-            for (int i = lane - kSubChunks; i >= 0 && i < p.q_len; i += 32 - kSubChunks)
+            for (int i = lane - 2 * kSubChunks; i >= 0 && i < p.q_len; i += 32 - 2 * kSubChunks)
               ptx::bulk_load(ptx::smem_u32(qbuf + stage * kQBytes) + i * p.group * D * 2,
                              p.q + seq_row(cu.b, kvh, i * p.group) * D,
                              static_cast<uint32_t>(p.group) * D * 2u, full_bar + 8 * stage);
-          } else if (lane == kSubChunks) {
+          } else if (lane == 2 * kSubChunks) {
             ptx::bulk_load(ptx::smem_u32(qbuf + stage * kQBytes), p.q + seq_row(cu.b, kvh, ht * NH) * D,
                            q_rows_bytes(cu), full_bar + 8 * stage);
           }
         }
       }
-      if (ok && !p.arm_without_copy) {
-        const int kvh = cu.seg / p.n_ht;
-        const int row = (page * p.num_kv_heads + kvh) * p.page_size +
-                        (cu.blk * kBlock + lane * kChunk) % p.page_size;
-        const uint32_t kdst = ring + stage * G_::kStageBytes + lane * G_::kSubBytes;
-        const uint32_t vdst = kdst + G_::kTileBytes;
-        const uint32_t bar = full_bar + 8 * stage;
-        if constexpr (F8) {
-          // the codes viewed as 128-byte rows: a sub-chunk is 16 * D / 128 of them
-          const int row8 = row / (128 / D);
-          ptx::tma_load_2d(kdst, &tmap_k, bar, 0, row8, policy);
-          ptx::tma_load_2d(vdst, &tmap_v, bar, 0, row8, policy);
-        } else {
-          // one copy per tensor brings all head_dim/64 column boxes of the 16 rows
-          ptx::tma_load_3d(kdst, &tmap_k, bar, 0, row, 0, policy);
-          ptx::tma_load_3d(vdst, &tmap_v, bar, 0, row, 0, policy);
+      if constexpr (!F8) {
+        // bf16: lane l < 8 copies sub-chunk l % 4 of K (l < 4) or V (l >= 4), one copy per lane
+        // (a warp issues tiled copies faster the more of its lanes take part: 52.7 against
+        // 53.0 us on the GQA batch); lanes 0-3 hold the pages.
+        const int sc = lane & (kSubChunks - 1);
+        const int pg = __shfl_sync(0xffffffffu, page, sc);
+        if (lane < 2 * kSubChunks && ((submask >> sc) & 1u) && !p.arm_without_copy) {
+          const int kvh = cu.seg / p.n_ht;
+          const int row = (pg * p.num_kv_heads + kvh) * p.page_size + (cu.blk * kBlock + sc * kChunk) % p.page_size;
+          const bool is_v = lane >= kSubChunks;
+          const uint32_t dst = ring + stage * G_::kStageBytes + sc * G_::kSubBytes + (is_v ? G_::kTileBytes : 0);
+          // one copy brings all head_dim/64 column boxes of the 16 rows
+          ptx::tma_load_3d(dst, is_v ? &tmap_v : &tmap_k, full_bar + 8 * stage, 0, row, 0, policy);
         }
+      } else if (ok && !p.arm_without_copy) {
+        // e4m3 codes: lane l < 4 copies sub-chunk l of K and of V (eight lanes measured slower
+        // here: 248.4 against 241.7 us on the long-context batch).  The codes are 128-byte
+        // rows: a sub-chunk is 16 * D / 128 of them.
+        const int kvh = cu.seg / p.n_ht;
+        const int row = (page * p.num_kv_heads + kvh) * p.page_size + (cu.blk * kBlock + lane * kChunk) % p.page_size;
+        const uint32_t kdst = ring + stage * G_::kStageBytes + lane * G_::kSubBytes;
+        ptx::tma_load_2d(kdst, &tmap_k, full_bar + 8 * stage, 0, row / (128 / D), policy);
+        ptx::tma_load_2d(kdst + G_::kTileBytes, &tmap_v, full_bar + 8 * stage, 0, row / (128 / D), policy);
       }
       if (last) first_piece = false;
       if (i + 1 < total) {
