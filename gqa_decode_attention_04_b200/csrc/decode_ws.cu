@@ -51,8 +51,8 @@ struct Geo {
   static constexpr int kBoxes = D / 64;                      // bf16: 64-column (128-byte) boxes
   static constexpr int kBoxBytes = kChunk * 128;             // bf16: 16 rows x 128 bytes
   static constexpr int kSubBytes = kChunk * D * kElem;       // one 16-token K (or V) tile
-  static constexpr int kTileBytes = kSubChunks * kSubBytes;  // 64-token K (or V) tile
-  static constexpr int kStageBytes = 2 * kTileBytes;
+  // A stage: for each of the 4 sub-chunks its K and V tiles, adjacent
+  static constexpr int kStageBytes = 2 * kSubChunks * kSubBytes;
   // Query heads whose fp32 partial O (D floats each) fit one sub-chunk tile: a consumer
   // hands its partial to the epilogue in its own K and V sub-chunk tiles.
   static constexpr int kHeadsPerSub = kSubBytes / (4 * D);
@@ -78,6 +78,8 @@ __device__ __forceinline__ int eff_len(int L, int cap) { return L < 0 ? 0 : (L >
 struct Cursor {
   int b;     // sequence
   int seg;   // kv_head * n_ht + head_tile
+  int kvh;   // seg / n_ht
+  int ht;    // seg % n_ht
   int blk;   // block within the segment
   int nblk;  // blocks per segment of sequence b
   int len;   // effective context length of sequence b
@@ -94,8 +96,14 @@ __device__ __forceinline__ void walk_next(Cursor& c, int& next_len, const Decode
                                           int cap) {
   if (++c.blk < c.nblk) return;
   c.blk = 0;
-  if (++c.seg < segs) return;
-  c.seg = 0;
+  if (++c.seg < segs) {
+    if (++c.ht == p.n_ht) {
+      c.ht = 0;
+      ++c.kvh;
+    }
+    return;
+  }
+  c.seg = c.kvh = c.ht = 0;
   do {
     ++c.b;
     c.len = (c.b < p.num_seqs) ? eff_len(next_len, cap) : 0;
@@ -535,6 +543,8 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int64_t off = x0 - start_base;
     cu.seg = static_cast<int>(off / cu.nblk);
     cu.blk = static_cast<int>(off % cu.nblk);
+    cu.kvh = cu.seg / p.n_ht;
+    cu.ht = cu.seg - cu.kvh * p.n_ht;
   }
 
   if (warp == C) {
@@ -546,8 +556,11 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const uint64_t policy = ptx::policy_evict_first();
     // Block-table rows are read 32 entries at a time (one per lane) into a register
     // window, with the window needed next already in flight, so no TMA issue waits on
-    // a dependent global load.  Lane s < 4 owns sub-chunk s of every block.
+    // a dependent global load.  Lanes s and s + 4 (s < 4) look up sub-chunk s of every
+    // block; lane s owns its copy.
     const int ps = p.page_size;
+    const uint32_t pm = p.ps_magic;
+    const int psh = p.ps_shift;
     auto load_window = [&](int b, int k) -> int {
       const int e = 32 * k + lane;
       return (b >= 0 && b < B && e < p.max_blocks)
@@ -558,14 +571,16 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
     // length of the sequence after cu.b, loaded ahead of the cursor reaching it
     int next_len = (cu.b + 1 < B) ? __ldg(p.seq_lens + cu.b + 1) : 0;
     auto prefetch_after = [&](const Cursor& c, int k) {
-      const int entries = (c.len + ps - 1) / ps;
+      const int entries = c.len > 0 ? fast_div(c.len - 1, pm, psh) + 1 : 0;
       if (32 * (k + 1) < entries) { nb = c.b; nk = k + 1; }
       else if (c.seg + 1 < segs) { nb = c.b; nk = 0; }
       else { nb = c.b + 1; nk = 0; }
       nval = load_window(nb, nk);
     };
-    auto page_of = [&](const Cursor& c) -> int {
-      const int e0 = (c.blk * kBlock) / ps;
+    // The page of this lane's sub-chunk (lanes < 8; -1 past the sequence's end) and the
+    // sub-chunk's first token within it (toff).
+    auto page_of = [&](const Cursor& c, int& toff) -> int {
+      const int e0 = fast_div(c.blk * kBlock, pm, psh);
       const int k = e0 >> 5;
       if (c.b != wb || k != wk) {
         if (c.b == nb && k == nk) { wval = nval; }
@@ -575,24 +590,28 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
         prefetch_after(c, k);
       }
       const int t = c.blk * kBlock + (lane & 3) * kChunk;
-      const int src = (t / ps) - 32 * k;  // 0..31: a block never straddles two windows
-      const int pg = __shfl_sync(0xffffffffu, wval, src);
-      return (lane < kSubChunks && t < c.len) ? pg : -1;
+      const int e = fast_div(t, pm, psh);
+      toff = t - e * ps;
+      const int pg = __shfl_sync(0xffffffffu, wval, e - 32 * k);  // a block never straddles two windows
+      return (lane < 2 * kSubChunks && t < c.len) ? pg : -1;
     };
     // Bytes of a piece's query rows (contiguous in q): the token split stages them.
     auto q_rows_bytes = [&](const Cursor& c) -> uint32_t {
-      const int ht = c.seg % p.n_ht;
-      return static_cast<uint32_t>(min(NH, grp - ht * NH)) * D * 2u;
+      return static_cast<uint32_t>(min(NH, grp - c.ht * NH)) * D * 2u;
     };
-    int page = page_of(cu);
+    // Stage layout: sub-chunk s holds its K tile then its V tile (V then K when the
+    // paired map's lower pool is V), each kSubBytes.
+    const int pair = p.kv_pair;
+    int toff = 0;
+    int page = page_of(cu, toff);
+    int stage = 0;
+    uint32_t phase = 0;  // parity of the current pass over the ring
     int piece_blk0 = cu.blk;
     bool first_piece = true;
     int64_t seg_base = x0 - cu.blk;
     for (int64_t i = 0; i < total; ++i) {
-      const int stage = static_cast<int>(i % S);
       if (i >= S) {
-        const bool ok = ptx::mbar_wait_bounded(empty_bar + 8 * stage,
-                                               static_cast<uint32_t>((i / S - 1) & 1), limit);
+        const bool ok = ptx::mbar_wait_bounded(empty_bar + 8 * stage, phase ^ 1u, limit);
         if (!__all_sync(0xffffffffu, ok)) {
           if (lane == 0) atomicOr(p.err, kErrTimeout);
           // give copies still in flight a bounded chance to land, then leave
@@ -602,7 +621,7 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
         }
       }
       const int nvalid = min(kBlock, cu.len - cu.blk * kBlock);
-      const bool want = lane < kSubChunks && lane * kChunk < nvalid;
+      const bool want = lane < kSubChunks && lane * kChunk < nvalid;  // (page >= 0 there)
       const bool ok = want && page >= 0 && page < p.num_pages;
       const uint32_t submask = __ballot_sync(0xffffffffu, ok) & 0xFu;
       if (__any_sync(0xffffffffu, want && !ok) && lane == 0) atomicOr(p.err, kErrBounds);
@@ -631,7 +650,7 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
       __syncwarp();
       {
         if (first && !p.arm_without_copy) {
-          const int kvh = cu.seg / p.n_ht, ht = cu.seg % p.n_ht;
+          const int kvh = cu.kvh, ht = cu.ht;
           if constexpr (MQ) {
             // One copy per query token (its group's rows are contiguous in q); a
             // segment is the whole kv head (ht == 0) when there are several tokens.
@@ -645,35 +664,43 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
           }
         }
       }
-      if constexpr (!F8) {
-        // bf16: lane l < 8 copies sub-chunk l % 4 of K (l < 4) or V (l >= 4), one copy per lane
-        // (a warp issues tiled copies faster the more of its lanes take part: 52.7 against
-        // 53.0 us on the GQA batch); lanes 0-3 hold the pages.
+      {
         const int sc = lane & (kSubChunks - 1);
-        const int pg = __shfl_sync(0xffffffffu, page, sc);
-        if (lane < 2 * kSubChunks && ((submask >> sc) & 1u) && !p.arm_without_copy) {
-          const int kvh = cu.seg / p.n_ht;
-          const int row = (pg * p.num_kv_heads + kvh) * p.page_size + (cu.blk * kBlock + sc * kChunk) % p.page_size;
-          const bool is_v = lane >= kSubChunks;
-          const uint32_t dst = ring + stage * G_::kStageBytes + sc * G_::kSubBytes + (is_v ? G_::kTileBytes : 0);
-          // one copy brings all head_dim/64 column boxes of the 16 rows
-          ptx::tma_load_3d(dst, is_v ? &tmap_v : &tmap_k, full_bar + 8 * stage, 0, row, 0, policy);
+        // first pool row of the sub-chunk (page, kv head, token); lanes s and s + 4 agree
+        const int row = (page * p.num_kv_heads + cu.kvh) * ps + toff;
+        const uint32_t dst = ring + stage * G_::kStageBytes + sc * 2 * G_::kSubBytes;
+        const uint32_t bar = full_bar + 8 * stage;
+        if (p.arm_without_copy) {
+        } else if constexpr (!F8) {
+          // bf16: lane l < 8 copies sub-chunk l % 4 of K (l < 4) or V (l >= 4), all head_dim/64
+          // column boxes of the 16 rows in one copy (a warp issues tiled copies faster the
+          // more of its lanes take part: 52.7 against 53.0 us on the GQA batch)
+          if (lane < 2 * kSubChunks && ((submask >> sc) & 1u)) {
+            const bool is_v = lane >= kSubChunks;
+            ptx::tma_load_3d(dst + (is_v ? G_::kSubBytes : 0), is_v ? &tmap_v : &tmap_k, bar, 0, row, 0, policy);
+          }
+        } else if (ok) {
+          // e4m3 codes, 128-byte rows (a sub-chunk is 16 * D / 128 of them): lane s < 4
+          // copies sub-chunk s of both pools in one copy when they share a map, else of K
+          // and of V apart (eight lanes measured slower: 248.4 against 241.7 us on the
+          // long-context batch)
+          if (pair != 0) {
+            ptx::tma_load_3d(dst, &tmap_k, bar, 0, row / (128 / D), 0, policy);
+          } else {
+            ptx::tma_load_2d(dst, &tmap_k, bar, 0, row / (128 / D), policy);
+            ptx::tma_load_2d(dst + G_::kSubBytes, &tmap_v, bar, 0, row / (128 / D), policy);
+          }
         }
-      } else if (ok && !p.arm_without_copy) {
-        // e4m3 codes: lane l < 4 copies sub-chunk l of K and of V (eight lanes measured slower
-        // here: 248.4 against 241.7 us on the long-context batch).  The codes are 128-byte
-        // rows: a sub-chunk is 16 * D / 128 of them.
-        const int kvh = cu.seg / p.n_ht;
-        const int row = (page * p.num_kv_heads + kvh) * p.page_size + (cu.blk * kBlock + lane * kChunk) % p.page_size;
-        const uint32_t kdst = ring + stage * G_::kStageBytes + lane * G_::kSubBytes;
-        ptx::tma_load_2d(kdst, &tmap_k, full_bar + 8 * stage, 0, row / (128 / D), policy);
-        ptx::tma_load_2d(kdst + G_::kTileBytes, &tmap_v, full_bar + 8 * stage, 0, row / (128 / D), policy);
       }
       if (last) first_piece = false;
+      if (++stage == S) {
+        stage = 0;
+        phase ^= 1u;
+      }
       if (i + 1 < total) {
         walk_next(cu, next_len, p, segs, cap);
         if (cu.blk == 0) seg_base = x0 + i + 1;
-        page = page_of(cu);
+        page = page_of(cu, toff);
       }
     }
     return;
@@ -725,8 +752,8 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
           for (int c = 0; c < CPL; ++c) acc[c] = 0.f;
 #pragma unroll
           for (int jj = 0; jj < C; ++jj) {
-            const float* src = reinterpret_cast<const float*>(st + (h >= HS ? G_::kTileBytes : 0) +
-                                                              jj * G_::kSubBytes) + (h % HS) * D + d0;
+            const float* src = reinterpret_cast<const float*>(st + jj * 2 * G_::kSubBytes +
+                                                              (h >= HS ? G_::kSubBytes : 0)) + (h % HS) * D + d0;
 #pragma unroll
             for (int c = 0; c < CPL; ++c) acc[c] += wj[jj] * src[c];
           }
@@ -834,6 +861,8 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
 
   // ============================================================== consumer warps
   const int j = warp;
+  // sub-chunk j's K tile within its K|V pair (V first when the paired map's lower pool is V)
+  const uint32_t koff = p.kv_pair == 2 ? G_::kSubBytes : 0u;
   const int g = lane >> 2;
   const int q = lane & 3;
   uint32_t kofs[4], vofs[4];
@@ -925,14 +954,14 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const StageInfo si = info[stage];
     if (si.flags & kFirstOfPiece) load_q(si.b, si.seg, stage);
 
-    const uint32_t kst = ring + stage * G_::kStageBytes;
     if ((si.submask >> j) & 1) {
-      const uint32_t kb = kst + j * G_::kSubBytes;
+      const uint32_t sub = ring + stage * G_::kStageBytes + j * 2 * G_::kSubBytes;
+      const uint32_t kb = sub + koff, vb = sub + (G_::kSubBytes - koff);
       if constexpr (F8)
-        attend_subchunk_f8<D, NT>(kb, kb + G_::kTileBytes, min(kChunk, si.nvalid - j * kChunk), ofs8, qf, o, mref,
+        attend_subchunk_f8<D, NT>(kb, vb, min(kChunk, si.nvalid - j * kChunk), ofs8, qf, o, mref,
                                   lsum, sl2, g, q);
       else
-        attend_subchunk<D, NT, MQ>(kb, kb + G_::kTileBytes, min(kChunk, si.nvalid - j * kChunk),
+        attend_subchunk<D, NT, MQ>(kb, vb, min(kChunk, si.nvalid - j * kChunk),
                                    kofs, vofs, qf, o, mref, lsum, sl2, g, q, si.rem - j * kChunk, max_drop,
                                    cdrop);
     }
@@ -977,7 +1006,8 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
             mlj[h * 2 + 1] = lt[nt][e];
           }
       }
-      // Head h of this consumer goes to its K sub-chunk tile (h < HS) or its V one.
+      // Head h of this consumer goes to the first tile of its sub-chunk (h < HS) or the
+      // second.
       // O^T M-row g of tile mt is dimension 16 mt + g (bf16; row g + 8: 16 mt + g + 8),
       // with the 8-bit cache 16 mt + dg (row g + 8: 16 mt + dg + d8).
       const int dg = F8 ? 4 * (g >> 1) + (g & 1) : g;
@@ -987,8 +1017,8 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int h = nt * 8 + 2 * q + e;
-          float* row = reinterpret_cast<float*>(base_ptr + stage * G_::kStageBytes + (h >= HS ? G_::kTileBytes : 0) +
-                                                j * G_::kSubBytes) + (h % HS) * D;
+          float* row = reinterpret_cast<float*>(base_ptr + stage * G_::kStageBytes + j * 2 * G_::kSubBytes +
+                                                (h >= HS ? G_::kSubBytes : 0)) + (h % HS) * D;
 #pragma unroll
           for (int mt = 0; mt < MT; ++mt) {
             row[mt * 16 + dg] = o[mt][nt][e];

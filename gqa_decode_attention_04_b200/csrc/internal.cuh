@@ -57,7 +57,33 @@ struct DecodeParams {
   // kv head (k_scales, v_scales [Hk] fp32).  nullptr for a bf16 cache.
   const float* k_scales;
   const float* v_scales;
+  // mma.sync kernel, e4m3 codes: 0 = separate K and V tensor maps; otherwise the K map
+  // spans both pools with an outer coordinate of extent 2, one copy bringing a
+  // sub-chunk's K and V: 1 = K at coordinate 0, V at 1; 2 = V at 0, K at 1 (the V pool
+  // lies lower in memory).  Always 0 for a bf16 cache.
+  int kv_pair;
+  // floor(x / page_size) == umulhi(x, ps_magic) >> ps_shift for 0 <= x < 2^31.
+  uint32_t ps_magic;
+  int ps_shift;
 };
+
+// Multiply-and-shift constants of division by d (1 < d < 2^31) for dividends below
+// 2^31, after Granlund and Montgomery, "Division by invariant integers using
+// multiplication" (1994): with l = ceil(log2 d), m = ceil(2^(31 + l) / d) fits in 32 bits
+// and m * d - 2^(31 + l) < d <= 2^l, so floor(x * m / 2^(31 + l)) == floor(x / d).
+inline void divisor_magic(uint32_t d, uint32_t* magic, int* shift) {
+  int l = 0;
+  while ((uint64_t{1} << l) < d) ++l;
+  const uint64_t num = uint64_t{1} << (31 + l);
+  *magic = static_cast<uint32_t>((num + d - 1) / d);
+  *shift = l - 1;  // umulhi already drops 32 of the 31 + l bits
+}
+
+#ifdef __CUDACC__
+__device__ __forceinline__ int fast_div(int x, uint32_t magic, int shift) {
+  return static_cast<int>(__umulhi(static_cast<uint32_t>(x), magic) >> shift);
+}
+#endif
 
 struct AppendParams {
   const uint4* k_new;

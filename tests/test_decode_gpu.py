@@ -38,6 +38,9 @@ SMALL_CASES = [
     ([70], 96, 1, 128, 64),                        # G=96 (MQA, workload-3 shape)
     ([5, 0, 33], 8, 8, 128, 16),                   # MHA (G=1) and an empty sequence
     ([1000, 3, 500, 2048], 8, 1, 64, 16),          # D=64 long
+    ([700, 47, 96], 16, 4, 128, 48),               # G=4, ps=48: blocks straddle pages
+    ([1300, 81], 8, 1, 64, 80),                    # G=8, D=64, ps=80
+    ([2000, 239, 240, 241], 12, 2, 128, 240),      # G=6, ps=240 (two 16-head windows of pages)
 ]
 
 
@@ -115,6 +118,26 @@ def test_identity_and_shuffled_block_tables_agree(cuda_device):
     _, o1 = _run(inp, cuda_device)
     _, o2 = _run(ident, cuda_device)
     assert torch.equal(o1, o2)
+
+
+@pytest.mark.parametrize("layout", ["v_pool_below_k_pool", "one_pool_for_both"])
+@pytest.mark.parametrize("heads", [(8, 2, 128), (16, 1, 64)], ids=["G4_D128", "G16_D64"])
+def test_pool_placement(cuda_device, layout, heads):
+    """Where the two pools lie in memory does not change the result: V below K in one
+    buffer, and one pool passed as both K and V (attention over V = K)."""
+    H, Hk, D = heads
+    inp = make_custom_inputs([150, 47, 16, 300], H, Hk, D, 16, seed=21)
+    d = inp.to(cuda_device)
+    if layout == "v_pool_below_k_pool":
+        both = torch.stack([d.v_pages, d.k_pages])
+        kp, vp = both[1], both[0]
+        assert vp.data_ptr() < kp.data_ptr()
+    else:
+        kp = vp = d.k_pages
+        inp.v_pages = inp.k_pages
+    out = gq.paged_decode_attn(d.q, kp, vp, d.block_table, d.seq_lens, scale=d.scale)
+    gq.check_device_error()
+    assert_close(gpu_f64(out), oracle_out(host_arrays(inp)), what=layout)
 
 
 def test_nan_in_unread_slots_does_not_leak(cuda_device):

@@ -98,6 +98,8 @@ SMALL_CASES = [
     ([5, 0, 33], 8, 8, 128, 16),                   # MHA (G = 1) and an empty sequence
     ([1000, 3, 500, 2048], 8, 1, 64, 16),          # D = 64 long
     ([700, 90], 8, 1, 128, 256),                   # ps = 256
+    ([700, 47, 96], 16, 4, 128, 48),               # G = 4, ps = 48: blocks straddle pages
+    ([1300, 81], 8, 1, 64, 80),                    # G = 8, D = 64, ps = 80
     # more than 16 query heads per kv head: the tcgen05 kernel with its converter warps
     ([70], 96, 1, 128, 64),                        # MQA, one partial block
     ([1000, 63, 129], 96, 1, 128, 64),             # MQA, several blocks, ragged tails
@@ -160,6 +162,28 @@ def test_fp8_many_short_pieces_in_one_cta(cuda_device, workers):
     want = _oracle_fp8(bf16_bits(inp.q), kc.cpu().numpy(), vc.cpu().numpy(), ks.cpu().numpy(), vs.cpu().numpy(),
                        inp.block_table.numpy(), inp.seq_lens.numpy(), inp.scale)
     assert_close(gpu_f64(out), want, what=f"workers={workers}")
+
+
+@pytest.mark.parametrize("layout", ["v_pool_below_k_pool", "one_pool_for_both"])
+def test_fp8_pool_placement(cuda_device, layout):
+    """Where the two code pools lie in memory does not change the result."""
+    inp = make_custom_inputs([150, 47, 16, 300], 8, 2, 128, 16, seed=22)
+    d = inp.to(cuda_device)
+    kc, vc, ks, vs = _coded(d)
+    if layout == "v_pool_below_k_pool":
+        both = torch.stack([vc, kc])
+        kp, vp = both[1], both[0]
+        assert vp.data_ptr() < kp.data_ptr()
+    else:
+        kp = vp = kc
+        vs = ks
+    out = gq.paged_decode_attn_fp8(d.q, kp, vp, ks, vs, d.block_table, d.seq_lens, scale=d.scale)
+    gq.check_device_error()
+    kcn = kc.cpu().numpy()
+    vcn = kcn if layout == "one_pool_for_both" else vc.cpu().numpy()
+    want = _oracle_fp8(bf16_bits(inp.q), kcn, vcn, ks.cpu().numpy(), vs.cpu().numpy(), inp.block_table.numpy(),
+                       inp.seq_lens.numpy(), inp.scale)
+    assert_close(gpu_f64(out), want, what=layout)
 
 
 def test_fp8_single_token_and_uniform_scores(cuda_device):
