@@ -365,14 +365,16 @@ __device__ __forceinline__ void attend_subchunk_f8(uint32_t kb, uint32_t vb, int
 
 constexpr int kWsCtasPerSm = GQA_CTAS_TOKEN_SPLIT;
 // The 8-bit cache moves half the bytes per stage; its launch shape is set on its own.
-// Three CTAs per SM (3 stages each, 96 registers) measured faster than two (5 stages):
-// 242.5 against 263.6 us on the long-context batch, 320 against 354 us on the
-// continuous batch, 45.8 against 45.2 us on the GQA serving batch.
+// With one copy per sub-chunk for K and V and multiply-shift page arithmetic in the
+// producer, two CTAs per SM (5 stages each) measure faster than three (3 stages, 96
+// registers, spills): 36.2 against 41.5 us on the GQA serving batch, 204 against 215 us
+// on the long-context batch, 284.5 against 281.5 us on the continuous batch.  (Before
+// those producer changes three CTAs were the faster shape.)
 #ifndef GQA_F8_CTAS
-#define GQA_F8_CTAS 3
+#define GQA_F8_CTAS 2
 #endif
 #ifndef GQA_F8_SMEM_PER_SM_KB
-#define GQA_F8_SMEM_PER_SM_KB 220
+#define GQA_F8_SMEM_PER_SM_KB 212
 #endif
 constexpr int kWsCtasPerSmF8 = GQA_F8_CTAS;
 
