@@ -518,6 +518,11 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
   const uint32_t full_bar = ptx::smem_u32(info + S);
   const uint32_t empty_bar = full_bar + 8 * S;
   const uint32_t comb_bar = empty_bar + 8 * S;  // token split: consumers -> epilogue
+  // The epilogue's merged partial of the other pieces of its final segment: [8][D] O then
+  // [8] (max, sum) pairs.
+  float* pre_o = reinterpret_cast<float*>(base_ptr + ((reinterpret_cast<uintptr_t>(info + S) + 24 * S + 15 -
+                                                       reinterpret_cast<uintptr_t>(base_ptr)) & ~uintptr_t{15}));
+  float* pre_ml = pre_o + 8 * D;
 
   const int start_b = s_start_b;
   const int64_t start_base = s_start_base;
@@ -609,7 +614,6 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
     int stage = 0;
     uint32_t phase = 0;  // parity of the current pass over the ring
     int piece_blk0 = cu.blk;
-    bool first_piece = true;
     int64_t seg_base = x0 - cu.blk;
     for (int64_t i = 0; i < total; ++i) {
       if (i >= S) {
@@ -642,7 +646,7 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
         si.rem = cu.len - cu.blk * kBlock;
         si.flags = (first ? kFirstOfPiece : 0) | (last ? kLastOfPiece : 0) |
                    ((last && piece_blk0 == 0 && cu.blk + 1 == cu.nblk) ? kSole : 0) |
-                   (first_piece ? kFirstPieceOfCta : 0);
+                   (seg_base <= x0 ? kFirstPieceOfCta : 0);
         uint32_t bytes = static_cast<uint32_t>(__popc(submask)) * 2u * G_::kSubBytes;
         if (first && !p.arm_without_copy) bytes += q_rows_bytes(cu);
         if (bytes) ptx::mbar_arrive_expect_tx(full_bar + 8 * stage, bytes);
@@ -694,7 +698,6 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
           }
         }
       }
-      if (last) first_piece = false;
       if (++stage == S) {
         stage = 0;
         phase ^= 1u;
@@ -719,9 +722,107 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
     const int hps = p.heads_per_seg;
     int next_len = (cu.b + 1 < B) ? __ldg(p.seq_lens + cu.b + 1) : 0;
     uint32_t comb_phase = 0;  // bit s: parity of the next completion of comb_bar[s]
+    // Rows h0..h0+7 of every piece of a segment except worker skip's, merged (log-sum-exp
+    // over the pieces' (max, sum) pairs); loads batched per piece.
+    auto merge_pieces = [&](int64_t sbase, int64_t wf, int64_t wl, int64_t skip, int h0, int nrows,
+                            float (&M)[8], float (&L)[8], float (&acc)[8][CPL]) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        M[k] = -INFINITY;
+        L[k] = 0.f;
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) acc[k][c] = 0.f;
+      }
+      for (int64_t ww = wf; ww <= wl; ++ww) {
+        if (ww == skip) continue;
+        const int64_t sl = piece_slot(ww, sbase, T, W);
+        float2 mlv[8];
+        float v[8][CPL];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int h = min(h0 + k, nrows - 1);
+          mlv[k] = __ldcg(reinterpret_cast<const float2*>(p.part_ml + (sl * hps + h) * 2));
+          const float* src = p.part_o + (sl * hps + h) * D + d0;
+          if constexpr (CPL == 4) {
+            const float4 t4 = __ldcg(reinterpret_cast<const float4*>(src));
+            v[k][0] = t4.x; v[k][1] = t4.y; v[k][2] = t4.z; v[k][3] = t4.w;
+          } else {
+            const float2 t2 = __ldcg(reinterpret_cast<const float2*>(src));
+            v[k][0] = t2.x; v[k][1] = t2.y;
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const float mn = fmaxf(M[k], mlv[k].x);
+          const float mu = (mn == -INFINITY) ? 0.f : mn;
+          const float a = ptx::ex2(M[k] - mu), bw = ptx::ex2(mlv[k].x - mu);
+          L[k] = L[k] * a + mlv[k].y * bw;
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) acc[k][c] = acc[k][c] * a + v[k][c] * bw;
+          M[k] = mn;
+        }
+      }
+    };
+    // Normalised bf16 row of out.
+    auto store_row = [&](int b, int kvh, int row, float L, const float (&acc)[CPL]) {
+      const float inv = L > 0.f ? 1.f / L : 0.f;
+      uint16_t* dst = p.out + seq_row(b, kvh, row) * D + d0;
+      if constexpr (CPL == 4) {
+        uint2 u;
+        u.x = ptx::pack_bf16x2(acc[0] * inv, acc[1] * inv);
+        u.y = ptx::pack_bf16x2(acc[2] * inv, acc[3] * inv);
+        *reinterpret_cast<uint2*>(dst) = u;
+      } else {
+        *reinterpret_cast<uint32_t*>(dst) = ptx::pack_bf16x2(acc[0] * inv, acc[1] * inv);
+      }
+    };
+    // Arrival count of a segment's pieces (relaxed; a fence follows a count that shows
+    // every other piece published, pairing with the publishers' fence before their add).
+    auto arrivals = [&](int64_t segid) -> int { return lane == 0 ? ptx::ld_relaxed_gpu(p.counters + segid) : 0; };
+    // The range's final piece, when cut, ends the CTA: if the segment's other pieces are
+    // all published by then (they usually finished long before), their merged partial is
+    // loaded while the consumers finish this one, and this CTA writes out without
+    // publishing its own piece (no store, fence and arrival round trip, no reload).  The
+    // count is read once on reaching the piece end and, if short, once more with the read
+    // in flight during the wait for the consumers.
+    bool pre = false;
+    int late = 0;  // the second read
+    // Merge the other pieces into the shared buffer (each lane its columns; the (max, sum)
+    // pairs, equal in every lane, from lane 0).
+    auto prefetch_others = [&](int64_t sbase, int64_t wf, int64_t wl, int nrows) {
+      __threadfence();
+      float M[8], L[8], acc[8][CPL];
+      merge_pieces(sbase, wf, wl, w, 0, nrows, M, L, acc);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) pre_o[k * D + d0 + c] = acc[k][c];
+        if (lane == 0) {
+          pre_ml[2 * k] = M[k];
+          pre_ml[2 * k + 1] = L[k];
+        }
+      }
+      __syncwarp();
+    };
+    int64_t seg_base = x0 - cu.blk;  // linear index of block 0 of the current block's segment
+    int e_blk0 = cu.blk;
     for (int64_t i = 0; i < total; ++i) {
+      if (i == 0 || cu.blk == 0) e_blk0 = cu.blk;
       if ((cu.blk + 1 == cu.nblk) || (i + 1 == total)) {
         const int stage = static_cast<int>(i % S);
+        // (the walk's block is the stage's: this piece's segment from the cursor)
+        const bool final_cut = NT == 1 && (i + 1 == total) && !(e_blk0 == 0 && cu.blk + 1 == cu.nblk);
+        if (final_cut) {
+          const int64_t sb = seg_base;
+          const int64_t wf = worker_of(sb, T, W), wl = worker_of(sb + cu.nblk - 1, T, W);
+          const int64_t sid = static_cast<int64_t>(cu.b) * segs + cu.seg;
+          if (__shfl_sync(0xffffffffu, arrivals(sid), 0) == static_cast<int>(wl - wf)) {
+            pre = true;
+            prefetch_others(sb, wf, wl, min(hps, grp - cu.ht * hps));
+          } else {
+            late = arrivals(sid);  // consumed after the wait
+          }
+        }
         const bool ok = ptx::mbar_wait_bounded(comb_bar + 8 * stage, (comb_phase >> stage) & 1u, limit);
         comb_phase ^= 1u << stage;
         if (!__all_sync(0xffffffffu, ok)) {
@@ -736,9 +837,11 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
         const bool sole = si.flags & kSole;
         const float vscale = F8 ? __ldg(p.v_scales + kvh) : 1.f;
         const int64_t slot = w * 2 + ((si.flags & kFirstPieceOfCta) ? 0 : 1);
-        for (int h = 0; h < nrows; ++h) {
+        // This piece's row h: the C consumers' states combined (max M, sum L, O acc).
+        auto combine = [&](int h, float& M, float& L, float (&acc)[CPL]) {
           float mj[C], wj[C];
-          float M = -INFINITY, L = 0.f;
+          M = -INFINITY;
+          L = 0.f;
 #pragma unroll
           for (int jj = 0; jj < C; ++jj) {
             mj[jj] = ml[(jj * NH + h) * 2];
@@ -749,7 +852,6 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
             wj[jj] = (mj[jj] == -INFINITY) ? 0.f : ptx::ex2(mj[jj] - M);
             L += wj[jj] * ml[(jj * NH + h) * 2 + 1];
           }
-          float acc[CPL];
 #pragma unroll
           for (int c = 0; c < CPL; ++c) acc[c] = 0.f;
 #pragma unroll
@@ -763,17 +865,41 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
 #pragma unroll
             for (int c = 0; c < CPL; ++c) acc[c] *= vscale;
           }
-          if (sole) {
-            const float inv = L > 0.f ? 1.f / L : 0.f;
-            uint16_t* dst = p.out + seq_row(si.b, kvh, ht * hps + h) * D + d0;
-            if constexpr (CPL == 4) {
-              uint2 v;
-              v.x = ptx::pack_bf16x2(acc[0] * inv, acc[1] * inv);
-              v.y = ptx::pack_bf16x2(acc[2] * inv, acc[3] * inv);
-              *reinterpret_cast<uint2*>(dst) = v;
-            } else {
-              *reinterpret_cast<uint32_t*>(dst) = ptx::pack_bf16x2(acc[0] * inv, acc[1] * inv);
+        };
+        const int64_t segid = static_cast<int64_t>(si.b) * segs + si.seg;
+        if (final_cut && !sole) {
+          const int64_t wf = worker_of(si.seg_base, T, W), wl = worker_of(si.seg_base + si.nblk - 1, T, W);
+          if (!pre && __shfl_sync(0xffffffffu, late, 0) == static_cast<int>(wl - wf)) {
+            pre = true;
+            prefetch_others(si.seg_base, wf, wl, nrows);
+          }
+          if (pre) {
+            for (int h = 0; h < nrows; ++h) {
+              float M, L, acc[CPL];
+              combine(h, M, L, acc);
+              const float pm = pre_ml[2 * h], pl = pre_ml[2 * h + 1];
+              const float mn = fmaxf(M, pm);
+              const float mu = (mn == -INFINITY) ? 0.f : mn;
+              const float a = ptx::ex2(M - mu), bw = ptx::ex2(pm - mu);
+              L = L * a + pl * bw;
+#pragma unroll
+              for (int c = 0; c < CPL; ++c) acc[c] = acc[c] * a + pre_o[h * D + d0 + c] * bw;
+              store_row(si.b, kvh, ht * hps + h, L, acc);
             }
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              ptx::mbar_arrive_cnt(empty_bar + 8 * stage, C);
+              p.counters[segid] = 0;  // every other piece has arrived: ready for the next launch
+            }
+            continue;  // the range's last block
+          }
+        }
+        for (int h = 0; h < nrows; ++h) {
+          float M, L, acc[CPL];
+          combine(h, M, L, acc);
+          if (sole) {
+            store_row(si.b, kvh, ht * hps + h, L, acc);
           } else {
             float* dst = p.part_o + (slot * hps + h) * D + d0;
 #pragma unroll
@@ -791,7 +917,6 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
           // Cross-CTA step: the last CTA to finish its piece merges every piece.
           __threadfence();
           __syncwarp();
-          const int64_t segid = static_cast<int64_t>(si.b) * segs + si.seg;
           int prev = 0;
           if (lane == 0) prev = atomicAdd(p.counters + segid, 1);
           prev = __shfl_sync(0xffffffffu, prev, 0);
@@ -801,62 +926,19 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
             __threadfence();
             for (int h0 = 0; h0 < nrows; h0 += 8) {
               float M[8], L[8], acc[8][CPL];
+              merge_pieces(si.seg_base, wf, wl, -1, h0, nrows, M, L, acc);
 #pragma unroll
-              for (int k = 0; k < 8; ++k) {
-                M[k] = -INFINITY;
-                L[k] = 0.f;
-#pragma unroll
-                for (int c = 0; c < CPL; ++c) acc[k][c] = 0.f;
-              }
-              for (int64_t ww = wf; ww <= wl; ++ww) {
-                const int64_t sl = piece_slot(ww, si.seg_base, T, W);
-                float2 mlv[8];
-                float v[8][CPL];
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                  const int h = min(h0 + k, nrows - 1);
-                  mlv[k] = __ldcg(reinterpret_cast<const float2*>(p.part_ml + (sl * hps + h) * 2));
-                  const float* src = p.part_o + (sl * hps + h) * D + d0;
-                  if constexpr (CPL == 4) {
-                    const float4 t4 = __ldcg(reinterpret_cast<const float4*>(src));
-                    v[k][0] = t4.x; v[k][1] = t4.y; v[k][2] = t4.z; v[k][3] = t4.w;
-                  } else {
-                    const float2 t2 = __ldcg(reinterpret_cast<const float2*>(src));
-                    v[k][0] = t2.x; v[k][1] = t2.y;
-                  }
-                }
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                  const float mn = fmaxf(M[k], mlv[k].x);
-                  const float mu = (mn == -INFINITY) ? 0.f : mn;
-                  const float a = ptx::ex2(M[k] - mu), bw = ptx::ex2(mlv[k].x - mu);
-                  L[k] = L[k] * a + mlv[k].y * bw;
-#pragma unroll
-                  for (int c = 0; c < CPL; ++c) acc[k][c] = acc[k][c] * a + v[k][c] * bw;
-                  M[k] = mn;
-                }
-              }
-#pragma unroll
-              for (int k = 0; k < 8; ++k) {
-                if (h0 + k < nrows) {
-                  const float inv = L[k] > 0.f ? 1.f / L[k] : 0.f;
-                  uint16_t* dst = p.out + seq_row(si.b, kvh, ht * hps + h0 + k) * D + d0;
-                  if constexpr (CPL == 4) {
-                    uint2 u;
-                    u.x = ptx::pack_bf16x2(acc[k][0] * inv, acc[k][1] * inv);
-                    u.y = ptx::pack_bf16x2(acc[k][2] * inv, acc[k][3] * inv);
-                    *reinterpret_cast<uint2*>(dst) = u;
-                  } else {
-                    *reinterpret_cast<uint32_t*>(dst) = ptx::pack_bf16x2(acc[k][0] * inv, acc[k][1] * inv);
-                  }
-                }
-              }
+              for (int k = 0; k < 8; ++k)
+                if (h0 + k < nrows) store_row(si.b, kvh, ht * hps + h0 + k, L[k], acc[k]);
             }
             if (lane == 0) p.counters[segid] = 0;
           }
         }
       }
-      if (i + 1 < total) walk_next(cu, next_len, p, segs, cap);
+      if (i + 1 < total) {
+        walk_next(cu, next_len, p, segs, cap);
+        if (cu.blk == 0) seg_base = x0 + i + 1;
+      }
     }
     return;
   }
@@ -1050,8 +1132,11 @@ struct Cfg {
   static constexpr int kStagesRaw =
       static_cast<int>((kBudget - kMerge) / (Geo<D, F8>::kStageBytes + kQBytes));
   static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+  // the epilogue's merged partial of the other pieces of its final segment ([8][D] O and
+  // 8 (max, sum) pairs, 16-byte aligned), outside the stage budget
+  static constexpr size_t kPre = (8 * D + 16) * sizeof(float) + 16;
   static constexpr size_t kSmem = 1024 + static_cast<size_t>(kStages) * (Geo<D, F8>::kStageBytes + kQBytes) +
-                                  kMerge + kStages * (sizeof(StageInfo) + 24);
+                                  kMerge + kStages * (sizeof(StageInfo) + 24) + kPre;
 };
 
 template <int D, int NT, int C, bool MQ, bool F8 = false>

@@ -120,6 +120,13 @@ __device__ __forceinline__ bool wait_counter(const volatile int* c, int v, uint6
   return true;
 }
 
+// Relaxed load at GPU scope (a fence after it, when the value says so, gives acquire).
+__device__ __forceinline__ int ld_relaxed_gpu(const int* p) {
+  int v;
+  asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 // Programmatic dependent launch: let the next kernel in the stream (launched with the
 // programmatic-serialization attribute) start its prologue now; and, in that kernel,
 // wait until the preceding grid has completed and its writes are visible.
