@@ -239,17 +239,18 @@ __device__ __forceinline__ void attend_subchunk(uint32_t kb, uint32_t vb, int nv
 }
 
 // The same sub-chunk over an e4m3 cache, on fp16 MMAs (e4m3 -> fp16 is exact; q is
-// converted to fp16 when its fragments are loaded, P is packed as fp16).  One 16-byte
+// converted to fp16 when its fragments are loaded, P is packed as fp16).  K: one 16-byte
 // ldmatrix row is 16 head-dim values of one token, so thread (g, q) receives values
-// 4q .. 4q + 3 of a 16-value chunk: the contraction over head_dim uses that order for
-// K (the q fragments follow it), and for V^T each converted pair is transposed with
-// movmatrix, which puts dimension 16 mt + 4 (g >> 1) + (g & 1) (+ 2 for row g + 8) on
-// M-row g of O^T tile mt.  (V^T from the transposing ldmatrix with one byte permute per
-// register instead -- fewer instructions -- measured slower: 270.5 against 262.6 us on
-// the long-context batch.)
+// 4q .. 4q + 3 of a 16-value chunk, and the contraction over head_dim uses that order
+// (the q fragments follow it).  V^T comes from the transposing byte ldmatrix (16 x 16
+// codes per matrix), whose lane (g, q) receives tokens 2q, 2q+1, 2q+8, 2q+9 of dims g and
+// g + 8: widened, that is the mma A fragment of V^T as it stands (1.8-3.1 % faster than
+// widening row-major codes and transposing each pair with movmatrix; the transposing
+// 16-bit ldmatrix with one byte permute per register measured slower than both).
 template <int D, int NT>
 __device__ __forceinline__ void attend_subchunk_f8(uint32_t kb, uint32_t vb, int nvalid,
-                                                   const uint32_t (&ofs)[D / 32], const uint32_t (&qf)[D / 16][NT][2],
+                                                   const uint32_t (&ofs)[D / 32], const uint32_t (&vofs)[D / 32],
+                                                   const uint32_t (&qf)[D / 16][NT][2],
                                                    float (&o)[D / 16][NT][4], float (&mref)[NT][2],
                                                    float (&lsum)[NT][2], float sl2, int g, int q) {
   constexpr int MT = D / 16;
@@ -337,14 +338,16 @@ __device__ __forceinline__ void attend_subchunk_f8(uint32_t kb, uint32_t vb, int
 #pragma unroll
   for (int vx = 0; vx < D / 32; ++vx) {
     uint32_t r[4];
-    ptx::ldmatrix_x4(vb + ofs[vx], r[0], r[1], r[2], r[3]);
+    // V^T straight from the transposing byte ldmatrix: r[2h] holds dim 16(2vx+h) + g and
+    // r[2h+1] dim 16(2vx+h) + g + 8, tokens 2q, 2q+1, 2q+8, 2q+9 in bytes 0..3
+    ptx::ldmatrix_m16n16_x2_trans_b8(vb + vofs[vx], r[0], r[1], r[2], r[3]);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {  // O^T tile mt = 2 vx + h
       uint32_t a[4];
-      a[0] = ptx::movmatrix_trans(ptx::e4m3x2_lo(r[2 * h])) & vm0;      // dims d(g), tokens 2q, 2q+1
-      a[1] = ptx::movmatrix_trans(ptx::e4m3x2_hi(r[2 * h])) & vm0;      // dims d(g) + 2
-      a[2] = ptx::movmatrix_trans(ptx::e4m3x2_lo(r[2 * h + 1])) & vm1;  // dims d(g), tokens 8 + 2q, ..
-      a[3] = ptx::movmatrix_trans(ptx::e4m3x2_hi(r[2 * h + 1])) & vm1;
+      a[0] = ptx::e4m3x2_lo(r[2 * h]) & vm0;      // dim g, tokens 2q, 2q+1
+      a[1] = ptx::e4m3x2_lo(r[2 * h + 1]) & vm0;  // dim g + 8
+      a[2] = ptx::e4m3x2_hi(r[2 * h]) & vm1;      // dim g, tokens 2q+8, 2q+9
+      a[3] = ptx::e4m3x2_hi(r[2 * h + 1]) & vm1;
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) ptx::mma_f16_16816(o[2 * vx + h][nt], a, pb[nt][0], pb[nt][1]);
     }
@@ -950,8 +953,22 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
   const int g = lane >> 2;
   const int q = lane & 3;
   uint32_t kofs[4], vofs[4];
-  uint32_t ofs8[D / 32];  // F8: ldmatrix row addresses, K and V alike
+  uint32_t ofs8[D / 32];   // F8: ldmatrix row addresses of K
+  uint32_t vofs8[D / 32];  // F8: transposing byte ldmatrix row addresses of V
   if constexpr (F8) {
+    // lane 16 m + j addresses token (j & 1) + 8 ((j >> 1) & 1) + 2 (j >> 2), 16-value chunk
+    // 2 x + m, so that lane (g, q) receives tokens 2q, 2q+1, 2q+8, 2q+9
+    {
+      const int j = lane & 15;
+      const int tok = (j & 1) + 8 * ((j >> 1) & 1) + 2 * (j >> 2);
+#pragma unroll
+      for (int x = 0; x < D / 32; ++x) {
+        const int chunk = 2 * x + (lane >> 4);
+        const int row = tok / (128 / D);
+        const int c = (tok % (128 / D)) * (D / 16) + chunk;
+        vofs8[x] = static_cast<uint32_t>(row * 128 + ((c ^ (row & 7)) << 4));
+      }
+    }
     // lane l addresses row l % 8 of matrix l / 8: token (l % 8) + 8 ((l / 8) & 1), 16-value
     // chunk 2 x + (l / 16) of the x-th 32 values; a token's D codes are D / 128 of a
     // 128-byte swizzled row
@@ -1042,7 +1059,7 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
       const uint32_t sub = ring + stage * G_::kStageBytes + j * 2 * G_::kSubBytes;
       const uint32_t kb = sub + koff, vb = sub + (G_::kSubBytes - koff);
       if constexpr (F8)
-        attend_subchunk_f8<D, NT>(kb, vb, min(kChunk, si.nvalid - j * kChunk), ofs8, qf, o, mref,
+        attend_subchunk_f8<D, NT>(kb, vb, min(kChunk, si.nvalid - j * kChunk), ofs8, vofs8, qf, o, mref,
                                   lsum, sl2, g, q);
       else
         attend_subchunk<D, NT, MQ>(kb, vb, min(kChunk, si.nvalid - j * kChunk),
@@ -1091,11 +1108,7 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
           }
       }
       // Head h of this consumer goes to the first tile of its sub-chunk (h < HS) or the
-      // second.
-      // O^T M-row g of tile mt is dimension 16 mt + g (bf16; row g + 8: 16 mt + g + 8),
-      // with the 8-bit cache 16 mt + dg (row g + 8: 16 mt + dg + d8).
-      const int dg = F8 ? 4 * (g >> 1) + (g & 1) : g;
-      constexpr int d8 = F8 ? 2 : 8;
+      // second.  O^T M-row g of tile mt is dimension 16 mt + g (row g + 8: 16 mt + g + 8).
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
@@ -1105,8 +1118,8 @@ decode_ws_kernel(const __grid_constant__ CUtensorMap tmap_k,
                                                 (h >= HS ? G_::kSubBytes : 0)) + (h % HS) * D;
 #pragma unroll
           for (int mt = 0; mt < MT; ++mt) {
-            row[mt * 16 + dg] = o[mt][nt][e];
-            row[mt * 16 + dg + d8] = o[mt][nt][e + 2];
+            row[mt * 16 + g] = o[mt][nt][e];
+            row[mt * 16 + g + 8] = o[mt][nt][e + 2];
           }
         }
       }

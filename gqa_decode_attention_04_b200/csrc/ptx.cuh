@@ -308,6 +308,17 @@ __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t& r0, u
 
 // Transpose an 8x8 matrix of 16-bit elements held one row-pair per thread
 // (thread t: row t/4, columns 2(t%4), 2(t%4)+1) into the same layout.
+// Two 16 x 16 byte matrices, transposed (sm_100a): lanes 16 m + j (j < 16) give the shared
+// address of 16-byte row j of matrix m; lane (g, q) = (lane / 4, lane % 4) receives, of
+// matrix 0, rows 4q .. 4q + 3 of column g in r0 and of column g + 8 in r1 (row 4q + u in
+// byte u), and the same of matrix 1 in r2, r3.
+__device__ __forceinline__ void ldmatrix_m16n16_x2_trans_b8(uint32_t addr, uint32_t& r0, uint32_t& r1,
+                                                            uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m16n16.x2.trans.shared.b8 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
 __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
   uint32_t d;
   asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
