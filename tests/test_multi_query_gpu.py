@@ -55,9 +55,12 @@ def test_multi_query_parity(cuda_device, case):
     assert_close(gpu_f64(out), _oracle(inp, q), what=str(case))
 
 
-@pytest.mark.parametrize("rows", [16, 64])
+@pytest.mark.parametrize("rows", [8, 16, 64])
 @pytest.mark.parametrize("workers", [1, 3, 57, 400])
 def test_multi_query_forced_splits(cuda_device, workers, rows):
+    """8 rows per kv head run on the one-n-tile mma.sync kernel, whose CTAs finish a cut
+    final piece by merging the segment's other pieces directly; 16 on two n-tiles; 64 on
+    tcgen05 with the merge kernel."""
     lens, Q, H, Hk, D, ps = [900, 333, 64, 2], rows // 4, 8, 2, 128, 16
     inp, q = _case(lens, Q, H, Hk, D, ps, seed=5)
     d = inp.to(cuda_device)
