@@ -46,7 +46,7 @@ import torch.distributed as dist
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from workloads import WORKLOADS, make_inputs, bf16_bits  # noqa: E402
+from workloads import WORKLOADS, make_inputs, make_shrunk_inputs, bf16_bits  # noqa: E402
 
 METRIC = "paged GQA decode attn: achieved HBM TB/s (% of B200 peak), tokens/s"
 FALLBACK_HBM_GBS = 6650.0
@@ -853,7 +853,12 @@ def run_profile(args):
     import gqa_decode_attention_04_b200 as gq
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    inp = make_inputs(args.workload, seed=1000 + args.workload, device=dev, poison=False)
+    if args.profile_shrink > 1:  # the same kernel on a smaller case (context lengths / N)
+        inp = make_shrunk_inputs(args.workload, args.profile_shrink, seed=1000 + args.workload, device=dev,
+                                 poison=False)
+    else:
+        inp = make_inputs(args.workload, seed=1000 + args.workload, device=dev, poison=False)
+    print(f"context tokens per launch: {int(inp.seq_lens.to(torch.int64).sum())}", flush=True)
     sets, _ = _pool_sets(inp, dev)
     sets = sets[:2]
     out = torch.empty((inp.num_seqs, inp.num_heads, inp.head_dim), dtype=torch.bfloat16, device=dev)
@@ -892,6 +897,8 @@ def main():
     ap.add_argument("--headline-only", action="store_true", help="skip the other workloads")
     ap.add_argument("--profile", choices=["bf16", "fp8"],
                     help="only run --warmup + --steps decode launches of --workload (ncu captures)")
+    ap.add_argument("--profile-shrink", type=int, default=1,
+                    help="with --profile: divide every context length by N (a smaller case of the same kernel)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

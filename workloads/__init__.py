@@ -36,6 +36,7 @@ __all__ = [
     "PagedDecodeInputs",
     "make_inputs",
     "make_custom_inputs",
+    "make_shrunk_inputs",
     "bf16_bits",
 ]
 
@@ -254,6 +255,24 @@ def make_inputs(index: int, seed: Optional[int] = None, device="cpu",
                  poison=poison, append=(index == 5),
                  spike_fraction=0.01 if index == 4 else 0.0)
     inp.meta["workload"] = index
+    return inp
+
+
+def make_shrunk_inputs(index: int, shrink: int, seed: Optional[int] = None, device="cpu",
+                       poison: bool = True) -> PagedDecodeInputs:
+    """Workload `index` with every context length divided by `shrink` (rounded up): the
+    same shapes, page size, length recipe and spike fraction on fewer tokens, for
+    profiler captures of a smaller case of the same kernel."""
+    spec = WORKLOADS[index]
+    if seed is None:
+        seed = 1000 + index
+    lens = _seq_lens_for(spec, torch.Generator().manual_seed(seed))
+    lens = [(int(L) + shrink - 1) // shrink for L in lens.tolist()]
+    inp = make_custom_inputs(lens, spec.num_heads, spec.num_kv_heads, spec.head_dim, spec.page_size,
+                             seed=seed, device=device, poison=poison,
+                             spike_fraction=0.01 if index == 4 else 0.0)
+    inp.meta["workload"] = index
+    inp.meta["shrink"] = shrink
     return inp
 
 
