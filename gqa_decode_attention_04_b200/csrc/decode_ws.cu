@@ -363,7 +363,7 @@ __device__ __forceinline__ void attend_subchunk_f8(uint32_t kb, uint32_t vb, int
 #define GQA_CTAS_TOKEN_SPLIT 2
 #endif
 #ifndef GQA_SMEM_PER_SM_KB
-#define GQA_SMEM_PER_SM_KB 212
+#define GQA_SMEM_PER_SM_KB 220
 #endif
 
 constexpr int kWsCtasPerSm = GQA_CTAS_TOKEN_SPLIT;
@@ -1137,17 +1137,18 @@ namespace {
 template <int D, int NT, int C, bool F8 = false>
 struct Cfg {
   static constexpr int kNH = 8 * NT;
-  // per-stage (max, sum) hand-off area, sized for up to 8 stages
-  static constexpr size_t kMerge = static_cast<size_t>(8 * C * kNH * 2) * sizeof(float);
+  // per stage: K/V tiles, the piece's query rows, the consumers' (max, sum) hand-off
+  static constexpr size_t kQBytes = static_cast<size_t>(kNH) * D * 2;
+  static constexpr size_t kMergePerStage = static_cast<size_t>(C * kNH * 2) * sizeof(float);
   static constexpr size_t kBudget = F8 ? static_cast<size_t>(GQA_F8_SMEM_PER_SM_KB) * 1024 / kWsCtasPerSmF8
                                       : static_cast<size_t>(GQA_SMEM_PER_SM_KB) * 1024 / kWsCtasPerSm;
-  static constexpr size_t kQBytes = static_cast<size_t>(kNH) * D * 2;
   static constexpr int kStagesRaw =
-      static_cast<int>((kBudget - kMerge) / (Geo<D, F8>::kStageBytes + kQBytes));
+      static_cast<int>(kBudget / (Geo<D, F8>::kStageBytes + kQBytes + kMergePerStage));
   static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
-  // the epilogue's merged partial of the other pieces of its final segment ([8][D] O and
-  // 8 (max, sum) pairs, 16-byte aligned), outside the stage budget
-  static constexpr size_t kPre = (8 * D + 16) * sizeof(float) + 16;
+  static constexpr size_t kMerge = kStages * kMergePerStage;
+  // one n-tile: the epilogue's merged partial of the other pieces of its final segment
+  // ([8][D] O and 8 (max, sum) pairs, 16-byte aligned), outside the stage budget
+  static constexpr size_t kPre = NT == 1 ? (8 * D + 16) * sizeof(float) + 16 : 0;
   static constexpr size_t kSmem = 1024 + static_cast<size_t>(kStages) * (Geo<D, F8>::kStageBytes + kQBytes) +
                                   kMerge + kStages * (sizeof(StageInfo) + 24) + kPre;
 };
