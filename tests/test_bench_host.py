@@ -83,3 +83,16 @@ def test_measured_peak_is_the_copy_rate_or_the_fallback(tmp_path, monkeypatch):
     assert bench.measured_peak() == (bench.FALLBACK_HBM_GBS, "fallback")
     (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 6554.6}))
     assert bench.measured_peak() == (6554.6, "measured")
+
+
+@pytest.mark.parametrize("index,shrink", [(4, 256), (5, 64), (2, 8)])
+def test_shrunk_workload_keeps_shapes_and_divides_every_length(index, shrink):
+    """The smaller case the profiler captures of a workload: same shapes, page size and
+    seeded length recipe, every context length divided by N (rounded up)."""
+    from workloads import WORKLOADS, _seq_lens_for, make_shrunk_inputs
+    spec = WORKLOADS[index]
+    small = make_shrunk_inputs(index, shrink, seed=1000 + index, poison=False)
+    full = _seq_lens_for(spec, torch.Generator().manual_seed(1000 + index)).tolist()
+    assert small.seq_lens.tolist() == [(L + shrink - 1) // shrink for L in full]
+    assert (small.num_seqs, small.num_heads, small.num_kv_heads, small.head_dim, small.page_size) == (
+        spec.num_seqs, spec.num_heads, spec.num_kv_heads, spec.head_dim, spec.page_size)
