@@ -445,3 +445,18 @@ def test_large_group_many_short_pieces_in_one_cta(cuda_device, workers):
     gq.set_num_workers(workers)
     d, out = _run(inp, cuda_device)
     assert_close(gpu_f64(out), oracle_out(host_arrays(inp)), what=f"workers={workers}")
+
+
+@pytest.mark.parametrize("heads", [(8, 2), (96, 1)], ids=["mma_sync", "tcgen05"])
+@pytest.mark.parametrize("workers", [0, 5])
+def test_every_sequence_empty_gives_zeros(cuda_device, heads, workers):
+    """No block of work at all: every CTA returns after zeroing its share of the empty
+    sequences' rows (out starts as NaN, so a row left unwritten fails)."""
+    H, Hk = heads
+    inp = make_custom_inputs([0, 0, 0], H, Hk, 128, 16, seed=31, extra_pages=2)
+    d = inp.to(cuda_device)
+    out = torch.full((3, H, 128), float("nan"), dtype=torch.bfloat16, device=cuda_device)
+    gq.set_num_workers(workers)
+    gq.paged_decode_attn(d.q, d.k_pages, d.v_pages, d.block_table, d.seq_lens, out=out, scale=d.scale)
+    gq.check_device_error()
+    assert torch.count_nonzero(out) == 0

@@ -298,3 +298,16 @@ def test_fp8_workload_parity(cuda_device, index):
         want = oracle.paged_decode_attention_fp8_rows(q, kcn, vcn, ksn, vsn, bt, sl, inp.scale, rows)
         mx, mean = assert_close(got, want, what=inp.name)
     print(f"{inp.name} fp8: max abs {mx:.2e} mean abs {mean:.2e}")
+
+
+@pytest.mark.parametrize("heads", [(8, 2), (96, 1)], ids=["mma_sync", "tcgen05"])
+def test_fp8_every_sequence_empty_gives_zeros(cuda_device, heads):
+    """No block of work at all over an e4m3 cache: the output rows are exact zeros."""
+    H, Hk = heads
+    inp = make_custom_inputs([0, 0, 0], H, Hk, 128, 16, seed=32, extra_pages=2)
+    d = inp.to(cuda_device)
+    kc, vc, ks, vs = _coded(d)
+    out = torch.full((3, H, 128), float("nan"), dtype=torch.bfloat16, device=cuda_device)
+    gq.paged_decode_attn_fp8(d.q, kc, vc, ks, vs, d.block_table, d.seq_lens, out=out, scale=d.scale)
+    gq.check_device_error()
+    assert torch.count_nonzero(out) == 0
